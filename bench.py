@@ -1,0 +1,469 @@
+#!/usr/bin/env python3
+"""Benchmark of the gated delta-rule layer on B200.
+
+One step = one pass of the layer's prefill hot path over one synthetic batch:
+causal conv k=4 + SiLU + q/k L2 (gdn_conv1d_silu) -> chunk-64 gated delta
+rule (gdn_chunked_prefill) -> gated RMS-norm (gdn_gated_rmsnorm), on the
+prefill workload B=1, T=8192, 16 key / 48 value heads, head dim 128, bf16
+activations, fp32 gates and state. The decode workload (256 sequences, one
+token per step: conv with in-place cache roll -> gdn_decode_step -> gated
+RMS-norm, fp32 state [256,48,128,128]) is timed in the same run and reported
+under "decode".
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+With N > 1 (launched by torch.distributed.run) every rank runs its own
+replica of the workload on its own synthetic data -- the layer shards by
+sequence with no exchange -- and the slowest rank's time is reported
+("scaling": "weak"). `--impl reference` times the fp64 CPU oracle on the
+host cores on a bounded sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import gdn_inputs as gi  # noqa: E402
+
+METRIC = "gated-delta-rule prefill tokens/s and decode tokens/s per layer; % of roofline"
+T_PREFILL = 8192
+N_DECODE = 256
+H_K, H_V, D, C = 16, 48, 128, 64
+# Algorithmic work per token, one layer, chunk C=64: 6d^2 (W S^T, Q S^T, U^T K)
+# + 6Cd (W, U, M U) + 4Cd/3 (K K^T, Q K^T shared by 3 value heads) + C^2/1.5
+# (triangular solve), for each of the 48 value heads.
+PREFILL_FLOP_PER_TOKEN = 48 * (6 * D * D + 6 * C * D + 4 * C * D / 3 + C * C / 1.5)
+# bf16 q,k,v,o + fp32 g,beta per token
+PREFILL_BYTES_PER_TOKEN = 2 * (2 * H_K * D) + 2 * H_V * D + 2 * 4 * H_V + 2 * H_V * D
+# decode: fp32 state read + write, plus q,k (bf16), v, o (bf16), g, beta (bf16)
+DECODE_BYTES_PER_TOKEN = 2 * H_V * D * D * 4 + 2 * (2 * H_K * D) + 2 * 2 * H_V * D + 2 * 2 * H_V
+L2_FLUSH_BYTES = 256 << 20
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+def kernel_traffic(kernel):
+    """DRAM bytes per launch from the committed ncu summary, or None when the
+    kernel's source changed since the counters were taken."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f).get(kernel)
+    if not d:
+        return None
+    src = os.path.join(ROOT, d["source"])
+    if not os.path.exists(src):
+        return None
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    return d["bytes_per_launch"] if h == d["source_sha256_16"] else None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples taken while the timed loop
+    runs (50 ms period)."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        rows = []
+        for line in (self.out or "").splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                rows.append((float(f[1]), float(f[2]), f[4:8]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r)
+                          if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- GPU arm --
+
+class PrefillWorkload:
+    """Device-resident buffers of the prefill workload and one step over it."""
+
+    def __init__(self, gdn, dev, seed):
+        self.gdn = gdn
+        p = gi.prefill_inputs(T=T_PREFILL, seed=seed)
+        self.host = p
+        self.x = p["x_pre"].to(dev)
+        self.w = p["conv_w"].to(dev)
+        self.g = p["g"].to(dev)
+        self.b = p["beta"].to(dev)
+        self.z = p["z"].to(dev)
+        self.nw = p["norm_w"].to(dev)
+        self.cu = p["cu_seqlens"].to(dev)
+        self.y = torch.empty_like(self.x)
+        self.o = torch.empty((T_PREFILL, H_V, D), dtype=torch.bfloat16, device=dev)
+        self.out = torch.empty_like(self.o)
+        self.state = torch.empty((1, H_V, D, D), dtype=torch.float32, device=dev)
+        self.launches_per_step = 3
+
+    def step(self, ev=None):
+        g = self.gdn
+        g.gdn_conv1d_silu(self.x, self.w, self.cu, y=self.y)
+        if ev is not None:
+            ev[0].record()
+        y = self.y
+        g.gdn_chunked_prefill(y[:, :2048].view(-1, H_K, D), y[:, 2048:4096].view(-1, H_K, D),
+                              y[:, 4096:].view(-1, H_V, D), self.g, self.b, self.cu,
+                              state_out=self.state, o=self.o)
+        if ev is not None:
+            ev[1].record()
+        g.gdn_gated_rmsnorm(self.o, self.z, self.nw, eps=1e-6, y=self.out)
+
+
+class DecodeWorkload:
+    def __init__(self, gdn, dev, seed, steps):
+        self.gdn = gdn
+        init = gi.decode_initial(N_DECODE, seed)
+        self.state = init["state"].to(dev)
+        self.cache = init["conv_state"].to(dev)
+        self.w = gi.conv_weight(seed).to(dev)
+        self.nw = torch.ones(D, device=dev)
+        self.cu = torch.arange(N_DECODE + 1, dtype=torch.int32, device=dev)
+        self.inputs = []
+        for s in range(steps):
+            st = gi.decode_step_inputs(s, N_DECODE, seed)
+            self.inputs.append({k: v.to(dev) for k, v in st.items()})
+        self.y = torch.empty((N_DECODE, gi.CONV_CHANNELS), dtype=torch.bfloat16, device=dev)
+        self.o = torch.empty((N_DECODE, H_V, D), dtype=torch.bfloat16, device=dev)
+        self.out = torch.empty_like(self.o)
+        self.launches_per_step = 4
+
+    def step(self, s, ev=None):
+        g, st = self.gdn, self.inputs[s % len(self.inputs)]
+        g.gdn_conv1d_silu(st["x_pre"], self.w, self.cu, conv_state_in=self.cache,
+                          conv_state_out=self.cache, y=self.y)
+        if ev is not None:
+            ev[0].record()
+        y = self.y
+        g.gdn_decode_step(y[:, :2048].view(-1, H_K, D), y[:, 2048:4096].view(-1, H_K, D),
+                          y[:, 4096:].view(-1, H_V, D), st["g"], st["beta"], self.state,
+                          o=self.o)
+        if ev is not None:
+            ev[1].record()
+        g.gdn_gated_rmsnorm(self.o, st["z"], self.nw, eps=1e-6, y=self.out)
+
+
+def timed_loop(step_fn, steps, warmup, flush, dist_barrier):
+    """Warm up, then time exactly `steps` steps. Each step's region and its
+    dominant kernel are bracketed by CUDA events on the current stream; an L2
+    flush (a write larger than L2) runs before each step, outside its events.
+    Returns (per-step ms list, dominant-kernel ms list)."""
+    for i in range(warmup):
+        step_fn(i, None)
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    dist_barrier()
+    torch.cuda.synchronize()
+    for i in range(steps):
+        flush.zero_()
+        e = evs[i]
+        e[0].record()
+        step_fn(i, (e[1], e[2]))
+        e[3].record()
+    torch.cuda.synchronize()
+    dist_barrier()
+    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
+    kern_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    return step_ms, kern_ms
+
+
+def e2e_prefill(gdn, wl, dev, steps, warmup):
+    """Same workload through the public API from pinned HOST buffers: the
+    step's inputs are copied host->device and its output device->host inside
+    the timed region."""
+    h = wl.host
+    hx = h["x_pre"].pin_memory()
+    hg, hb, hz = h["g"].pin_memory(), h["beta"].pin_memory(), h["z"].pin_memory()
+    hout = torch.empty(wl.out.shape, dtype=wl.out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (hx, hg, hb, hz))
+    d2h = hout.numel() * hout.element_size()
+
+    def one():
+        wl.x.copy_(hx, non_blocking=True)
+        wl.g.copy_(hg, non_blocking=True)
+        wl.b.copy_(hb, non_blocking=True)
+        wl.z.copy_(hz, non_blocking=True)
+        wl.step()
+        hout.copy_(wl.out, non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        one()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    return ms, h2d, d2h
+
+
+def gpu_arm(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU (B200)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if dist is None:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    import gated_delta_rule_106_b200 as gdn
+    gdn.load()
+    peaks, peak_src = load_peaks()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    pre = PrefillWorkload(gdn, dev, seed=rank)
+    with ClockSampler(local) as clk:
+        step_ms, kern_ms = timed_loop(lambda i, ev: pre.step(ev), args.steps,
+                                      args.warmup, flush, barrier)
+    ms = max_over_ranks(statistics.mean(step_ms))
+    kms = max_over_ranks(statistics.mean(kern_ms))
+    e2e_ms, h2d, d2h = e2e_prefill(gdn, pre, dev, max(2, args.steps // 4), 2)
+    e2e_ms = max_over_ranks(e2e_ms)
+
+    dec_steps = 128
+    dwl = DecodeWorkload(gdn, dev, seed=rank, steps=dec_steps)
+    d_step_ms, d_kern_ms = timed_loop(lambda i, ev: dwl.step(i, ev), dec_steps,
+                                      args.warmup, flush, barrier)
+    d_ms = max_over_ranks(statistics.mean(d_step_ms))
+    d_kms = max_over_ranks(statistics.mean(d_kern_ms))
+
+    tokens = T_PREFILL * world
+    flops = PREFILL_FLOP_PER_TOKEN * T_PREFILL
+    pre_ach = flops / (kms * 1e-3) / 1e12
+    dec_bytes = DECODE_BYTES_PER_TOKEN * N_DECODE
+    dec_ach = dec_bytes / (d_kms * 1e-3) / 1e9
+    tr = kernel_traffic("prefill")
+    dtr = kernel_traffic("decode")
+    line = {
+        "metric": METRIC,
+        "value": tokens / (ms * 1e-3),
+        "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded; shapes and distributions of the layer)",
+        "config": {
+            "workload": "prefill: one delta-rule layer, B=1, T=8192, 16 key / 48 value "
+                        "heads, d=128; conv k=4+SiLU+L2 -> chunked C=64 -> gated RMSNorm",
+            "global_batch": world, "seq_len": T_PREFILL,
+            "parallelism": f"replicas{world}" if world > 1 else "single",
+            "l2": "256 MiB write before every timed step, outside its events; "
+                  "x_pre (168 MB) also exceeds L2",
+        },
+        "roofline": {
+            "kernel": "gdn_chunked_prefill",
+            "bound": "tensor", "achieved": pre_ach,
+            "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": pre_ach / peaks["bf16_tflops"],
+            "peak_source": f"{peak_src} bf16 dense (burst)",
+            "traffic": tr,
+            "algorithmic_flop_per_launch": flops,
+            "kernel_ms": kms,
+        },
+        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_ms},
+        "gpu_launches": pre.launches_per_step * args.steps,
+        "clocks": clk.summary(),
+        "decode": {
+            "workload": "decode: 256 sequences x 128 steps, 1 token each, fp32 state "
+                        "[256,48,128,128]; conv (cache roll) -> decode step -> gated RMSNorm",
+            "value": N_DECODE * world / (d_ms * 1e-3), "unit": "tokens/s",
+            "ms_per_step": d_ms,
+            "roofline": {"kernel": "gdn_decode_step", "bound": "hbm",
+                         "achieved": dec_ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": dec_ach / peaks["hbm_gbs"],
+                         "peak_source": f"{peak_src} HBM copy",
+                         "traffic": dtr, "algorithmic_bytes_per_launch": dec_bytes,
+                         "kernel_ms": d_kms},
+            "gpu_launches": dwl.launches_per_step * dec_steps,
+        },
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.cpu_budget_s)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------- CPU arm --
+
+def oracle_sample(threads=0, heads=H_V, tokens=T_PREFILL, seed=0):
+    """The oracle on (part of) the prefill workload: conv of every channel of
+    `tokens` tokens, the recurrence for `heads` value heads (whole key-head
+    groups) and the gated RMS-norm of those heads. Returns (seconds, threads)."""
+    import oracle
+    p = gi.prefill_inputs(T=tokens, seed=seed)
+    x = gi.as_f64(p["x_pre"])
+    w = gi.as_f64(p["conv_w"])
+    cu = np.array([0, tokens], dtype=np.int32)
+    hw = oracle.hardware_threads()
+    nthreads = min(threads or hw, heads)
+    t0 = time.perf_counter()
+    y, _ = oracle.conv1d_silu_l2(x, w, None, cu, None, gi.L2_CHANNELS, 1e-6)
+    nk = heads // 3
+    q = y[:, :2048].reshape(tokens, H_K, D)[:, :nk]
+    k = y[:, 2048:4096].reshape(tokens, H_K, D)[:, :nk]
+    v = y[:, 4096:].reshape(tokens, H_V, D)[:, :heads]
+    o, _ = oracle.recurrence(q, k, v, gi.as_f64(p["g"])[:, :heads],
+                             gi.as_f64(p["beta"])[:, :heads], None, cu,
+                             threads=nthreads)
+    oracle.gated_rmsnorm(o, gi.as_f64(p["z"])[:, :heads], gi.as_f64(p["norm_w"]),
+                         1e-6, threads=nthreads)
+    return time.perf_counter() - t0, nthreads
+
+
+def cpu_baseline(budget_s=20.0):
+    """Oracle throughput on the host cores, scaled to tokens/s of the whole
+    layer: a short probe on 3 heads sizes a sample of ~budget_s seconds."""
+    probe_s, _ = oracle_sample(heads=3, tokens=1024)
+    hw = os.cpu_count() or 1
+    # conv dominates the probe's fixed part; size heads so the sample fits
+    est_per_head = probe_s / 3 * (T_PREFILL / 1024)
+    heads = int(max(3, min(H_V, (budget_s / max(est_per_head, 1e-9)) * min(hw, H_V))))
+    heads -= heads % 3
+    sec, threads = oracle_sample(heads=heads)
+    # the conv covers all heads already; scale the recurrence+norm share
+    layer_s = sec * (H_V / heads) if heads < H_V else sec
+    return {"value": T_PREFILL / layer_s, "unit": "tokens/s", "cores": threads,
+            "kind": "oracle",
+            "sample": f"T={T_PREFILL}: full conv, recurrence + gated RMSNorm for "
+                      f"{heads}/{H_V} value heads ({sec:.1f} s), scaled to 48 heads"}
+
+
+def reference_arm(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    # each step: the oracle on a bounded sample of the prefill workload
+    heads = 3
+    for _ in range(args.warmup):
+        oracle_sample(heads=heads, tokens=1024)
+    secs = []
+    threads = 0
+    for _ in range(args.steps):
+        s, threads = oracle_sample(heads=heads, tokens=1024)
+        secs.append(s)
+    per_step = statistics.mean(secs)
+    # tokens/s of the whole layer: 1024 tokens, 3 of 48 heads (conv: all)
+    value = 1024 / (per_step * H_V / heads)
+    line = {
+        "impl": "reference",
+        "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": per_step * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "prefill: one delta-rule layer, B=1, T=8192, 16 key / 48 "
+                               "value heads, d=128 (sampled: 1024 tokens, 3 heads per step)",
+                   "global_batch": 1, "seq_len": T_PREFILL, "parallelism": "host threads"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads,
+                         "kind": "oracle",
+                         "sample": "1024 tokens: full conv, recurrence + norm for 3 of 48 "
+                                   "value heads, scaled to the layer"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="gdn", choices=["gdn", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget-s", type=float, default=20.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        reference_arm(args)
+    else:
+        gpu_arm(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,214 @@
+"""gated_delta_rule_106_b200 -- B200-native gated delta-rule layer.
+
+Thin ctypes binding over the C ABI of ``libgdn.so`` (declared in
+``include/gdn.h``). Each function here has the name of its C entry point and
+only marshals arguments: torch CUDA tensors supply device memory and the
+current CUDA stream; every step of the computation runs in the library's
+sm_100a kernels. There is no CPU or PyTorch fallback: if ``libgdn.so`` is
+missing, or a tensor is not on a CUDA device, the call raises.
+
+Sources of the layer: "Agnes-3.0-Flash Preview" leaderboard commentary,
+section 二.1 (16 key / 48 value heads, head dim 128, kernel-4 causal conv,
+fp32 state, chunked prefill with chunk 64 and stepwise decode) and the
+Agnes-3.0-Flash Preview model card, 架构 table (gated RMS-norm).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+__all__ = ["GDN_BF16", "GDN_F32", "GdnError", "library_path", "load",
+           "gdn_conv1d_silu", "gdn_chunked_prefill",
+           "gdn_chunked_prefill_workspace", "gdn_decode_step",
+           "gdn_gated_rmsnorm", "gdn_status_string", "gdn_version",
+           "H_K", "H_V", "HEAD_DIM", "CHUNK"]
+
+GDN_BF16 = 0
+GDN_F32 = 1
+H_K, H_V, HEAD_DIM, CHUNK = 16, 48, 128, 64
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libgdn.so")
+_lib = None
+_lock = threading.Lock()
+
+_vp = ctypes.c_void_p
+_i64 = ctypes.c_int64
+_int = ctypes.c_int
+_f32 = ctypes.c_float
+
+# name -> (restype, argtypes)
+_SIGNATURES = {
+    "gdn_status_string": (ctypes.c_char_p, [_int]),
+    "gdn_version": (ctypes.c_char_p, []),
+    "gdn_conv1d_silu": (_int, [_vp, _i64, _int, _vp, _int, _vp, _int, _int, _f32,
+                               _vp, _int, _i64, _vp, _vp, _vp, _i64, _int, _vp]),
+    "gdn_chunked_prefill": (_int, [_vp, _vp, _vp, _int, _i64, _i64, _i64, _vp,
+                                   _vp, _int, _vp, _vp, _vp, _int, _i64, _int,
+                                   _int, _f32, _vp, _int, _vp, ctypes.c_size_t,
+                                   _vp]),
+    "gdn_chunked_prefill_workspace": (ctypes.c_size_t, [_int, _i64, _int, _int]),
+    "gdn_decode_step": (_int, [_vp, _vp, _vp, _int, _i64, _i64, _i64, _vp, _vp,
+                               _int, _vp, _int, _int, _int, _f32, _vp, _int,
+                               _vp]),
+    "gdn_gated_rmsnorm": (_int, [_vp, _int, _vp, _int, _vp, _int, _i64, _int,
+                                 _f32, _vp, _int, _vp]),
+}
+
+
+class GdnError(RuntimeError):
+    """A libgdn entry point returned a non-zero gdn_status."""
+
+    def __init__(self, fn, status):
+        self.status = status
+        super().__init__(f"{fn}: {gdn_status_string(status)} ({status})")
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load():
+    """Load libgdn.so (in-tree). Raises if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(_LIB_PATH):
+                raise RuntimeError(
+                    f"{_LIB_PATH} is missing: build it with "
+                    "`python -m gated_delta_rule_106_b200._build` (nvcc, sm_100a)")
+            lib = ctypes.CDLL(_LIB_PATH)
+            for name, (res, args) in _SIGNATURES.items():
+                fn = getattr(lib, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = lib
+        return _lib
+
+
+def gdn_status_string(status: int) -> str:
+    return load().gdn_status_string(int(status)).decode()
+
+
+def gdn_version() -> str:
+    return load().gdn_version().decode()
+
+
+def _dtype_code(t: torch.dtype) -> int:
+    if t == torch.bfloat16:
+        return GDN_BF16
+    if t == torch.float32:
+        return GDN_F32
+    raise TypeError(f"unsupported dtype {t}; use torch.bfloat16 or torch.float32")
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libgdn takes CUDA tensors only (no CPU path)")
+    return t.data_ptr()
+
+
+def _row_stride(t):
+    """Token-row stride (elements) of a tensor whose trailing dims are dense."""
+    if t.dim() >= 2:
+        inner = 1
+        for size, stride in zip(reversed(t.shape[1:]), reversed(t.stride()[1:])):
+            if size != 1 and stride != inner:
+                raise ValueError("trailing dimensions must be contiguous")
+            inner *= size
+    return t.stride(0)
+
+
+def _stream(stream, device):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return stream.cuda_stream if isinstance(stream, torch.cuda.Stream) else int(stream)
+
+
+def _check(fn, status):
+    if status != 0:
+        raise GdnError(fn, status)
+
+
+def gdn_conv1d_silu(x, w, cu_seqlens, *, bias=None, conv_state_in=None,
+                    conv_state_out=None, l2norm_channels=2 * H_K * HEAD_DIM,
+                    l2_eps=1e-6, y=None, y_dtype=None, stream=None):
+    """Causal kernel-4 conv + SiLU + per-head L2 norm of the leading
+    ``l2norm_channels`` channels. x [T, C]; w [C, 4]; cu_seqlens int32 [N+1];
+    conv states [N, 3, C] (x's dtype). Returns y [T, C]."""
+    T, C = x.shape
+    N = cu_seqlens.numel() - 1
+    if y is None:
+        y = torch.empty((T, C), dtype=y_dtype or x.dtype, device=x.device)
+    _check("gdn_conv1d_silu", load().gdn_conv1d_silu(
+        _ptr(x), _row_stride(x), _dtype_code(x.dtype), _ptr(w),
+        _dtype_code(w.dtype), _ptr(bias), C, l2norm_channels, l2_eps,
+        _ptr(cu_seqlens), N, T, _ptr(conv_state_in), _ptr(conv_state_out),
+        _ptr(y), _row_stride(y), _dtype_code(y.dtype), _stream(stream, x.device)))
+    return y
+
+
+def gdn_chunked_prefill_workspace(N, T_total, H_k=H_K, H_v=H_V) -> int:
+    return int(load().gdn_chunked_prefill_workspace(N, T_total, H_k, H_v))
+
+
+def gdn_chunked_prefill(q, k, v, g, beta, cu_seqlens, *, state_in=None,
+                        state_out=None, scale=1.0, o=None, o_dtype=None,
+                        workspace=None, stream=None):
+    """Chunked (C=64) gated delta rule over packed sequences.
+    q, k [T, H_k, 128] (views with any token stride); v [T, H_v, 128];
+    g, beta [T, H_v]; states fp32 [N, H_v, 128, 128]. Returns o [T, H_v, 128]."""
+    T, H_k, _ = q.shape
+    H_v = v.shape[1]
+    N = cu_seqlens.numel() - 1
+    if o is None:
+        o = torch.empty((T, H_v, HEAD_DIM), dtype=o_dtype or v.dtype, device=v.device)
+    need = gdn_chunked_prefill_workspace(N, T, H_k, H_v)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=v.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("gdn_chunked_prefill", load().gdn_chunked_prefill(
+        _ptr(q), _ptr(k), _ptr(v), _dtype_code(q.dtype), _row_stride(q),
+        _row_stride(k), _row_stride(v), _ptr(g), _ptr(beta), _dtype_code(g.dtype),
+        _ptr(state_in), _ptr(state_out), _ptr(cu_seqlens), N, T, H_k, H_v,
+        scale, _ptr(o), _dtype_code(o.dtype), _ptr(workspace), ws_bytes,
+        _stream(stream, v.device)))
+    return o
+
+
+def gdn_decode_step(q, k, v, g, beta, state, *, scale=1.0, o=None,
+                    o_dtype=None, stream=None):
+    """One decode token per sequence: q, k [N, H_k, 128]; v [N, H_v, 128];
+    g, beta [N, H_v]; state fp32 [N, H_v, 128, 128] updated in place.
+    Returns o [N, H_v, 128]."""
+    N, H_k, _ = q.shape
+    H_v = v.shape[1]
+    if o is None:
+        o = torch.empty((N, H_v, HEAD_DIM), dtype=o_dtype or v.dtype, device=v.device)
+    _check("gdn_decode_step", load().gdn_decode_step(
+        _ptr(q), _ptr(k), _ptr(v), _dtype_code(q.dtype), _row_stride(q),
+        _row_stride(k), _row_stride(v), _ptr(g), _ptr(beta), _dtype_code(g.dtype),
+        _ptr(state), N, H_k, H_v, scale, _ptr(o), _dtype_code(o.dtype),
+        _stream(stream, v.device)))
+    return o
+
+
+def gdn_gated_rmsnorm(x, z, w, *, eps=1e-6, y=None, y_dtype=None, stream=None):
+    """y = x / sqrt(mean(x^2) + eps) * w * SiLU(z) over the last dim (128)."""
+    dim = x.shape[-1]
+    rows = x.numel() // dim if dim else 0
+    if y is None:
+        y = torch.empty(x.shape, dtype=y_dtype or x.dtype, device=x.device)
+    for t in (x, z, y):
+        if not t.is_contiguous():
+            raise ValueError("gdn_gated_rmsnorm takes contiguous tensors")
+    _check("gdn_gated_rmsnorm", load().gdn_gated_rmsnorm(
+        _ptr(x), _dtype_code(x.dtype), _ptr(z), _dtype_code(z.dtype), _ptr(w),
+        _dtype_code(w.dtype), rows, dim, eps, _ptr(y), _dtype_code(y.dtype),
+        _stream(stream, x.device)))
+    return y

@@ -1,0 +1,185 @@
+// C-ABI entry points of libgdn.so: host-side validation, then dispatch to the
+// kernels. Nothing is launched when validation fails. The declarations, with
+// the passages each operation follows, are in include/gdn.h.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "gdn.h"
+#include "gdn_common.cuh"
+#include "launch.h"
+
+namespace {
+
+using gdn::kHeadDim;
+
+bool valid_dtype(gdn_dtype t) { return t == GDN_BF16 || t == GDN_F32; }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned_to(const void* p, int bytes) {
+  return (reinterpret_cast<uintptr_t>(p) % (uintptr_t)bytes) == 0;
+}
+bool stride_ok(int64_t stride_elems, gdn_dtype t) {
+  return (stride_elems * gdn::elem_bytes(t)) % 16 == 0;
+}
+gdn_status from_cuda(cudaError_t e) { return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA; }
+
+// [a, a+na) and [b, b+nb) overlap without being identical ranges
+bool partial_overlap(const void* a, size_t na, const void* b, size_t nb) {
+  if (!a || !b || na == 0 || nb == 0) return false;
+  uintptr_t a0 = (uintptr_t)a, b0 = (uintptr_t)b;
+  if (a0 == b0 && na == nb) return false;
+  return a0 < b0 + nb && b0 < a0 + na;
+}
+
+// Checks shared by the prefill and decode recurrences.
+gdn_status check_recurrence(const void* q, const void* k, const void* v,
+                            gdn_dtype qkv_dtype, int64_t qs, int64_t ks,
+                            int64_t vs, const void* g, const void* beta,
+                            gdn_dtype gate_dtype, int H_k, int H_v, void* o,
+                            gdn_dtype o_dtype, bool have_tokens) {
+  if (!valid_dtype(qkv_dtype) || !valid_dtype(gate_dtype) || !valid_dtype(o_dtype))
+    return GDN_ERR_INVALID_ARG;
+  if (H_k <= 0 || H_v <= 0 || H_v % H_k != 0) return GDN_ERR_INVALID_ARG;
+  if (qs < (int64_t)H_k * kHeadDim || ks < (int64_t)H_k * kHeadDim ||
+      vs < (int64_t)H_v * kHeadDim)
+    return GDN_ERR_INVALID_ARG;
+  if (!have_tokens) return GDN_OK;
+  if (!q || !k || !v || !g || !beta || !o) return GDN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return GDN_ERR_MISALIGNED;
+  if (!stride_ok(qs, qkv_dtype) || !stride_ok(ks, qkv_dtype) || !stride_ok(vs, qkv_dtype))
+    return GDN_ERR_MISALIGNED;
+  const int gb = gdn::elem_bytes(gate_dtype);
+  if (!aligned_to(g, gb) || !aligned_to(beta, gb)) return GDN_ERR_MISALIGNED;
+  return GDN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* gdn_status_string(gdn_status s) {
+  switch (s) {
+    case GDN_OK: return "GDN_OK";
+    case GDN_ERR_INVALID_ARG: return "GDN_ERR_INVALID_ARG: invalid argument";
+    case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED: unsupported shape or option";
+    case GDN_ERR_MISALIGNED: return "GDN_ERR_MISALIGNED: pointer or stride not 16-byte aligned";
+    case GDN_ERR_CUDA: return "GDN_ERR_CUDA: CUDA launch failed";
+  }
+  return "unknown gdn_status";
+}
+
+const char* gdn_version(void) { return "0.1.0"; }
+
+gdn_status gdn_conv1d_silu(const void* x, int64_t x_row_stride,
+                           gdn_dtype x_dtype, const void* w, gdn_dtype w_dtype,
+                           const void* bias, int channels, int l2norm_channels,
+                           float l2_eps, const int32_t* cu_seqlens, int N,
+                           int64_t T_total, const void* conv_state_in,
+                           void* conv_state_out, void* y, int64_t y_row_stride,
+                           gdn_dtype y_dtype, cudaStream_t stream) {
+  if (!valid_dtype(x_dtype) || !valid_dtype(w_dtype) || !valid_dtype(y_dtype))
+    return GDN_ERR_INVALID_ARG;
+  if (N < 0 || T_total < 0 || channels <= 0 || channels % 8 != 0)
+    return GDN_ERR_INVALID_ARG;
+  if (l2norm_channels < 0 || l2norm_channels % kHeadDim != 0 ||
+      l2norm_channels > channels || !(l2_eps >= 0.f))
+    return GDN_ERR_INVALID_ARG;
+  if (N == 0) return T_total == 0 ? GDN_OK : GDN_ERR_INVALID_ARG;
+  if (!cu_seqlens || !w) return GDN_ERR_INVALID_ARG;
+  if (T_total > 0) {
+    if (!x || !y) return GDN_ERR_INVALID_ARG;
+    if (x_row_stride < channels || y_row_stride < channels) return GDN_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(y)) return GDN_ERR_MISALIGNED;
+    if (!stride_ok(x_row_stride, x_dtype) || !stride_ok(y_row_stride, y_dtype))
+      return GDN_ERR_MISALIGNED;
+  }
+  if (!aligned16(w) || (bias && !aligned16(bias)) ||
+      (conv_state_in && !aligned16(conv_state_in)) ||
+      (conv_state_out && !aligned16(conv_state_out)))
+    return GDN_ERR_MISALIGNED;
+  const size_t cs_bytes = (size_t)N * 3 * channels * gdn::elem_bytes(x_dtype);
+  if (partial_overlap(conv_state_in, cs_bytes, conv_state_out, cs_bytes))
+    return GDN_ERR_INVALID_ARG;
+  gdn::ConvArgs a{x, x_row_stride, x_dtype, w, w_dtype, bias, channels,
+                  l2norm_channels, l2_eps, cu_seqlens, N, T_total,
+                  conv_state_in, conv_state_out, y, y_row_stride, y_dtype,
+                  stream};
+  return from_cuda(gdn::launch_conv1d_silu(a));
+}
+
+size_t gdn_chunked_prefill_workspace(int N, int64_t T_total, int H_k, int H_v) {
+  (void)N; (void)T_total; (void)H_k; (void)H_v;
+  return 0;
+}
+
+gdn_status gdn_chunked_prefill(const void* q, const void* k, const void* v,
+                               gdn_dtype qkv_dtype, int64_t q_row_stride,
+                               int64_t k_row_stride, int64_t v_row_stride,
+                               const void* g, const void* beta,
+                               gdn_dtype gate_dtype, const float* state_in,
+                               float* state_out, const int32_t* cu_seqlens,
+                               int N, int64_t T_total, int H_k, int H_v,
+                               float scale, void* o, gdn_dtype o_dtype,
+                               void* workspace, size_t workspace_bytes,
+                               cudaStream_t stream) {
+  if (N < 0 || T_total < 0) return GDN_ERR_INVALID_ARG;
+  gdn_status st = check_recurrence(q, k, v, qkv_dtype, q_row_stride, k_row_stride,
+                                   v_row_stride, g, beta, gate_dtype, H_k, H_v,
+                                   o, o_dtype, T_total > 0);
+  if (st != GDN_OK) return st;
+  if (N == 0) return T_total == 0 ? GDN_OK : GDN_ERR_INVALID_ARG;
+  if (!cu_seqlens) return GDN_ERR_INVALID_ARG;
+  if ((state_in && !aligned16(state_in)) || (state_out && !aligned16(state_out)))
+    return GDN_ERR_MISALIGNED;
+  const size_t st_bytes = (size_t)N * H_v * kHeadDim * kHeadDim * sizeof(float);
+  if (partial_overlap(state_in, st_bytes, state_out, st_bytes)) return GDN_ERR_INVALID_ARG;
+  if (workspace_bytes < gdn_chunked_prefill_workspace(N, T_total, H_k, H_v))
+    return GDN_ERR_INVALID_ARG;
+  gdn::RecurArgs a{q, k, v, qkv_dtype, q_row_stride, k_row_stride, v_row_stride,
+                   g, beta, gate_dtype, state_in, state_out, cu_seqlens, N,
+                   T_total, H_k, H_v, scale, o, o_dtype, workspace,
+                   workspace_bytes, stream};
+  return from_cuda(gdn::launch_prefill_stepwise(a));
+}
+
+gdn_status gdn_decode_step(const void* q, const void* k, const void* v,
+                           gdn_dtype qkv_dtype, int64_t q_row_stride,
+                           int64_t k_row_stride, int64_t v_row_stride,
+                           const void* g, const void* beta,
+                           gdn_dtype gate_dtype, float* state, int N, int H_k,
+                           int H_v, float scale, void* o, gdn_dtype o_dtype,
+                           cudaStream_t stream) {
+  if (N < 0) return GDN_ERR_INVALID_ARG;
+  gdn_status st = check_recurrence(q, k, v, qkv_dtype, q_row_stride, k_row_stride,
+                                   v_row_stride, g, beta, gate_dtype, H_k, H_v,
+                                   o, o_dtype, N > 0);
+  if (st != GDN_OK) return st;
+  if (N == 0) return GDN_OK;
+  if (!state) return GDN_ERR_INVALID_ARG;
+  if (!aligned16(state)) return GDN_ERR_MISALIGNED;
+  gdn::RecurArgs a{q, k, v, qkv_dtype, q_row_stride, k_row_stride, v_row_stride,
+                   g, beta, gate_dtype, state, state, nullptr, N, N, H_k, H_v,
+                   scale, o, o_dtype, nullptr, 0, stream};
+  return from_cuda(gdn::launch_decode_step(a));
+}
+
+gdn_status gdn_gated_rmsnorm(const void* x, gdn_dtype x_dtype, const void* z,
+                             gdn_dtype z_dtype, const void* w,
+                             gdn_dtype w_dtype, int64_t rows, int dim,
+                             float eps, void* y, gdn_dtype y_dtype,
+                             cudaStream_t stream) {
+  if (!valid_dtype(x_dtype) || !valid_dtype(z_dtype) || !valid_dtype(w_dtype) ||
+      !valid_dtype(y_dtype) || rows < 0 || !(eps >= 0.f))
+    return GDN_ERR_INVALID_ARG;
+  if (dim != kHeadDim) return GDN_ERR_UNSUPPORTED;
+  if (rows == 0) return GDN_OK;
+  if (!x || !z || !w || !y) return GDN_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(z) || !aligned16(w) || !aligned16(y))
+    return GDN_ERR_MISALIGNED;
+  if (x == y && x_dtype != y_dtype) return GDN_ERR_INVALID_ARG;
+  gdn::NormArgs a{x, x_dtype, z, z_dtype, w, w_dtype, rows, dim, eps, y, y_dtype,
+                  stream};
+  return from_cuda(gdn::launch_gated_rmsnorm(a));
+}
+
+}  // extern "C"

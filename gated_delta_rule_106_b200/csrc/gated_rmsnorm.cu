@@ -1,0 +1,87 @@
+// Gated RMS-norm on the delta-rule layer output (Agnes-3.0-Flash Preview model
+// card, 架构 table: "gated RMS-norm"):
+//   y = x / sqrt(mean(x^2) + eps) * w * SiLU(z)      per 128-channel row.
+//
+// HBM-bound: x and z are read once, y written once. 16 threads own one row
+// (8 channels = one 16-byte bf16 vector each); the sum of squares is a
+// 16-lane shuffle reduction. A grid-stride loop over rows keeps the grid at a
+// multiple of the SM count.
+#include "gdn_common.cuh"
+#include "launch.h"
+
+namespace gdn {
+namespace {
+
+constexpr int kNormThreads = 256;
+constexpr int kRowsPerIter = kNormThreads / 16;
+
+template <class Tx, class Tz, class Tw, class Ty>
+__global__ void __launch_bounds__(kNormThreads)
+gated_rmsnorm_kernel(const Tx* __restrict__ x, const Tz* __restrict__ z,
+                     const Tw* __restrict__ w, int64_t rows, float eps,
+                     Ty* y) {
+  const int sub = threadIdx.x & 15;          // 8-channel slice of the row
+  float wf[8];
+  load8(w + sub * 8, wf);
+  for (int64_t r = (int64_t)blockIdx.x * kRowsPerIter + (threadIdx.x >> 4);
+       r - (threadIdx.x >> 4) < rows;        // warp-uniform loop condition
+       r += (int64_t)gridDim.x * kRowsPerIter) {
+    const bool live = r < rows;
+    float xf[8], zf[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) xf[e] = zf[e] = 0.f;
+    if (live) {
+      load8(x + r * kHeadDim + sub * 8, xf);
+      load8(z + r * kHeadDim + sub * 8, zf);
+    }
+    float ss = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) ss = fmaf(xf[e], xf[e], ss);
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    const float inv = 1.0f / sqrtf(ss * (1.0f / kHeadDim) + eps);
+    float out[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) out[e] = xf[e] * inv * wf[e] * silu(zf[e]);
+    if (live) store8(y + r * kHeadDim + sub * 8, out);
+  }
+}
+
+template <class Tx, class Tz, class Tw, class Ty>
+cudaError_t launch_typed(const NormArgs& a) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int64_t blocks = (a.rows + kRowsPerIter - 1) / kRowsPerIter;
+  const int64_t cap = (int64_t)sms * 8;
+  if (blocks > cap) blocks = cap;
+  gated_rmsnorm_kernel<Tx, Tz, Tw, Ty><<<(unsigned)blocks, kNormThreads, 0, a.stream>>>(
+      static_cast<const Tx*>(a.x), static_cast<const Tz*>(a.z),
+      static_cast<const Tw*>(a.w), a.rows, a.eps, static_cast<Ty*>(a.y));
+  return cudaGetLastError();
+}
+
+template <class Tx, class Tz, class Tw>
+cudaError_t pick_y(const NormArgs& a) {
+  return a.y_dtype == GDN_F32 ? launch_typed<Tx, Tz, Tw, float>(a)
+                              : launch_typed<Tx, Tz, Tw, __nv_bfloat16>(a);
+}
+template <class Tx, class Tz>
+cudaError_t pick_w(const NormArgs& a) {
+  return a.w_dtype == GDN_F32 ? pick_y<Tx, Tz, float>(a)
+                              : pick_y<Tx, Tz, __nv_bfloat16>(a);
+}
+template <class Tx>
+cudaError_t pick_z(const NormArgs& a) {
+  return a.z_dtype == GDN_F32 ? pick_w<Tx, float>(a)
+                              : pick_w<Tx, __nv_bfloat16>(a);
+}
+
+}  // namespace
+
+cudaError_t launch_gated_rmsnorm(const NormArgs& a) {
+  if (a.rows == 0) return cudaSuccess;
+  return a.x_dtype == GDN_F32 ? pick_z<float>(a) : pick_z<__nv_bfloat16>(a);
+}
+
+}  // namespace gdn

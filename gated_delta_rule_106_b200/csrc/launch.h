@@ -1,0 +1,49 @@
+// Internal launch interface between the C-ABI layer (api.cu) and the kernels.
+// Arguments arrive here already validated.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "gdn.h"
+
+namespace gdn {
+
+struct ConvArgs {
+  const void* x; int64_t x_row_stride; gdn_dtype x_dtype;
+  const void* w; gdn_dtype w_dtype; const void* bias;
+  int channels; int l2norm_channels; float l2_eps;
+  const int32_t* cu_seqlens; int N; int64_t T_total;
+  const void* conv_state_in; void* conv_state_out;
+  void* y; int64_t y_row_stride; gdn_dtype y_dtype;
+  cudaStream_t stream;
+};
+
+struct RecurArgs {
+  const void* q; const void* k; const void* v; gdn_dtype qkv_dtype;
+  int64_t q_row_stride, k_row_stride, v_row_stride;
+  const void* g; const void* beta; gdn_dtype gate_dtype;
+  const float* state_in; float* state_out;   // decode: both = state
+  const int32_t* cu_seqlens;                 // decode: unused
+  int N; int64_t T_total; int H_k; int H_v; float scale;
+  void* o; gdn_dtype o_dtype;
+  void* workspace; size_t workspace_bytes;
+  cudaStream_t stream;
+};
+
+struct NormArgs {
+  const void* x; gdn_dtype x_dtype; const void* z; gdn_dtype z_dtype;
+  const void* w; gdn_dtype w_dtype; int64_t rows; int dim; float eps;
+  void* y; gdn_dtype y_dtype; cudaStream_t stream;
+};
+
+cudaError_t launch_conv1d_silu(const ConvArgs& a);
+cudaError_t launch_gated_rmsnorm(const NormArgs& a);
+cudaError_t launch_decode_step(const RecurArgs& a);
+// Stepwise fp32 recurrence on the CUDA cores (any input dtype).
+cudaError_t launch_prefill_stepwise(const RecurArgs& a);
+// Chunk-64 tensor-core prefill (bf16 inputs).
+cudaError_t launch_prefill_chunked_tc(const RecurArgs& a);
+
+}  // namespace gdn

@@ -1,0 +1,190 @@
+/*
+ * gdn.h -- C ABI of the gated delta-rule layer library (libgdn.so, sm_100a).
+ *
+ * The layer is the recurrent ("delta-rule") layer of the Agnes-3.0-Flash
+ * Preview hybrid decoder. Sources, cited by page and section:
+ *   [P2]  "Agnes-3.0-Flash Preview" leaderboard commentary (discosf.com),
+ *         section 二.1 "72 层里只有 18 层吃 KV cache": delta-rule layers are
+ *         recurrent with 16 key / 48 value heads and head dim 128, a kernel-4
+ *         causal conv comes first, the recurrent state is fp32
+ *         (mamba_ssm_dtype float32), and the modeling code has a chunked
+ *         prefill path (chunk = 64) and a stepwise decode path.
+ *   [P3]  Agnes-3.0-Flash Preview model card (modelscope.cn README_zh),
+ *         section 架构, architecture table: 3 of every 4 layers are gated
+ *         delta-rule layers (54 of 72), state size independent of sequence
+ *         length, causal conv (kernel 4) in front, gated RMS-norm, fp32 state.
+ * The pages name the operations but print neither equations nor an
+ * interface. The recurrence implemented is the gated delta rule
+ *     S_t = g_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T
+ *     o_t = scale * S_t q_t
+ * with S_t in R^{d_v x d_k} per (sequence, value head). Value head h reads
+ * key/query head h / (H_v / H_k) (contiguous groups).
+ *
+ * Conventions for every entry point:
+ *   - Every pointer is a DEVICE pointer on the current device, unless the
+ *     parameter says otherwise. The caller owns all memory; the library never
+ *     allocates, frees or synchronises, and launches only on `stream`.
+ *   - Data pointers must be 16-byte aligned and row strides (given in
+ *     ELEMENTS) must be multiples of 16 bytes; otherwise GDN_ERR_MISALIGNED.
+ *   - Arguments are validated on the host before anything is launched; on
+ *     any error nothing is launched and the outputs are untouched.
+ *     GDN_ERR_CUDA reports a launch failure (cudaGetLastError after launch).
+ *   - Head dim is fixed at 128 (d_k = d_v = 128) and H_v % H_k == 0.
+ *   - Packed variable-length batches: tokens of N sequences are concatenated
+ *     into T_total rows; cu_seqlens (device, int32, N+1 entries) holds the
+ *     prefix sums with cu_seqlens[0] = 0, cu_seqlens[N] = T_total and
+ *     non-decreasing entries (empty sequences allowed). cu_seqlens is read on
+ *     the device only (no device-to-host copy). Entries outside [0, T_total]
+ *     are clamped, so no access leaves the buffers, but the results for a
+ *     malformed cu_seqlens are unspecified.
+ *   - Recurrent states are fp32, [N, H_v, d_v=128, d_k=128], row-major
+ *     (d_k contiguous): row i of a head's state is an independent 512-byte
+ *     line.
+ */
+#ifndef GDN_H_
+#define GDN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  GDN_OK = 0,
+  GDN_ERR_INVALID_ARG = -1, /* null pointer, negative size, bad dtype ...  */
+  GDN_ERR_UNSUPPORTED = -2, /* valid but not implemented (head dim != 128) */
+  GDN_ERR_MISALIGNED = -3,  /* pointer or stride not 16-byte aligned        */
+  GDN_ERR_CUDA = -4         /* a CUDA launch or query failed               */
+} gdn_status;
+
+typedef enum { GDN_BF16 = 0, GDN_F32 = 1 } gdn_dtype;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* gdn_status_string(gdn_status status);
+
+/* Library version as "major.minor.patch" (static string). */
+const char* gdn_version(void);
+
+/*
+ * gdn_conv1d_silu -- fused causal depthwise conv (kernel 4) + SiLU + per-head
+ * L2 normalisation of the q and k channels.            [P2 二.1], [P3 架构]
+ *
+ *   y[t,c] = SiLU( bias[c] + sum_{j=0..3} w[c,j] * xh(t-3+j, c) )
+ *   then for each 128-channel group m with 128*m < l2norm_channels:
+ *   y[t, group] <- y[t, group] / sqrt(sum(y[t, group]^2) + l2_eps)
+ *
+ * xh(p, c) is the pre-conv input of the same sequence at position p; for
+ * positions before the sequence's first token it is the carried history
+ * conv_state_in[n, 3 + p_local, c] (p_local = -3..-1), or 0 when
+ * conv_state_in is NULL. Tap j = 3 multiplies the current token.
+ *
+ *   x               [T_total, channels], x_dtype, row stride x_row_stride.
+ *   w               [channels, 4], w_dtype (contiguous).
+ *   bias            [channels], w_dtype, or NULL (no bias).
+ *   channels        multiple of 8 (10240 = q 2048 | k 2048 | v 6144 here).
+ *   l2norm_channels leading channels normalised per 128 (4096 = q|k), a
+ *                   multiple of 128 and <= channels; 0 disables.
+ *   cu_seqlens      [N+1] int32 (device), see conventions.
+ *   conv_state_in   [N, 3, channels], x_dtype, oldest row first, or NULL.
+ *   conv_state_out  [N, 3, channels], x_dtype, or NULL. Receives the last
+ *                   three pre-conv rows of each sequence (shifted in from
+ *                   conv_state_in for sequences shorter than 3). It may alias
+ *                   conv_state_in (in-place roll for decode).
+ *   y               [T_total, channels], y_dtype, row stride y_row_stride.
+ *                   Must not overlap x.
+ * T_total == 0 is valid (only the conv state is rolled, i.e. copied).
+ * Decode uses the same call with one token per sequence.
+ */
+gdn_status gdn_conv1d_silu(const void* x, int64_t x_row_stride,
+                           gdn_dtype x_dtype, const void* w, gdn_dtype w_dtype,
+                           const void* bias, int channels, int l2norm_channels,
+                           float l2_eps, const int32_t* cu_seqlens, int N,
+                           int64_t T_total, const void* conv_state_in,
+                           void* conv_state_out, void* y, int64_t y_row_stride,
+                           gdn_dtype y_dtype, cudaStream_t stream);
+
+/*
+ * gdn_chunked_prefill -- the gated delta rule over packed sequences, computed
+ * chunk by chunk (chunk = 64 tokens, the chunked prefill path of [P2 二.1]).
+ * Results equal the stepwise recurrence above up to rounding.
+ *
+ *   q, k        [T_total, H_k, 128], qkv_dtype, token row strides
+ *               q_row_stride / k_row_stride (elements; heads contiguous).
+ *   v           [T_total, H_v, 128], qkv_dtype, row stride v_row_stride.
+ *               (Strides let the call read the packed conv output in place.)
+ *   g           [T_total, H_v] multiplicative decay in (0, 1], gate_dtype.
+ *   beta        [T_total, H_v] write strength, gate_dtype.
+ *   state_in    [N, H_v, 128, 128] fp32, or NULL for zero initial states.
+ *   state_out   [N, H_v, 128, 128] fp32, or NULL (not written). May alias
+ *               state_in exactly (in-place update); no partial overlap.
+ *   scale       multiplies every output (1.0 for the plain rule).
+ *   o           [T_total, H_v, 128] contiguous, o_dtype.
+ *   workspace   device scratch of gdn_chunked_prefill_workspace(...) bytes
+ *               (may be NULL when that is 0).
+ * Numerics: with qkv_dtype == GDN_BF16 the chunk products run on the tensor
+ * cores with binary16 operands and fp32 accumulation (bf16 inputs convert to
+ * binary16 exactly when |x| lies in [2^-14, 65504]; smaller magnitudes keep
+ * an absolute error below 2^-25); the state is carried in fp32. Inputs,
+ * states and outputs must stay well inside the binary16 range (|x| < 6e4).
+ * With qkv_dtype == GDN_F32 every product is fp32 on the CUDA cores.
+ */
+gdn_status gdn_chunked_prefill(const void* q, const void* k, const void* v,
+                               gdn_dtype qkv_dtype, int64_t q_row_stride,
+                               int64_t k_row_stride, int64_t v_row_stride,
+                               const void* g, const void* beta,
+                               gdn_dtype gate_dtype, const float* state_in,
+                               float* state_out, const int32_t* cu_seqlens,
+                               int N, int64_t T_total, int H_k, int H_v,
+                               float scale, void* o, gdn_dtype o_dtype,
+                               void* workspace, size_t workspace_bytes,
+                               cudaStream_t stream);
+
+/* Device scratch bytes gdn_chunked_prefill needs for these sizes (host). */
+size_t gdn_chunked_prefill_workspace(int N, int64_t T_total, int H_k, int H_v);
+
+/*
+ * gdn_decode_step -- one stepwise update of the gated delta rule for N
+ * sequences, one token each (the stepwise decode path of [P2 二.1]):
+ *   S <- g S (I - beta k k^T) + beta v k^T ;  o = scale * S q
+ * The state is read and written in place; each head's 64 KiB state crosses
+ * HBM once per call.
+ *
+ *   q, k    [N, H_k, 128], qkv_dtype, row strides q_row_stride/k_row_stride.
+ *   v       [N, H_v, 128], qkv_dtype, row stride v_row_stride.
+ *   g, beta [N, H_v], gate_dtype.
+ *   state   [N, H_v, 128, 128] fp32, updated in place.
+ *   o       [N, H_v, 128] contiguous, o_dtype.
+ * N == 0 is valid (nothing is launched).
+ */
+gdn_status gdn_decode_step(const void* q, const void* k, const void* v,
+                           gdn_dtype qkv_dtype, int64_t q_row_stride,
+                           int64_t k_row_stride, int64_t v_row_stride,
+                           const void* g, const void* beta,
+                           gdn_dtype gate_dtype, float* state, int N, int H_k,
+                           int H_v, float scale, void* o, gdn_dtype o_dtype,
+                           cudaStream_t stream);
+
+/*
+ * gdn_gated_rmsnorm -- gated RMS-norm on the layer output ([P3 架构]):
+ *   y = x / sqrt(mean(x^2) + eps) * w * SiLU(z)
+ * over rows of `dim` channels (one row per token and value head).
+ *
+ *   x  [rows, dim] x_dtype; z [rows, dim] z_dtype; w [dim] w_dtype (shared by
+ *   all rows); y [rows, dim] y_dtype (may alias x when the dtypes match).
+ *   dim must be 128. rows == 0 is valid.
+ */
+gdn_status gdn_gated_rmsnorm(const void* x, gdn_dtype x_dtype, const void* z,
+                             gdn_dtype z_dtype, const void* w,
+                             gdn_dtype w_dtype, int64_t rows, int dim,
+                             float eps, void* y, gdn_dtype y_dtype,
+                             cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H_ */

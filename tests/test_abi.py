@@ -1,0 +1,166 @@
+"""The C ABI: libgdn.so loads, exports every function include/gdn.h declares,
+and rejects bad arguments on the host before launching anything.
+
+These run without a GPU: every call here fails validation, which happens
+before any CUDA call, so no device work is attempted.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import gated_delta_rule_106_b200 as gdn
+from gated_delta_rule_106_b200 import _build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdn.h")
+
+OK, INVALID, UNSUPPORTED, MISALIGNED = 0, -1, -2, -3
+BF16, F32 = gdn.GDN_BF16, gdn.GDN_F32
+A = 0x10000          # a 16-byte aligned fake device address (never dereferenced)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    _build.build()
+    return gdn.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gdn_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_four_entry_points():
+    names = declared_functions()
+    for n in ("gdn_conv1d_silu", "gdn_chunked_prefill", "gdn_decode_step",
+              "gdn_gated_rmsnorm"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", gdn.library_path()],
+                         capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\b(gdn_\w+)$", out, flags=re.M))
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, missing
+    for n in declared_functions():
+        getattr(lib, n)
+
+
+def test_header_compiles_as_plain_c(tmp_path):
+    src = tmp_path / "t.c"
+    src.write_text('#include "gdn.h"\nint main(void){return (int)GDN_OK;}\n')
+    subprocess.run(["gcc", "-std=c99", "-fsyntax-only", "-I", os.path.join(ROOT, "include"),
+                    "-I", "/usr/local/cuda/include", str(src)], check=True)
+
+
+def test_status_strings(lib):
+    assert gdn.gdn_status_string(0) == "GDN_OK"
+    for s in (INVALID, UNSUPPORTED, MISALIGNED, -4):
+        assert "GDN_ERR" in gdn.gdn_status_string(s)
+    assert gdn.gdn_version().count(".") == 2
+
+
+def conv(lib, **kw):
+    a = dict(x=A, xs=10240, xdt=BF16, w=A, wdt=F32, bias=None, C=10240,
+             l2c=4096, eps=1e-6, cu=A, N=1, T=8, csi=None, cso=None, y=A,
+             ys=10240, ydt=BF16, s=None)
+    a.update(kw)
+    return lib.gdn_conv1d_silu(*a.values())
+
+
+def test_conv_validation(lib):
+    assert conv(lib, C=10241) == INVALID                 # channels % 8
+    assert conv(lib, l2c=100) == INVALID                 # not a multiple of 128
+    assert conv(lib, l2c=20480) == INVALID               # beyond channels
+    assert conv(lib, xdt=7) == INVALID
+    assert conv(lib, N=-1) == INVALID
+    assert conv(lib, T=-1) == INVALID
+    assert conv(lib, x=None) == INVALID
+    assert conv(lib, cu=None) == INVALID
+    assert conv(lib, xs=100) == INVALID                  # stride < channels
+    assert conv(lib, x=A + 2) == MISALIGNED
+    assert conv(lib, y=A + 8) == MISALIGNED
+    assert conv(lib, xs=10244) == MISALIGNED             # 20488 B not /16
+    assert conv(lib, csi=A + 4) == MISALIGNED
+    assert conv(lib, csi=A, cso=A + 16) == INVALID       # partial overlap
+    assert conv(lib, N=0, T=0) == OK                     # nothing to do
+    assert conv(lib, N=0, T=5) == INVALID
+
+
+def prefill(lib, **kw):
+    a = dict(q=A, k=A, v=A, dt=BF16, qs=10240, ks=10240, vs=10240, g=A, b=A,
+             gdt=F32, si=None, so=None, cu=A, N=1, T=64, Hk=16, Hv=48,
+             scale=1.0, o=A, odt=BF16, ws=None, wsb=0, s=None)
+    a.update(kw)
+    return lib.gdn_chunked_prefill(*a.values())
+
+
+def test_prefill_validation(lib):
+    assert prefill(lib, Hv=40) == INVALID                # H_v % H_k
+    assert prefill(lib, Hk=0) == INVALID
+    assert prefill(lib, qs=100) == INVALID               # stride < H_k * 128
+    assert prefill(lib, q=None) == INVALID
+    assert prefill(lib, cu=None) == INVALID
+    assert prefill(lib, dt=5) == INVALID
+    assert prefill(lib, q=A + 2) == MISALIGNED
+    assert prefill(lib, o=A + 4) == MISALIGNED
+    assert prefill(lib, qs=10244) == MISALIGNED
+    assert prefill(lib, g=A + 2) == MISALIGNED           # fp32 gate needs 4 B
+    assert prefill(lib, si=A + 8) == MISALIGNED
+    st = 48 * 128 * 128 * 4
+    assert prefill(lib, si=A, so=A + st // 2) == INVALID  # partial overlap
+    assert prefill(lib, N=0, T=0) == OK
+    assert prefill(lib, N=0, T=3) == INVALID
+    assert prefill(lib, N=-1) == INVALID
+
+
+def test_prefill_workspace_query(lib):
+    assert gdn.gdn_chunked_prefill_workspace(16, 135000) >= 0
+
+
+def decode(lib, **kw):
+    a = dict(q=A, k=A, v=A, dt=BF16, qs=10240, ks=10240, vs=10240, g=A, b=A,
+             gdt=BF16, state=A, N=256, Hk=16, Hv=48, scale=1.0, o=A, odt=BF16,
+             s=None)
+    a.update(kw)
+    return lib.gdn_decode_step(*a.values())
+
+
+def test_decode_validation(lib):
+    assert decode(lib, state=None) == INVALID
+    assert decode(lib, state=A + 4) == MISALIGNED
+    assert decode(lib, Hv=47) == INVALID
+    assert decode(lib, v=A + 2) == MISALIGNED
+    assert decode(lib, N=-2) == INVALID
+    assert decode(lib, N=0) == OK
+
+
+def norm(lib, **kw):
+    a = dict(x=A, xdt=BF16, z=A, zdt=BF16, w=A, wdt=F32, rows=10, dim=128,
+             eps=1e-6, y=A, ydt=BF16, s=None)
+    a.update(kw)
+    return lib.gdn_gated_rmsnorm(*a.values())
+
+
+def test_rmsnorm_validation(lib):
+    assert norm(lib, dim=64) == UNSUPPORTED
+    assert norm(lib, rows=-1) == INVALID
+    assert norm(lib, z=None) == INVALID
+    assert norm(lib, eps=-1.0) == INVALID
+    assert norm(lib, x=A + 2) == MISALIGNED
+    assert norm(lib, ydt=F32) == INVALID                 # y aliases x, other dtype
+    assert norm(lib, rows=0) == OK
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import torch
+    x = torch.zeros(4, 16, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        gdn.gdn_gated_rmsnorm(torch.zeros(2, 128), torch.zeros(2, 128),
+                              torch.ones(128))
+    del x

@@ -1,0 +1,225 @@
+"""GPU parity: gdn_chunked_prefill against the fp64 stepwise oracle.
+
+Bars (written here, per the gated delta rule spec): max|o - o_ref|/rms(o_ref)
+<= 1e-2 and per-sequence final-state relative Frobenius error <= 1e-3 for
+bf16 inputs; <= 1e-4 for fp32 inputs. Outputs stored in bf16 get half a bf16
+ulp of |o_ref| on top. The oracle is fed exactly the values the kernel read.
+
+Cases: the small fp32 case (T=256, stepwise and chunked), ragged edges
+around the 64-token chunk (1, 63, 64, 65, 130), empty sequences, null and
+in-place states, and the layer workloads at full size -- T=8192, 16 packed
+sequences of 512..16384 tokens, and T=262144 in 64 carried segments -- each
+checked on sampled head groups (every value head of the sampled key heads).
+"""
+import numpy as np
+import pytest
+import torch
+
+import gdn_inputs as gi
+import oracle
+import gated_delta_rule_106_b200 as gdn
+from _parity import O_TOL, S_TOL, bf16_out_bound, f64, o_err, state_err
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def random_qkv(seed, T, dtype, H_k=16, H_v=48, gate_dtype=torch.float32):
+    q = torch.from_numpy(gi.unit_heads(seed, "pq", T, H_k)).to(dtype)
+    k = torch.from_numpy(gi.unit_heads(seed, "pk", T, H_k)).to(dtype)
+    v = torch.from_numpy(gi.normal(seed, "pv", (T, H_v, 128))).to(dtype)
+    g, b = gi.gates(seed, T, H_v, dtype=gate_dtype, tag="pg")
+    return q, k, v, g, b
+
+
+def run_prefill(q, k, v, g, b, cu, state_in=None, o_dtype=torch.float32,
+                scale=1.0, in_place=False, want_state=True):
+    N = cu.numel() - 1
+    si = state_in.to(DEV) if state_in is not None else None
+    if in_place:
+        so = si
+    elif want_state:
+        so = torch.full((N, v.shape[1], 128, 128), float("nan"), device=DEV)
+    else:
+        so = None
+    o = gdn.gdn_chunked_prefill(q.to(DEV), k.to(DEV), v.to(DEV), g.to(DEV),
+                                b.to(DEV), cu.to(DEV), state_in=si, state_out=so,
+                                scale=scale, o_dtype=o_dtype)
+    torch.cuda.synchronize()
+    return o, so
+
+
+def check(o, S, o_ref, S_ref, dtype, o_dtype=torch.float32):
+    eo = o_err(o, o_ref)
+    bound = O_TOL[dtype] + (bf16_out_bound(o_ref) if o_dtype == torch.bfloat16 else 0)
+    assert eo <= bound, f"output error {eo:.3e} > {bound:.3e}"
+    if S is not None:
+        es = state_err(S, S_ref)
+        assert es <= S_TOL[dtype], f"state error {es:.3e} > {S_TOL[dtype]:.1e}"
+
+
+def cu_of(lens):
+    return torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32)
+
+
+def test_small_fp32_case_chunked_and_stepwise():
+    """T=256, fp32 q,k (unit), v ~ N(0,1), zero initial state: the chunked
+    call and 256 stepwise decode calls both match the oracle to 1e-4."""
+    p = gi.recurrence_inputs(T=256, seed=0)
+    cu = p["cu_seqlens"]
+    args = [p[n] for n in ("q", "k", "v", "g", "beta")]
+    o_ref, S_ref = oracle.recurrence(*map(f64, args), cu_seqlens=cu.numpy())
+    o, S = run_prefill(*args, cu)
+    check(o, S, o_ref, S_ref, torch.float32)
+    # stepwise: one decode call per token on a single sequence
+    Sd = torch.zeros(1, 48, 128, 128, device=DEV)
+    qd, kd, vd, gd, bd = (a.to(DEV) for a in args)
+    outs = [gdn.gdn_decode_step(qd[t:t + 1], kd[t:t + 1], vd[t:t + 1], gd[t:t + 1],
+                                bd[t:t + 1], Sd, o_dtype=torch.float32)
+            for t in range(256)]
+    torch.cuda.synchronize()
+    check(torch.cat(outs), Sd, o_ref, S_ref, torch.float32)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("lens", [[1], [63], [64], [65], [1, 63, 64, 65, 130]])
+def test_ragged_chunk_edges(dtype, lens):
+    cu = cu_of(lens)
+    T, N = int(cu[-1]), len(lens)
+    q, k, v, g, b = random_qkv(11, T, dtype)
+    S0 = gi.initial_states(11, N)
+    o_ref, S_ref = oracle.recurrence(f64(q), f64(k), f64(v), f64(g), f64(b),
+                                     f64(S0), cu.numpy())
+    o, S = run_prefill(q, k, v, g, b, cu, state_in=S0)
+    check(o, S, o_ref, S_ref, dtype)
+
+
+def test_empty_sequences_pass_state_through():
+    lens = [0, 70, 0, 0, 5]
+    cu = cu_of(lens)
+    q, k, v, g, b = random_qkv(12, int(cu[-1]), torch.bfloat16)
+    S0 = gi.initial_states(12, len(lens))
+    o_ref, S_ref = oracle.recurrence(f64(q), f64(k), f64(v), f64(g), f64(b),
+                                     f64(S0), cu.numpy())
+    o, S = run_prefill(q, k, v, g, b, cu, state_in=S0)
+    check(o, S, o_ref, S_ref, torch.bfloat16)
+    assert torch.equal(S[0].cpu(), S0[0]) and torch.equal(S[2].cpu(), S0[2])
+
+
+def test_null_state_in_in_place_and_no_state_out():
+    lens = [130, 64]
+    cu = cu_of(lens)
+    q, k, v, g, b = random_qkv(13, int(cu[-1]), torch.bfloat16)
+    o_ref, S_ref = oracle.recurrence(f64(q), f64(k), f64(v), f64(g), f64(b),
+                                     None, cu.numpy(), scale=128 ** -0.5)
+    o, S = run_prefill(q, k, v, g, b, cu, scale=128 ** -0.5)      # zeros in
+    check(o, S, o_ref, S_ref, torch.bfloat16)
+    o2, _ = run_prefill(q, k, v, g, b, cu, scale=128 ** -0.5, want_state=False)
+    check(o2, None, o_ref, None, torch.bfloat16)
+    S0 = gi.initial_states(13, 2)
+    o_ref3, S_ref3 = oracle.recurrence(f64(q), f64(k), f64(v), f64(g), f64(b),
+                                       f64(S0), cu.numpy())
+    o3, S3 = run_prefill(q, k, v, g, b, cu, state_in=S0, in_place=True)
+    check(o3, S3, o_ref3, S_ref3, torch.bfloat16)
+
+
+def test_bf16_output_and_long_memory_gates():
+    """g = exp(-0.01 softplus(N)) (long memory) and beta = 1 stress the
+    state carry across many chunks; output stored in bf16."""
+    T = 700
+    cu = cu_of([T])
+    q, k, v, g, b = random_qkv(14, T, torch.bfloat16)
+    g = (g.double() ** 0.01).float()
+    b = torch.ones_like(b)
+    S0 = gi.initial_states(14, 1)
+    o_ref, S_ref = oracle.recurrence(f64(q), f64(k), f64(v), f64(g), f64(b),
+                                     f64(S0), cu.numpy())
+    o, S = run_prefill(q, k, v, g, b, cu, state_in=S0, o_dtype=torch.bfloat16)
+    check(o, S, o_ref, S_ref, torch.bfloat16, o_dtype=torch.bfloat16)
+
+
+# ---- layer workloads at full size, checked on sampled head groups ----------
+
+def conv_gpu(x_pre, conv_w, cu, conv_state=None):
+    return gdn.gdn_conv1d_silu(x_pre.to(DEV), conv_w.to(DEV), cu.to(DEV),
+                               conv_state_in=conv_state, conv_state_out=conv_state)
+
+
+def qkv_views(y):
+    T = y.shape[0]
+    return (y[:, :2048].view(T, 16, 128), y[:, 2048:4096].view(T, 16, 128),
+            y[:, 4096:].view(T, 48, 128))
+
+
+def group_slices(y, key_heads):
+    """Host float64 q,k [T, len(kh), 128] and v [T, 3*len(kh), 128] for the
+    sampled key heads and all their value heads (mapping h//3 preserved)."""
+    q, k, v = qkv_views(y)
+    vh = [3 * kh + j for kh in key_heads for j in range(3)]
+    return (f64(q[:, key_heads]), f64(k[:, key_heads]), f64(v[:, vh]), vh)
+
+
+def test_prefill_8192_layer():
+    p = gi.prefill_inputs(T=8192, seed=0)
+    cu = p["cu_seqlens"]
+    y = conv_gpu(p["x_pre"], p["conv_w"], cu)
+    q, k, v = qkv_views(y)
+    S = torch.empty(1, 48, 128, 128, device=DEV)
+    o = gdn.gdn_chunked_prefill(q, k, v, p["g"].to(DEV), p["beta"].to(DEV),
+                                cu.to(DEV), state_out=S, o_dtype=torch.float32)
+    torch.cuda.synchronize()
+    kh = [0, 7, 15]
+    qs, ks, vs, vh = group_slices(y, kh)
+    o_ref, S_ref = oracle.recurrence(qs, ks, vs, f64(p["g"][:, vh]),
+                                     f64(p["beta"][:, vh]), None, cu.numpy())
+    check(o[:, vh], S[:, vh], o_ref, S_ref, torch.bfloat16)
+
+
+def test_prefill_varlen_16_sequences():
+    cu = gi.varlen_cu_seqlens(16, 512, 16384, seed=0)
+    T = int(cu[-1])
+    p = gi.prefill_inputs(T=T, seed=0, cu_seqlens=cu, with_state=True)
+    y = conv_gpu(p["x_pre"], p["conv_w"], cu)
+    q, k, v = qkv_views(y)
+    S = torch.empty(16, 48, 128, 128, device=DEV)
+    o = gdn.gdn_chunked_prefill(q, k, v, p["g"].to(DEV), p["beta"].to(DEV),
+                                cu.to(DEV), state_in=p["state_in"].to(DEV),
+                                state_out=S, o_dtype=torch.float32)
+    torch.cuda.synchronize()
+    lens = np.diff(cu.numpy())
+    seqs = sorted({int(np.argmin(lens)), int(np.argmax(lens)), 3, 9})
+    for n, kh in zip(seqs, [0, 15, 5, 10]):
+        a, e = int(cu[n]), int(cu[n + 1])
+        qs, ks, vs, vh = group_slices(y[a:e], [kh])
+        o_ref, S_ref = oracle.recurrence(qs, ks, vs, f64(p["g"][a:e, vh]),
+                                         f64(p["beta"][a:e, vh]),
+                                         f64(p["state_in"][n:n + 1, vh]))
+        check(o[a:e, vh], S[n:n + 1, vh], o_ref, S_ref, torch.bfloat16)
+
+
+def test_prefill_262144_in_64_segments():
+    """T=262144 as 64 calls of 4096 tokens with the recurrent state and the
+    conv history carried between calls; the final state and the last 4096
+    outputs of key head 15's value heads (45, 46, 47) are checked against the
+    oracle run over the whole sequence."""
+    seg, nseg, kh = 4096, 64, [15]
+    conv_w = gi.conv_weight(0)
+    cu = torch.tensor([0, seg], dtype=torch.int32)
+    S = torch.zeros(1, 48, 128, 128, device=DEV)
+    cache = torch.zeros(1, 3, gi.CONV_CHANNELS, dtype=torch.bfloat16, device=DEV)
+    parts, gates = [], []
+    for i in range(nseg):
+        p = gi.prefill_inputs(T=seg, seed=0, tag=f"seg{i}")
+        y = conv_gpu(p["x_pre"], conv_w, cu, conv_state=cache)
+        q, k, v = qkv_views(y)
+        o = gdn.gdn_chunked_prefill(q, k, v, p["g"].to(DEV), p["beta"].to(DEV),
+                                    cu.to(DEV), state_in=S, state_out=S,
+                                    o_dtype=torch.float32)
+        qs, ks, vs, vh = group_slices(y, kh)
+        parts.append((qs, ks, vs))
+        gates.append((f64(p["g"][:, vh]), f64(p["beta"][:, vh])))
+    torch.cuda.synchronize()
+    cat = lambda i, src: np.concatenate([x[i] for x in src])
+    o_ref, S_ref = oracle.recurrence(cat(0, parts), cat(1, parts), cat(2, parts),
+                                     cat(0, gates), cat(1, gates), None)
+    check(o[:, vh], S[:, vh], o_ref[-seg:], S_ref, torch.bfloat16)
