@@ -139,7 +139,8 @@ gdn_status gdn_chunked_prefill(const void* q, const void* k, const void* v,
                    g, beta, gate_dtype, state_in, state_out, cu_seqlens, N,
                    T_total, H_k, H_v, scale, o, o_dtype, workspace,
                    workspace_bytes, stream};
-  return from_cuda(gdn::launch_prefill_stepwise(a));
+  return from_cuda(qkv_dtype == GDN_BF16 ? gdn::launch_prefill_chunked_tc(a)
+                                         : gdn::launch_prefill_stepwise(a));
 }
 
 gdn_status gdn_decode_step(const void* q, const void* k, const void* v,
