@@ -108,8 +108,9 @@ gdn_status gdn_conv1d_silu(const void* x, int64_t x_row_stride,
 }
 
 size_t gdn_chunked_prefill_workspace(int N, int64_t T_total, int H_k, int H_v) {
-  (void)N; (void)T_total; (void)H_k; (void)H_v;
-  return 0;
+  (void)H_k;
+  if (N <= 0 || T_total <= 0 || H_v <= 0) return 0;
+  return gdn::prefill_pc_workspace(N, T_total, H_v);
 }
 
 gdn_status gdn_chunked_prefill(const void* q, const void* k, const void* v,
@@ -133,13 +134,17 @@ gdn_status gdn_chunked_prefill(const void* q, const void* k, const void* v,
     return GDN_ERR_MISALIGNED;
   const size_t st_bytes = (size_t)N * H_v * kHeadDim * kHeadDim * sizeof(float);
   if (partial_overlap(state_in, st_bytes, state_out, st_bytes)) return GDN_ERR_INVALID_ARG;
-  if (workspace_bytes < gdn_chunked_prefill_workspace(N, T_total, H_k, H_v))
-    return GDN_ERR_INVALID_ARG;
+  if (qkv_dtype == GDN_BF16 && T_total > 0) {
+    if (workspace_bytes < gdn_chunked_prefill_workspace(N, T_total, H_k, H_v) ||
+        (workspace_bytes > 0 && !workspace))
+      return GDN_ERR_INVALID_ARG;
+    if (!aligned16(workspace)) return GDN_ERR_MISALIGNED;
+  }
   gdn::RecurArgs a{q, k, v, qkv_dtype, q_row_stride, k_row_stride, v_row_stride,
                    g, beta, gate_dtype, state_in, state_out, cu_seqlens, N,
                    T_total, H_k, H_v, scale, o, o_dtype, workspace,
                    workspace_bytes, stream};
-  return from_cuda(qkv_dtype == GDN_BF16 ? gdn::launch_prefill_chunked_tc(a)
+  return from_cuda(qkv_dtype == GDN_BF16 ? gdn::launch_prefill_pc(a)
                                          : gdn::launch_prefill_stepwise(a));
 }
 

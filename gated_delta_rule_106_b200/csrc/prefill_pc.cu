@@ -1,0 +1,800 @@
+// Chunked gated delta rule on B200: a persistent producer/consumer kernel.
+//
+// The chunked prefill path ("delta_rule_chunked", chunk = 64: "Agnes-3.0-
+// Flash Preview" leaderboard commentary, section 二.1; fp32 recurrent state:
+// model card, 架构 table) splits, per 64-token chunk, into work that does not
+// depend on the state entering the chunk and work that does. With
+// G_t = sum_{s<=t} log g_s and S0 the state entering a chunk of L tokens:
+//   state-free:  A_ts = beta_t e^{G_t-G_s} k_t.k_s (s<t);  T = (I + A)^{-1}
+//                W = T diag(beta e^G) K;  U = T diag(beta) V;
+//                M_ts = e^{G_t-G_s} q_t.k_s (s<=t)
+//   state chain: Delta = U - W S0^T
+//                O     = scale (diag(e^G) Q S0^T + M Delta)
+//                S_L   = e^{G_L} S0 + Delta^T diag(e^{G_L-G}) K
+//
+// One cooperative launch, one CTA per SM, two roles:
+//  * state CTAs (about a third of the SMs) each own a list of (sequence,
+//    value head) items and run their chunks in order: per chunk two tcgen05
+//    MMAs on the critical path (Delta^T = U^T - S0 W^T, then P = Delta~^T K),
+//    the fp32 state in registers (four threads per row), outputs from
+//    S0 Q^T and Delta^T M^T.
+//  * prep CTAs claim (item, chunk) work in chunk order from a global counter
+//    and compute the state-free part: bf16 TMA tiles of K, Q, V; the Gram
+//    [K;Q] K^T on the tensor cores (bf16, exact products); decays; the UT
+//    solve in fp32; W and U as bf16 hi/lo MMAs (~17 significant bits, unit
+//    diagonal included); binary16 images of -W, K, Q and M (hi/lo). They
+//    publish one chunk per ring slot in the caller's workspace (3 slots per
+//    state CTA, ~97 KB each, L2-resident) with a release flag; the state CTA
+//    acquires it, bulk-copies the operand images into shared memory and
+//    releases the slot once read.
+// Deadlock freedom: all CTAs are co-resident (cooperative launch); a prep CTA
+// works on claims in increasing order and a claim only waits on the
+// consumption of an earlier step of the same state CTA. Every wait is
+// bounded (2 s); on a timeout the CTA raises a global abort word, every CTA
+// leaves its loops, and the outputs of unfinished items are left NaN-marked.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "gdn_common.cuh"
+#include "launch.h"
+#include "sm100.cuh"
+
+namespace gdn {
+namespace {
+
+using namespace sm100;
+
+constexpr int kPcThreads = 512;
+constexpr int kRing = 3;
+constexpr uint64_t kLimitNs = 2000000000ull;
+
+// ---- ring slot (global), 1024-aligned sections ---------------------------
+constexpr uint32_t SL_WN = 0;          // -W binary16, MN-major B image [128 d_k][64 t]
+constexpr uint32_t SL_KF = 16384;      // K binary16 image [2 blocks][64 t][64]
+constexpr uint32_t SL_QF = 32768;      // Q binary16 image [2 blocks][64 t][64]
+constexpr uint32_t SL_MH = 49152;      // M strictly lower, binary16 high part [64 t][64 s]
+constexpr uint32_t SL_ML = 57344;      // low part
+constexpr uint32_t SL_VEC = 65536;     // gamma[64] tail[64] mdiag[64] gL
+constexpr uint32_t SL_IMG = 66560;     // bytes of the shared-memory image above
+constexpr uint32_t SL_UT = 66560;      // U^T fp32 [64 t][128 i] (read straight from L2)
+constexpr uint32_t SLOT_BYTES = 99328;
+
+constexpr uint32_t CTRL_BYTES = 16384; // counter, abort word, per-state-CTA flags
+constexpr int kFlagStride = 16;        // ints per state CTA: full[kRing], consumed
+
+// ---- prep CTA shared memory ---------------------------------------------
+constexpr uint32_t P_KQ = 0;           // [blk0: K 8K | Q 8K][blk1: K | Q] bf16, TMA 128B swizzle
+constexpr uint32_t P_V = 32768;        // [blk0 8K][blk1 8K] bf16
+constexpr uint32_t P_AF = 49152;       // fp32 A [64][65]
+constexpr uint32_t P_TF = 65792;       // fp32 T [64][65]
+constexpr uint32_t P_XS = 82432;       // fp32 block-solve scratch [3][16][16]
+constexpr uint32_t P_T = 86016;        // bf16 T'hi, T'lo, T''hi, T''lo [64][64] each
+constexpr uint32_t P_STG = 118784;     // slot image staging (SL_IMG bytes)
+constexpr uint32_t P_SMALL = 185344;
+// ---- state CTA shared memory --------------------------------------------
+constexpr uint32_t S_BUF = 0;          // 2 x slot image
+constexpr uint32_t S_S0 = 133120;      // binary16 state, K-major [2 blocks][128 rows]
+constexpr uint32_t S_DTH = 165888;     // Delta^T high, K-major A [128][64 t]
+constexpr uint32_t S_DTL = 182272;     // Delta^T low
+constexpr uint32_t S_DKF = 198656;     // Delta~^T
+constexpr uint32_t S_SMALL = 215040;
+constexpr uint32_t PC_SMEM_BYTES = 215040 + 1024;
+constexpr uint32_t PC_SMEM_ALLOC = PC_SMEM_BYTES + 1024;
+
+// TMEM columns
+constexpr uint32_t PT_GR = 0, PT_W = 64, PT_U = 128, PT_COLS = 256;      // prep
+constexpr uint32_t ST_DT = 0, ST_P = 64, ST_OA = 192, ST_OB = 256, ST_COLS = 512;  // state
+
+struct PcParams {
+  const void* g; const void* beta;
+  const float* state_in; float* state_out;
+  const int32_t* cu; int64_t T; int N; int H_k; int H_v; float scale;
+  void* o;
+  uint8_t* ws;          // workspace base
+  int NS;               // state CTAs
+};
+
+struct PrepSmall {
+  float G[64], beta[64], gamma[64], bg[64], tail[64], mdiag[64];
+  float gL;
+  int claim;
+  int max_steps;
+  int ok;
+  uint32_t tmem;
+  uint64_t bar_tma, bar_mma;
+};
+struct StateSmall {
+  uint32_t tmem;
+  int ok;
+  uint64_t bar_slot[2], bar_dt, bar_p, bar_o;
+};
+
+__device__ __forceinline__ uint32_t swz(int r, int c) {
+  return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4));
+}
+__device__ __forceinline__ uint4 pack_half8(const float* f) {
+  uint4 u;
+  __half2* h = reinterpret_cast<__half2*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) h[i] = __floats2half2_rn(f[2 * i], f[2 * i + 1]);
+  return u;
+}
+__device__ __forceinline__ uint4 pack_bf8(const float* f) {
+  uint4 u;
+  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+  return u;
+}
+__device__ __forceinline__ float half_lo(float x) {
+  return x - __half2float(__float2half_rn(x));
+}
+__device__ __forceinline__ float bf_lo(float x) {
+  return x - __bfloat162float(__float2bfloat16_rn(x));
+}
+
+__device__ __forceinline__ int* flags_of(uint8_t* ws, int s) {
+  return reinterpret_cast<int*>(ws + 128) + s * kFlagStride;
+}
+__device__ __forceinline__ uint8_t* slot_of(uint8_t* ws, int s, int r) {
+  return ws + CTRL_BYTES + ((size_t)s * kRing + (size_t)(r % kRing)) * SLOT_BYTES;
+}
+
+// chunks of sequence n (clamped cu_seqlens)
+__device__ __forceinline__ int seq_chunks(const int32_t* cu, int64_t T, int n, int64_t* s0,
+                                          int64_t* s1) {
+  int64_t a = clamp_t(__ldg(cu + n), T), b = clamp_t(__ldg(cu + n + 1), T);
+  if (b < a) b = a;
+  *s0 = a;
+  *s1 = b;
+  return (int)((b - a + kChunk - 1) / kChunk);
+}
+__device__ int steps_of(const PcParams& p, int s) {
+  int total = 0;
+  int64_t a, b;
+  for (int i = s; i < p.N * p.H_v; i += p.NS) total += seq_chunks(p.cu, p.T, i / p.H_v, &a, &b);
+  return total;
+}
+// step r of state CTA s -> item i and chunk c (false if r is past its steps)
+__device__ bool locate(const PcParams& p, int s, int r, int* item, int* chunk) {
+  int64_t a, b;
+  for (int i = s; i < p.N * p.H_v; i += p.NS) {
+    const int nc = seq_chunks(p.cu, p.T, i / p.H_v, &a, &b);
+    if (r < nc) {
+      *item = i;
+      *chunk = r;
+      return true;
+    }
+    r -= nc;
+  }
+  return false;
+}
+
+// ===================================================================== prep ==
+template <class Tg>
+__device__ void prep_role(const PcParams& p, const CUtensorMap* tm_q, const CUtensorMap* tm_k,
+                          const CUtensorMap* tm_v, uint8_t* sm) {
+  PrepSmall& ss = *reinterpret_cast<PrepSmall*>(sm + P_SMALL);
+  float* Af = reinterpret_cast<float*>(sm + P_AF);
+  float* Tf = reinterpret_cast<float*>(sm + P_TF);
+  float* Xs = reinterpret_cast<float*>(sm + P_XS);
+  uint8_t* kq = sm + P_KQ;
+  uint8_t* vv = sm + P_V;
+  uint8_t* stg = sm + P_STG;
+  int* ctrl = reinterpret_cast<int*>(p.ws);   // [0] counter, [1] abort
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int q4 = warp & 3, cg = warp >> 2;          // TMEM lane quadrant, 16-column group
+  const int row = (q4 << 5) | lane;
+  const uint32_t lane_base = (uint32_t)(q4 << 5) << 16;
+
+  if (warp == 0) {
+    tmem_alloc(&ss.tmem, PT_COLS);
+    tmem_relinquish();
+  }
+  if (tid == 32) {
+    mbar_init(&ss.bar_tma, 1);
+    mbar_init(&ss.bar_mma, 1);
+    fence_mbar_init();
+  }
+  if (tid == 0) ss.max_steps = 0;
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ss.tmem;
+  for (int s = tid; s < p.NS; s += kPcThreads) atomicMax(&ss.max_steps, steps_of(p, s));
+  if (tid == 0) ss.claim = atomicAdd(&ctrl[0], 1);
+  __syncthreads();
+  const int64_t E = (int64_t)p.NS * ss.max_steps;
+  int e = ss.claim;
+  uint32_t tma_par = 0, mma_par = 0;
+  const uint32_t a_kq = smem_u32(kq), a_v = smem_u32(vv), a_t = smem_u32(sm + P_T);
+  const uint32_t id_gram = idesc_bf16(128, 64, false, false);
+  const uint32_t id_mn = idesc_bf16(128, 64, true, false);
+
+  while (e < E) {
+    const int s = e % p.NS, r = e / p.NS;
+    int item, c;
+    bool ok = true;
+    if (locate(p, s, r, &item, &c)) {
+      const int n = item / p.H_v, h = item % p.H_v, kh = h / (p.H_v / p.H_k);
+      int64_t s0, s1;
+      seq_chunks(p.cu, p.T, n, &s0, &s1);
+      const int64_t t0 = s0 + (int64_t)c * kChunk;
+      const int L = (int)((s1 - t0) < kChunk ? (s1 - t0) : kChunk);
+
+      if (tid == 0) {
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(&ss.bar_tma, 6 * 8192);
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {
+          tma_load_2d(kq + b * 16384, tm_k, kh * kHeadDim + b * 64, (int)t0, &ss.bar_tma);
+          tma_load_2d(kq + b * 16384 + 8192, tm_q, kh * kHeadDim + b * 64, (int)t0, &ss.bar_tma);
+          tma_load_2d(vv + b * 8192, tm_v, h * kHeadDim + b * 64, (int)t0, &ss.bar_tma);
+        }
+      }
+      if (warp == 1) {   // gates: cumulative log-decay and derived vectors
+        const Tg* g = static_cast<const Tg*>(p.g);
+        const Tg* bt = static_cast<const Tg*>(p.beta);
+        float lg[2], be[2];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int t = 2 * lane + j;
+          lg[j] = 0.f;
+          be[j] = 0.f;
+          if (t < L) {
+            const int64_t idx = (t0 + t) * p.H_v + h;
+            lg[j] = logf(fmaxf(to_f32(g[idx]), 1.17549435e-38f));
+            be[j] = to_f32(bt[idx]);
+          }
+        }
+        float incl = lg[0] + lg[1];
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const float y = __shfl_up_sync(0xffffffffu, incl, off);
+          if (lane >= off) incl += y;
+        }
+        const float excl = incl - (lg[0] + lg[1]);
+        const float Gl = __shfl_sync(0xffffffffu, incl, 31);
+        const float Gt[2] = {excl + lg[0], excl + lg[0] + lg[1]};
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int t = 2 * lane + j;
+          const float gam = __expf(Gt[j]);
+          ss.G[t] = Gt[j];
+          ss.beta[t] = be[j];
+          ss.gamma[t] = gam;
+          ss.bg[t] = be[j] * gam;
+          ss.tail[t] = __expf(Gl - Gt[j]);
+        }
+        if (lane == 0) ss.gL = __expf(Gl);
+      }
+      ok = mbar_wait_bounded(&ss.bar_tma, tma_par, kLimitNs);
+      tma_par ^= 1;
+      if (__syncthreads_or(!ok)) goto fail;
+
+      if (L < kChunk) {   // rows past the sequence end hold other data: zero them
+        for (int idx = tid; idx < 3072; idx += kPcThreads) {
+          const int rr = (idx & 511) >> 3;
+          if (rr >= L) {
+            uint8_t* ptr = idx < 2048 ? kq + idx * 16 : vv + (idx - 2048) * 16;
+            *reinterpret_cast<uint4*>(ptr) = make_uint4(0, 0, 0, 0);
+          }
+        }
+        fence_proxy_async_smem();
+        __syncthreads();
+      }
+      // ---- Gram [K;Q] K^T (bf16, exact products) ----
+      if (tid == 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_f16(tmem + PT_GR, sw128_desc(a_kq + off, 16, 1024),
+                  sw128_desc(a_kq + off, 16, 1024), id_gram, kk > 0);
+        }
+        mma_commit(&ss.bar_mma);
+      }
+      // K, Q -> binary16 images for the state CTA (overlaps the MMA)
+      for (int idx = tid; idx < 2048; idx += kPcThreads) {
+        const int which = idx >> 10, b = (idx >> 9) & 1, x = idx & 511;
+        const uint8_t* src = kq + b * 16384 + which * 8192 + x * 16;
+        float f[8];
+        load8(reinterpret_cast<const __nv_bfloat16*>(src), f);
+        *reinterpret_cast<uint4*>(stg + (which ? SL_QF : SL_KF) + b * 8192 + x * 16) =
+            pack_half8(f);
+      }
+      ok = mbar_wait_bounded(&ss.bar_mma, mma_par, kLimitNs);
+      mma_par ^= 1;
+      tc_fence_after();
+      {
+        float v[16];
+        tmem_ld16(tmem + lane_base + PT_GR + 16 * cg, v);
+        if (row < 64) {
+          const int t = row;
+          const float Gt = ss.G[t], bt = ss.beta[t];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int s2 = 16 * cg + j;
+            Af[t * 65 + s2] = (s2 < t) ? bt * __expf(Gt - ss.G[s2]) * v[j] : 0.f;
+          }
+        } else {
+          const int t = row - 64;
+          const float Gt = ss.G[t];
+          float mh[16], ml[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int s2 = 16 * cg + j;
+            const float val = (s2 <= t) ? __expf(Gt - ss.G[s2]) * v[j] : 0.f;
+            if (s2 == t) ss.mdiag[t] = val;
+            mh[j] = (s2 < t) ? val : 0.f;
+            ml[j] = half_lo(mh[j]);
+          }
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            *reinterpret_cast<uint4*>(stg + SL_MH + swz(t, 2 * cg + q)) = pack_half8(mh + 8 * q);
+            *reinterpret_cast<uint4*>(stg + SL_ML + swz(t, 2 * cg + q)) = pack_half8(ml + 8 * q);
+          }
+        }
+      }
+      tc_fence_before();
+      if (__syncthreads_or(!ok)) goto fail;
+
+      // ---- T = (I + A)^{-1}: 16x16 diagonal blocks, then block rows ----
+      if (tid < 64) {
+        const int I = tid >> 4, j = tid & 15;
+        float x[16];
+#pragma unroll
+        for (int rr = 0; rr < 16; ++rr) {
+          float acc = (rr == j) ? 1.f : 0.f;
+#pragma unroll
+          for (int m = 0; m < rr; ++m) acc = fmaf(-Af[(16 * I + rr) * 65 + 16 * I + m], x[m], acc);
+          x[rr] = acc;
+        }
+#pragma unroll
+        for (int rr = 0; rr < 16; ++rr) Tf[(16 * I + rr) * 65 + 16 * I + j] = x[rr];
+      }
+      __syncthreads();
+      for (int I = 1; I < 4; ++I) {
+        for (int task = tid; task < I * 256; task += kPcThreads) {
+          const int J = task >> 8, i = (task >> 4) & 15, j = task & 15;
+          float acc = 0.f;
+          for (int K = J; K < I; ++K) {
+#pragma unroll
+            for (int m = 0; m < 16; ++m)
+              acc = fmaf(Af[(16 * I + i) * 65 + 16 * K + m], Tf[(16 * K + m) * 65 + 16 * J + j], acc);
+          }
+          Xs[J * 256 + i * 16 + j] = acc;
+        }
+        __syncthreads();
+        for (int task = tid; task < I * 256; task += kPcThreads) {
+          const int J = task >> 8, i = (task >> 4) & 15, j = task & 15;
+          float acc = 0.f;
+#pragma unroll
+          for (int m = 0; m < 16; ++m)
+            acc = fmaf(Tf[(16 * I + i) * 65 + 16 * I + m], Xs[J * 256 + m * 16 + j], acc);
+          Tf[(16 * I + i) * 65 + 16 * J + j] = -acc;
+        }
+        __syncthreads();
+      }
+      // T' = T diag(beta e^G), T'' = T diag(beta) (unit diagonal included) as
+      // bf16 hi/lo K-major B images [t][s]
+      {
+        const int t = tid >> 3, c8 = tid & 7;
+        float ph[8], pl[8], qh[8], ql[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int s2 = c8 * 8 + j;
+          const float val = (s2 < t) ? Tf[t * 65 + s2] : (s2 == t ? 1.f : 0.f);
+          const float a = val * ss.bg[s2], b = val * ss.beta[s2];
+          ph[j] = a;
+          pl[j] = bf_lo(a);
+          qh[j] = b;
+          ql[j] = bf_lo(b);
+        }
+        *reinterpret_cast<uint4*>(sm + P_T + 0 * 8192 + swz(t, c8)) = pack_bf8(ph);
+        *reinterpret_cast<uint4*>(sm + P_T + 1 * 8192 + swz(t, c8)) = pack_bf8(pl);
+        *reinterpret_cast<uint4*>(sm + P_T + 2 * 8192 + swz(t, c8)) = pack_bf8(qh);
+        *reinterpret_cast<uint4*>(sm + P_T + 3 * 8192 + swz(t, c8)) = pack_bf8(ql);
+      }
+      fence_proxy_async_smem();
+      __syncthreads();
+      // ---- W^T = K^T T'^T, U^T = V^T T''^T (bf16 hi + lo) ----
+      if (tid == 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint64_t ak = sw128_desc(a_kq + ks * 2048, 16384, 1024);
+          const uint64_t av = sw128_desc(a_v + ks * 2048, 8192, 1024);
+          mma_f16(tmem + PT_W, ak, sw128_desc(a_t + 0 * 8192 + ks * 32, 16, 1024), id_mn, ks > 0);
+          mma_f16(tmem + PT_W, ak, sw128_desc(a_t + 1 * 8192 + ks * 32, 16, 1024), id_mn, 1);
+          mma_f16(tmem + PT_U, av, sw128_desc(a_t + 2 * 8192 + ks * 32, 16, 1024), id_mn, ks > 0);
+          mma_f16(tmem + PT_U, av, sw128_desc(a_t + 3 * 8192 + ks * 32, 16, 1024), id_mn, 1);
+        }
+        mma_commit(&ss.bar_mma);
+      }
+      // the slot must be free before anything is written to it
+      if (tid == 0)
+        ss.ok = wait_flag_ge(flags_of(p.ws, s) + kRing, r + 1 - kRing, &ctrl[1], kLimitNs);
+      ok = mbar_wait_bounded(&ss.bar_mma, mma_par, kLimitNs);
+      mma_par ^= 1;
+      tc_fence_after();
+      __syncthreads();
+      ok = ok && ss.ok;
+      if (__syncthreads_or(!ok)) goto fail;
+      {
+        uint8_t* slot = slot_of(p.ws, s, r);
+        float v[16];
+        tmem_ld16(tmem + lane_base + PT_W + 16 * cg, v);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[j] = -v[j];
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+          *reinterpret_cast<uint4*>(stg + SL_WN + swz(row, 2 * cg + q)) = pack_half8(v + 8 * q);
+        tmem_ld16(tmem + lane_base + PT_U + 16 * cg, v);
+        float* ut = reinterpret_cast<float*>(slot + SL_UT);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) ut[(16 * cg + j) * kHeadDim + row] = v[j];
+        float* vec = reinterpret_cast<float*>(stg + SL_VEC);
+        if (tid < 64) {
+          vec[tid] = ss.gamma[tid];
+          vec[64 + tid] = ss.tail[tid];
+          vec[128 + tid] = ss.mdiag[tid];
+        }
+        if (tid == 64) vec[192] = ss.gL;
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __threadfence();
+        __syncthreads();
+        if (tid == 0) {
+          bulk_s2g(slot, stg, SL_IMG);
+          bulk_commit();
+          bulk_wait_all();
+          fence_proxy_async_all();
+          __threadfence();
+          st_release(flags_of(p.ws, s) + (r % kRing), r + 1);
+        }
+      }
+    }
+    if (tid == 0) ss.claim = atomicAdd(&ctrl[0], 1);
+    __syncthreads();
+    e = ss.claim;
+    if (ld_acquire(&ctrl[1]) != 0) break;
+    continue;
+  fail:
+    if (tid == 0) atomicExch(&ctrl[1], 1);
+    break;
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, PT_COLS);
+}
+
+// ==================================================================== state ==
+template <class To>
+__device__ void state_role(const PcParams& p, uint8_t* sm, int s) {
+  StateSmall& ss = *reinterpret_cast<StateSmall*>(sm + S_SMALL);
+  int* ctrl = reinterpret_cast<int*>(p.ws);
+  int* flags = flags_of(p.ws, s);
+  To* o = static_cast<To*>(p.o);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int q4 = warp & 3, cg = warp >> 2;     // TMEM lane quadrant, column group (0..3)
+  const int row = (q4 << 5) | lane;            // state row (d_v index)
+  const uint32_t lane_base = (uint32_t)(q4 << 5) << 16;
+
+  if (warp == 0) {
+    tmem_alloc(&ss.tmem, ST_COLS);
+    tmem_relinquish();
+  }
+  if (tid == 32) {
+    mbar_init(&ss.bar_slot[0], 1);
+    mbar_init(&ss.bar_slot[1], 1);
+    mbar_init(&ss.bar_dt, 1);
+    mbar_init(&ss.bar_p, 1);
+    mbar_init(&ss.bar_o, 1);
+    fence_mbar_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ss.tmem;
+  const int total = steps_of(p, s);
+  const uint32_t a_s0 = smem_u32(sm + S_S0), a_dth = smem_u32(sm + S_DTH);
+  const uint32_t a_dtl = smem_u32(sm + S_DTL), a_dkf = smem_u32(sm + S_DKF);
+  const uint32_t id_kk = idesc_f16(128, 64, false, false);
+  const uint32_t id_mnb = idesc_f16(128, 64, false, true);
+  const uint32_t id_p = idesc_f16(128, 128, false, true);
+
+  int issued = 0;                 // slot copies issued (thread 0's view)
+  uint32_t par_dt = 0, par_p = 0, par_o = 0;
+  bool ok = true;
+  int r = 0;
+  auto issue_copy = [&](int step, bool block) -> bool {
+    int* full = flags + (step % kRing);
+    if (!block && ld_acquire(full) < step + 1) return false;
+    if (block && !wait_flag_ge(full, step + 1, &ctrl[1], kLimitNs)) return false;
+    fence_proxy_async_all();
+    uint64_t* bar = &ss.bar_slot[step & 1];
+    mbar_arrive_expect_tx(bar, SL_IMG);
+    bulk_g2s(sm + S_BUF + (step & 1) * SL_IMG, slot_of(p.ws, s, step), SL_IMG, bar);
+    return true;
+  };
+
+  for (int i = s; i < p.N * p.H_v && ok; i += p.NS) {
+    const int n = i / p.H_v, h = i % p.H_v;
+    int64_t s0, s1;
+    const int nch = seq_chunks(p.cu, p.T, n, &s0, &s1);
+    const int64_t nh = (int64_t)n * p.H_v + h;
+    float S[32];
+    {
+      const float* src = p.state_in ? p.state_in + (nh * kHeadDim + row) * kHeadDim + cg * 32 : nullptr;
+#pragma unroll
+      for (int j = 0; j < 32; j += 4) {
+        float4 v = src ? *reinterpret_cast<const float4*>(src + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+        S[j] = v.x; S[j + 1] = v.y; S[j + 2] = v.z; S[j + 3] = v.w;
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        *reinterpret_cast<uint4*>(sm + S_S0 + (cg >> 1) * 16384 + swz(row, (cg & 1) * 4 + q)) =
+            pack_half8(S + 8 * q);
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+
+    for (int c = 0; c < nch; ++c, ++r) {
+      const int b = r & 1;
+      uint8_t* buf = sm + S_BUF + b * SL_IMG;
+      const uint32_t a_buf = smem_u32(buf);
+      const int64_t t0 = s0 + (int64_t)c * kChunk;
+      const int L = (int)((s1 - t0) < kChunk ? (s1 - t0) : kChunk);
+      if (tid == 0) {
+        ss.ok = 1;
+        if (issued == r) {
+          if (issue_copy(r, true)) issued = r + 1;
+          else ss.ok = 0;
+        }
+      }
+      __syncthreads();
+      if (!ss.ok) { ok = false; break; }
+      // U^T values of this thread (row, tokens 16cg..16cg+15), straight from L2
+      float ut[16];
+      {
+        const float* src = reinterpret_cast<const float*>(slot_of(p.ws, s, r) + SL_UT);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) ut[j] = __ldcg(src + (16 * cg + j) * kHeadDim + row);
+      }
+      if (!mbar_wait_bounded(&ss.bar_slot[b], (uint32_t)((r >> 1) & 1), kLimitNs)) ok = false;
+      if (__syncthreads_or(!ok)) { ok = false; break; }
+      // ---- OA = S0 Q^T and Delta^T = S0 (-W^T) ----
+      if (tid == 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t a = sw128_desc(a_s0 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+          mma_f16(tmem + ST_DT, a, sw128_desc(a_buf + SL_WN + kk * 2048, 16384, 1024), id_mnb,
+                  kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t a = sw128_desc(a_s0 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+          mma_f16(tmem + ST_OA, a,
+                  sw128_desc(a_buf + SL_QF + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id_kk,
+                  kk > 0);
+        }
+        mma_commit(&ss.bar_dt);
+      }
+      if (!mbar_wait_bounded(&ss.bar_dt, par_dt, kLimitNs)) ok = false;
+      par_dt ^= 1;
+      tc_fence_after();
+      // ---- Delta = U + (-W S0^T): operands Delta^T (hi, lo) and Delta~^T ----
+      const float* vec = reinterpret_cast<const float*>(buf + SL_VEC);
+      float d[16];
+      {
+        float v[16], dh[16], dl[16], dk[16];
+        tmem_ld16(tmem + lane_base + ST_DT + 16 * cg, v);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          d[j] = v[j] + ut[j];
+          dh[j] = d[j];
+          dl[j] = half_lo(d[j]);
+          dk[j] = d[j] * vec[64 + 16 * cg + j];
+        }
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          *reinterpret_cast<uint4*>(sm + S_DTH + swz(row, 2 * cg + q)) = pack_half8(dh + 8 * q);
+          *reinterpret_cast<uint4*>(sm + S_DTL + swz(row, 2 * cg + q)) = pack_half8(dl + 8 * q);
+          *reinterpret_cast<uint4*>(sm + S_DKF + swz(row, 2 * cg + q)) = pack_half8(dk + 8 * q);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      if (__syncthreads_or(!ok)) { ok = false; break; }
+      // ---- P = Delta~^T K (critical), then OB = Delta^T M^T (hi/lo) ----
+      if (tid == 0) {
+        st_release(flags + kRing, r + 1);      // slot r fully read
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          mma_f16(tmem + ST_P, sw128_desc(a_dkf + ks * 32, 16, 1024),
+                  sw128_desc(a_buf + SL_KF + ks * 2048, 8192, 1024), id_p, ks > 0);
+        mma_commit(&ss.bar_p);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint64_t mh = sw128_desc(a_buf + SL_MH + ks * 32, 16, 1024);
+          const uint64_t ml = sw128_desc(a_buf + SL_ML + ks * 32, 16, 1024);
+          mma_f16(tmem + ST_OB, sw128_desc(a_dth + ks * 32, 16, 1024), mh, id_kk, ks > 0);
+          mma_f16(tmem + ST_OB, sw128_desc(a_dtl + ks * 32, 16, 1024), mh, id_kk, 1);
+          mma_f16(tmem + ST_OB, sw128_desc(a_dth + ks * 32, 16, 1024), ml, id_kk, 1);
+        }
+        mma_commit(&ss.bar_o);
+        // prefetch the next step's slot into the other buffer if it is ready
+        if (issued == r + 1 && r + 1 < total && issue_copy(r + 1, false)) issued = r + 2;
+      }
+      if (!mbar_wait_bounded(&ss.bar_p, par_p, kLimitNs)) ok = false;
+      par_p ^= 1;
+      tc_fence_after();
+      {
+        const float gL = vec[192];
+        float pv[32];
+        tmem_ld32(tmem + lane_base + ST_P + 32 * cg, pv);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) S[j] = fmaf(gL, S[j], pv[j]);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          *reinterpret_cast<uint4*>(sm + S_S0 + (cg >> 1) * 16384 + swz(row, (cg & 1) * 4 + q)) =
+              pack_half8(S + 8 * q);
+      }
+      if (!mbar_wait_bounded(&ss.bar_o, par_o, kLimitNs)) ok = false;
+      par_o ^= 1;
+      tc_fence_after();
+      {
+        float oa[16], ob[16];
+        tmem_ld16(tmem + lane_base + ST_OA + 16 * cg, oa);
+        tmem_ld16(tmem + lane_base + ST_OB + 16 * cg, ob);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int t = 16 * cg + j;
+          if (t < L) {
+            const float val = p.scale * (vec[t] * oa[j] + ob[j] + vec[128 + t] * d[j]);
+            o[((t0 + t) * p.H_v + h) * kHeadDim + row] = from_f32<To>(val);
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      if (__syncthreads_or(!ok)) { ok = false; break; }
+    }
+    if (p.state_out) {
+      float* dst = p.state_out + (nh * kHeadDim + row) * kHeadDim + cg * 32;
+      const float qnan = __int_as_float(0x7fc00000);
+#pragma unroll
+      for (int j = 0; j < 32; j += 4)
+        *reinterpret_cast<float4*>(dst + j) =
+            ok ? make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]) : make_float4(qnan, qnan, qnan, qnan);
+    }
+  }
+  if (!ok && tid == 0) atomicExch(&ctrl[1], 1);
+  // drain our own copies before leaving (bounded)
+  if (tid == 0)
+    for (int st = r; st < issued; ++st)
+      mbar_wait_bounded(&ss.bar_slot[st & 1], (uint32_t)((st >> 1) & 1), kLimitNs);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, ST_COLS);
+}
+
+template <class Tg, class To>
+__global__ void __launch_bounds__(kPcThreads, 1)
+prefill_pc_kernel(const __grid_constant__ CUtensorMap tm_q,
+                  const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const PcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  if ((int)blockIdx.x < p.NS) state_role<To>(p, sm, blockIdx.x);
+  else prep_role<Tg>(p, &tm_q, &tm_k, &tm_v, sm);
+}
+
+// ------------------------------------------------------------------ host --
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void* ptr = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+bool make_map(CUtensorMap* m, const void* base, int64_t cols, int64_t rows, int64_t stride) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(stride * 2)};
+  cuuint32_t box[2] = {64, 64};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+template <class Tg, class To>
+cudaError_t launch_typed(const RecurArgs& a, int nsm, int NS) {
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, a.q, (int64_t)a.H_k * kHeadDim, a.T_total, a.q_row_stride) ||
+      !make_map(&mk, a.k, (int64_t)a.H_k * kHeadDim, a.T_total, a.k_row_stride) ||
+      !make_map(&mv, a.v, (int64_t)a.H_v * kHeadDim, a.T_total, a.v_row_stride))
+    return cudaErrorInvalidValue;
+  auto kern = prefill_pc_kernel<Tg, To>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)PC_SMEM_ALLOC);
+  if (e != cudaSuccess) return e;
+  e = cudaMemsetAsync(a.workspace, 0, CTRL_BYTES, a.stream);
+  if (e != cudaSuccess) return e;
+  PcParams p{a.g, a.beta, a.state_in, a.state_out, a.cu_seqlens, a.T_total, a.N,
+             a.H_k, a.H_v, a.scale, a.o, static_cast<uint8_t*>(a.workspace), NS};
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)nsm);
+  cfg.blockDim = dim3(kPcThreads);
+  cfg.dynamicSmemBytes = PC_SMEM_ALLOC;
+  cfg.stream = a.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, p);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+template <class Tg>
+cudaError_t pick_o(const RecurArgs& a, int nsm, int NS) {
+  return a.o_dtype == GDN_F32 ? launch_typed<Tg, float>(a, nsm, NS)
+                              : launch_typed<Tg, __nv_bfloat16>(a, nsm, NS);
+}
+
+// State CTAs: about a third of the SMs (a multiple of H_v when that fits, so
+// that every state CTA gets the same heads of every sequence), at most one per
+// item; the remaining SMs prepare chunks.
+int state_ctas(int64_t items, int H_v, int nsm) {
+  int base = nsm / 3;
+  if (base < 1) base = 1;
+  if (items <= base) return (int)items;
+  if (H_v <= base) return (base / H_v) * H_v;
+  return base;
+}
+
+}  // namespace
+
+size_t prefill_pc_workspace(int N, int64_t T_total, int H_v) {
+  const int nsm = sm_count();
+  if (nsm < 2 || N <= 0 || T_total <= 0) return 0;
+  const int NS = state_ctas((int64_t)N * H_v, H_v, nsm);
+  return CTRL_BYTES + (size_t)NS * kRing * SLOT_BYTES;
+}
+
+cudaError_t launch_prefill_pc(const RecurArgs& a) {
+  if (a.N == 0) return cudaSuccess;
+  if (a.T_total == 0) return launch_prefill_stepwise(a);   // only state copies
+  const int nsm = sm_count();
+  if (nsm < 2) return cudaErrorInvalidDevice;
+  const int NS = state_ctas((int64_t)a.N * a.H_v, a.H_v, nsm);
+  if (a.workspace_bytes < CTRL_BYTES + (size_t)NS * kRing * SLOT_BYTES || !a.workspace)
+    return cudaErrorInvalidValue;
+  return a.gate_dtype == GDN_F32 ? pick_o<float>(a, nsm, NS) : pick_o<__nv_bfloat16>(a, nsm, NS);
+}
+
+}  // namespace gdn
