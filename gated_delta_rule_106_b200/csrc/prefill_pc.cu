@@ -56,7 +56,7 @@ constexpr uint32_t SL_MH = 49152;      // M strictly lower, binary16 high part [
 constexpr uint32_t SL_ML = 57344;      // low part
 constexpr uint32_t SL_VEC = 65536;     // gamma[64] tail[64] mdiag[64] gL
 constexpr uint32_t SL_IMG = 66560;     // bytes of the shared-memory image above
-constexpr uint32_t SL_UT = 66560;      // U^T fp32 [64 t][128 i] (read straight from L2)
+constexpr uint32_t SL_UT = 66560;      // U^T fp32 [64 t][128 i] (the consumer reads it from L2)
 constexpr uint32_t SLOT_BYTES = 99328;
 
 constexpr uint32_t CTRL_BYTES = 16384; // counter, abort word, per-state-CTA flags
@@ -65,12 +65,12 @@ constexpr int kFlagStride = 16;        // ints per state CTA: full[kRing], consu
 // ---- prep CTA shared memory ---------------------------------------------
 constexpr uint32_t P_KQ = 0;           // [blk0: K 8K | Q 8K][blk1: K | Q] bf16, TMA 128B swizzle
 constexpr uint32_t P_V = 32768;        // [blk0 8K][blk1 8K] bf16
-constexpr uint32_t P_AF = 49152;       // fp32 A [64][65]
-constexpr uint32_t P_TF = 65792;       // fp32 T [64][65]
-constexpr uint32_t P_XS = 82432;       // fp32 block-solve scratch [3][16][16]
+constexpr int kLd = 68;                // row stride (floats) of the fp32 A and T tiles
+constexpr uint32_t P_AF = 49152;       // fp32 A [64][kLd]
+constexpr uint32_t P_TF = 66560;       // fp32 T [64][kLd]
 constexpr uint32_t P_T = 86016;        // bf16 T'hi, T'lo, T''hi, T''lo [64][64] each
-constexpr uint32_t P_STG = 118784;     // slot image staging (SL_IMG bytes)
-constexpr uint32_t P_SMALL = 185344;
+constexpr uint32_t P_STG = 118784;     // whole-slot staging (SLOT_BYTES), one bulk store
+constexpr uint32_t P_SMALL = 218112;
 // ---- state CTA shared memory --------------------------------------------
 constexpr uint32_t S_BUF = 0;          // 2 x slot image
 constexpr uint32_t S_S0 = 133120;      // binary16 state, K-major [2 blocks][128 rows]
@@ -78,7 +78,7 @@ constexpr uint32_t S_DTH = 165888;     // Delta^T high, K-major A [128][64 t]
 constexpr uint32_t S_DTL = 182272;     // Delta^T low
 constexpr uint32_t S_DKF = 198656;     // Delta~^T
 constexpr uint32_t S_SMALL = 215040;
-constexpr uint32_t PC_SMEM_BYTES = 215040 + 1024;
+constexpr uint32_t PC_SMEM_BYTES = P_SMALL + 2048;
 constexpr uint32_t PC_SMEM_ALLOC = PC_SMEM_BYTES + 1024;
 
 // TMEM columns
@@ -170,6 +170,63 @@ __device__ bool locate(const PcParams& p, int s, int r, int* item, int* chunk) {
   return false;
 }
 
+// One merge level of the blocked inverse of a 64x64 unit lower-triangular
+// matrix: for each pair of b x b diagonal blocks already inverted (T11, T22),
+// T21 = -T22 (A21 T11). T holds zeros above its diagonal; rows of A, T and
+// X are read four floats at a time; at b = 32 each thread makes two adjacent
+// outputs.
+template <int b>
+__device__ __forceinline__ void merge_level(const float* Af, float* Tf, float* Xs, int tid) {
+  constexpr int bb = b * b, pairs = 64 / (2 * b), outs = pairs * bb;
+  constexpr int per = outs / kPcThreads > 0 ? outs / kPcThreads : 1;   // 1 or 2 adjacent columns
+  constexpr int threads = outs / per;
+  if (tid < threads) {
+    const int idx = tid * per;
+    const int pr = idx / bb, i = (idx / b) % b, j = idx % b, o = 2 * b * pr;
+    const float4* arow = reinterpret_cast<const float4*>(Af + (o + b + i) * kLd + o);
+    float acc[per][2];
+#pragma unroll
+    for (int c = 0; c < per; ++c) acc[c][0] = acc[c][1] = 0.f;
+#pragma unroll
+    for (int m4 = 0; m4 < b / 4; ++m4) {
+      const float4 a = arow[m4];
+      const float av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float* tr = Tf + (o + 4 * m4 + u) * kLd + o + j;
+#pragma unroll
+        for (int c = 0; c < per; ++c) acc[c][u & 1] = fmaf(av[u], tr[c], acc[c][u & 1]);
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < per; ++c) Xs[idx + c] = acc[c][0] + acc[c][1];
+  }
+  __syncthreads();
+  if (tid < threads) {
+    const int idx = tid * per;
+    const int pr = idx / bb, i = (idx / b) % b, j = idx % b, o = 2 * b * pr;
+    const float4* trow = reinterpret_cast<const float4*>(Tf + (o + b + i) * kLd + o + b);
+    const float* xcol = Xs + pr * bb + j;
+    float acc[per][2];
+#pragma unroll
+    for (int c = 0; c < per; ++c) acc[c][0] = acc[c][1] = 0.f;
+#pragma unroll
+    for (int m4 = 0; m4 < b / 4; ++m4) {
+      const float4 t4 = trow[m4];
+      const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float* xr = xcol + (4 * m4 + u) * b;
+#pragma unroll
+        for (int c = 0; c < per; ++c) acc[c][u & 1] = fmaf(tv[u], xr[c], acc[c][u & 1]);
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < per; ++c) Tf[(o + b + i) * kLd + o + j + c] = -(acc[c][0] + acc[c][1]);
+  }
+  __syncthreads();
+}
+
 // ===================================================================== prep ==
 template <class Tg>
 __device__ void prep_role(const PcParams& p, const CUtensorMap* tm_q, const CUtensorMap* tm_k,
@@ -177,7 +234,7 @@ __device__ void prep_role(const PcParams& p, const CUtensorMap* tm_q, const CUte
   PrepSmall& ss = *reinterpret_cast<PrepSmall*>(sm + P_SMALL);
   float* Af = reinterpret_cast<float*>(sm + P_AF);
   float* Tf = reinterpret_cast<float*>(sm + P_TF);
-  float* Xs = reinterpret_cast<float*>(sm + P_XS);
+  float* Xs = reinterpret_cast<float*>(sm + P_T);   // solve scratch (T' tiles are written after)
   uint8_t* kq = sm + P_KQ;
   uint8_t* vv = sm + P_V;
   uint8_t* stg = sm + P_STG;
@@ -203,11 +260,57 @@ __device__ void prep_role(const PcParams& p, const CUtensorMap* tm_q, const CUte
   tc_fence_after();
   const uint32_t tmem = ss.tmem;
   for (int s = tid; s < p.NS; s += kPcThreads) atomicMax(&ss.max_steps, steps_of(p, s));
-  if (tid == 0) ss.claim = atomicAdd(&ctrl[0], 1);
   __syncthreads();
   const int64_t E = (int64_t)p.NS * ss.max_steps;
-  int e = ss.claim;
+  // Claim the next (state CTA, step) that exists: thread 0 claims, all read.
+  auto claim_valid = [&]() -> int {
+    if (tid == 0) {
+      int x, it_, c_;
+      do {
+        x = atomicAdd(&ctrl[0], 1);
+      } while (x < E && !locate(p, x % p.NS, x / p.NS, &it_, &c_));
+      ss.claim = x;
+    }
+    __syncthreads();
+    const int x = ss.claim;
+    __syncthreads();
+    return x;
+  };
+  // TMA of claim x's K, Q (key head) and V (value head) tiles.
+  auto issue_tiles = [&](int x) {
+    if (tid != 0) return;
+    int it_, c_;
+    locate(p, x % p.NS, x / p.NS, &it_, &c_);
+    const int n_ = it_ / p.H_v, h_ = it_ % p.H_v, kh_ = h_ / (p.H_v / p.H_k);
+    int64_t a_, b_;
+    seq_chunks(p.cu, p.T, n_, &a_, &b_);
+    const int y = (int)(a_ + (int64_t)c_ * kChunk);
+    fence_proxy_async_smem();
+    mbar_arrive_expect_tx(&ss.bar_tma, 6 * 8192);
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+      tma_load_2d(kq + b * 16384, tm_k, kh_ * kHeadDim + b * 64, y, &ss.bar_tma);
+      tma_load_2d(kq + b * 16384 + 8192, tm_q, kh_ * kHeadDim + b * 64, y, &ss.bar_tma);
+      tma_load_2d(vv + b * 8192, tm_v, h_ * kHeadDim + b * 64, y, &ss.bar_tma);
+    }
+  };
+  // Completion of the last bulk store, then the release of its slot's flag.
+  int* pend_flag = nullptr;   // thread 0 only
+  int pend_val = 0;
+  auto publish = [&](int*& flag, int val) {
+    if (!flag) return;
+    bulk_wait_all();
+    fence_proxy_async_all();
+    st_release(flag, val);
+    flag = nullptr;
+  };
   uint32_t tma_par = 0, mma_par = 0;
+  int e = claim_valid();
+  bool tiles_pending = false;
+  if (e < E) {
+    issue_tiles(e);
+    tiles_pending = true;
+  }
   const uint32_t a_kq = smem_u32(kq), a_v = smem_u32(vv), a_t = smem_u32(sm + P_T);
   const uint32_t id_gram = idesc_bf16(128, 64, false, false);
   const uint32_t id_mn = idesc_bf16(128, 64, true, false);
@@ -215,6 +318,7 @@ __device__ void prep_role(const PcParams& p, const CUtensorMap* tm_q, const CUte
   while (e < E) {
     const int s = e % p.NS, r = e / p.NS;
     int item, c;
+    int e_next = (int)E;
     bool ok = true;
     if (locate(p, s, r, &item, &c)) {
       const int n = item / p.H_v, h = item % p.H_v, kh = h / (p.H_v / p.H_k);
@@ -223,16 +327,7 @@ __device__ void prep_role(const PcParams& p, const CUtensorMap* tm_q, const CUte
       const int64_t t0 = s0 + (int64_t)c * kChunk;
       const int L = (int)((s1 - t0) < kChunk ? (s1 - t0) : kChunk);
 
-      if (tid == 0) {
-        fence_proxy_async_smem();
-        mbar_arrive_expect_tx(&ss.bar_tma, 6 * 8192);
-#pragma unroll
-        for (int b = 0; b < 2; ++b) {
-          tma_load_2d(kq + b * 16384, tm_k, kh * kHeadDim + b * 64, (int)t0, &ss.bar_tma);
-          tma_load_2d(kq + b * 16384 + 8192, tm_q, kh * kHeadDim + b * 64, (int)t0, &ss.bar_tma);
-          tma_load_2d(vv + b * 8192, tm_v, h * kHeadDim + b * 64, (int)t0, &ss.bar_tma);
-        }
-      }
+      (void)kh;
       if (warp == 1) {   // gates: cumulative log-decay and derived vectors
         const Tg* g = static_cast<const Tg*>(p.g);
         const Tg* bt = static_cast<const Tg*>(p.beta);
@@ -271,6 +366,8 @@ __device__ void prep_role(const PcParams& p, const CUtensorMap* tm_q, const CUte
       }
       ok = mbar_wait_bounded(&ss.bar_tma, tma_par, kLimitNs);
       tma_par ^= 1;
+      if (ok) tiles_pending = false;
+      if (tid == 0) publish(pend_flag, pend_val);   // previous item's slot
       if (__syncthreads_or(!ok)) goto fail;
 
       if (L < kChunk) {   // rows past the sequence end hold other data: zero them
@@ -316,7 +413,7 @@ __device__ void prep_role(const PcParams& p, const CUtensorMap* tm_q, const CUte
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int s2 = 16 * cg + j;
-            Af[t * 65 + s2] = (s2 < t) ? bt * __expf(Gt - ss.G[s2]) * v[j] : 0.f;
+            Af[t * kLd + s2] = (s2 < t) ? bt * __expf(Gt - ss.G[s2]) * v[j] : 0.f;
           }
         } else {
           const int t = row - 64;
@@ -340,43 +437,31 @@ __device__ void prep_role(const PcParams& p, const CUtensorMap* tm_q, const CUte
       tc_fence_before();
       if (__syncthreads_or(!ok)) goto fail;
 
-      // ---- T = (I + A)^{-1}: 16x16 diagonal blocks, then block rows ----
+      // ---- T = (I + A)^{-1}: 8x8 diagonal blocks by forward substitution,
+      //      then pairwise merges 8 -> 16 -> 32 -> 64:  T21 = -T22 A21 T11 ----
+      for (int idx = tid; idx < 64 * kLd; idx += kPcThreads) Tf[idx] = 0.f;
+      __syncthreads();
       if (tid < 64) {
-        const int I = tid >> 4, j = tid & 15;
-        float x[16];
+        const int B = tid >> 3, j = tid & 7;
+        float a[8][8], x[8];
 #pragma unroll
-        for (int rr = 0; rr < 16; ++rr) {
+        for (int rr = 1; rr < 8; ++rr)
+#pragma unroll
+          for (int m = 0; m < rr; ++m) a[rr][m] = Af[(8 * B + rr) * kLd + 8 * B + m];
+#pragma unroll
+        for (int rr = 0; rr < 8; ++rr) {
           float acc = (rr == j) ? 1.f : 0.f;
 #pragma unroll
-          for (int m = 0; m < rr; ++m) acc = fmaf(-Af[(16 * I + rr) * 65 + 16 * I + m], x[m], acc);
+          for (int m = 0; m < rr; ++m) acc = fmaf(-a[rr][m], x[m], acc);
           x[rr] = acc;
         }
 #pragma unroll
-        for (int rr = 0; rr < 16; ++rr) Tf[(16 * I + rr) * 65 + 16 * I + j] = x[rr];
+        for (int rr = 0; rr < 8; ++rr) Tf[(8 * B + rr) * kLd + 8 * B + j] = x[rr];
       }
       __syncthreads();
-      for (int I = 1; I < 4; ++I) {
-        for (int task = tid; task < I * 256; task += kPcThreads) {
-          const int J = task >> 8, i = (task >> 4) & 15, j = task & 15;
-          float acc = 0.f;
-          for (int K = J; K < I; ++K) {
-#pragma unroll
-            for (int m = 0; m < 16; ++m)
-              acc = fmaf(Af[(16 * I + i) * 65 + 16 * K + m], Tf[(16 * K + m) * 65 + 16 * J + j], acc);
-          }
-          Xs[J * 256 + i * 16 + j] = acc;
-        }
-        __syncthreads();
-        for (int task = tid; task < I * 256; task += kPcThreads) {
-          const int J = task >> 8, i = (task >> 4) & 15, j = task & 15;
-          float acc = 0.f;
-#pragma unroll
-          for (int m = 0; m < 16; ++m)
-            acc = fmaf(Tf[(16 * I + i) * 65 + 16 * I + m], Xs[J * 256 + m * 16 + j], acc);
-          Tf[(16 * I + i) * 65 + 16 * J + j] = -acc;
-        }
-        __syncthreads();
-      }
+      merge_level<8>(Af, Tf, Xs, tid);
+      merge_level<16>(Af, Tf, Xs, tid);
+      merge_level<32>(Af, Tf, Xs, tid);
       // T' = T diag(beta e^G), T'' = T diag(beta) (unit diagonal included) as
       // bf16 hi/lo K-major B images [t][s]
       {
@@ -385,7 +470,7 @@ __device__ void prep_role(const PcParams& p, const CUtensorMap* tm_q, const CUte
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const int s2 = c8 * 8 + j;
-          const float val = (s2 < t) ? Tf[t * 65 + s2] : (s2 == t ? 1.f : 0.f);
+          const float val = (s2 < t) ? Tf[t * kLd + s2] : (s2 == t ? 1.f : 0.f);
           const float a = val * ss.bg[s2], b = val * ss.beta[s2];
           ph[j] = a;
           pl[j] = bf_lo(a);
@@ -422,6 +507,12 @@ __device__ void prep_role(const PcParams& p, const CUtensorMap* tm_q, const CUte
       __syncthreads();
       ok = ok && ss.ok;
       if (__syncthreads_or(!ok)) goto fail;
+      // the tiles are no longer read: prefetch the next claim's tiles
+      e_next = claim_valid();
+      if (e_next < E) {
+        issue_tiles(e_next);
+        tiles_pending = true;
+      }
       {
         uint8_t* slot = slot_of(p.ws, s, r);
         float v[16];
@@ -432,7 +523,7 @@ __device__ void prep_role(const PcParams& p, const CUtensorMap* tm_q, const CUte
         for (int q = 0; q < 2; ++q)
           *reinterpret_cast<uint4*>(stg + SL_WN + swz(row, 2 * cg + q)) = pack_half8(v + 8 * q);
         tmem_ld16(tmem + lane_base + PT_U + 16 * cg, v);
-        float* ut = reinterpret_cast<float*>(slot + SL_UT);
+        float* ut = reinterpret_cast<float*>(stg + SL_UT);
 #pragma unroll
         for (int j = 0; j < 16; ++j) ut[(16 * cg + j) * kHeadDim + row] = v[j];
         float* vec = reinterpret_cast<float*>(stg + SL_VEC);
@@ -444,26 +535,28 @@ __device__ void prep_role(const PcParams& p, const CUtensorMap* tm_q, const CUte
         if (tid == 64) vec[192] = ss.gL;
         fence_proxy_async_smem();
         tc_fence_before();
-        __threadfence();
         __syncthreads();
+        // one bulk store of the whole slot; its completion and the release of
+        // the slot's flag happen at the next item, after that item's tiles land
         if (tid == 0) {
-          bulk_s2g(slot, stg, SL_IMG);
+          bulk_s2g(slot, stg, SLOT_BYTES);
           bulk_commit();
-          bulk_wait_all();
-          fence_proxy_async_all();
-          __threadfence();
-          st_release(flags_of(p.ws, s) + (r % kRing), r + 1);
+          pend_flag = flags_of(p.ws, s) + (r % kRing);
+          pend_val = r + 1;
         }
       }
     }
-    if (tid == 0) ss.claim = atomicAdd(&ctrl[0], 1);
-    __syncthreads();
-    e = ss.claim;
+    e = e_next;
     if (ld_acquire(&ctrl[1]) != 0) break;
     continue;
   fail:
     if (tid == 0) atomicExch(&ctrl[1], 1);
     break;
+  }
+  if (tid == 0) {
+    if (tiles_pending) mbar_wait_bounded(&ss.bar_tma, tma_par, kLimitNs);
+    if (ld_acquire(&ctrl[1]) == 0) publish(pend_flag, pend_val);
+    else bulk_wait_all();
   }
   tc_fence_before();
   __syncthreads();
@@ -510,10 +603,11 @@ __device__ void state_role(const PcParams& p, uint8_t* sm, int s) {
   uint32_t par_dt = 0, par_p = 0, par_o = 0;
   bool ok = true;
   int r = 0;
-  auto issue_copy = [&](int step, bool block) -> bool {
+  // Copy the operand image of `step` into its buffer; unless `acquired`, first
+  // wait (bounded) for the producer's release of that slot.
+  auto issue_copy = [&](int step, bool acquired) -> bool {
     int* full = flags + (step % kRing);
-    if (!block && ld_acquire(full) < step + 1) return false;
-    if (block && !wait_flag_ge(full, step + 1, &ctrl[1], kLimitNs)) return false;
+    if (!acquired && !wait_flag_ge(full, step + 1, &ctrl[1], kLimitNs)) return false;
     fence_proxy_async_all();
     uint64_t* bar = &ss.bar_slot[step & 1];
     mbar_arrive_expect_tx(bar, SL_IMG);
@@ -548,12 +642,15 @@ __device__ void state_role(const PcParams& p, uint8_t* sm, int s) {
       const uint32_t a_buf = smem_u32(buf);
       const int64_t t0 = s0 + (int64_t)c * kChunk;
       const int L = (int)((s1 - t0) < kChunk ? (s1 - t0) : kChunk);
-      if (tid == 0) {
+      int poll = 0;
+      if (tid == 32) {
         ss.ok = 1;
         if (issued == r) {
-          if (issue_copy(r, true)) issued = r + 1;
+          if (issue_copy(r, false)) issued = r + 1;
           else ss.ok = 0;
         }
+        // early, non-blocking look at the next slot's flag (consumed after the readout)
+        if (issued == r + 1 && r + 1 < total) poll = ld_relaxed(flags + ((r + 1) % kRing));
       }
       __syncthreads();
       if (!ss.ok) { ok = false; break; }
@@ -566,7 +663,7 @@ __device__ void state_role(const PcParams& p, uint8_t* sm, int s) {
       }
       if (!mbar_wait_bounded(&ss.bar_slot[b], (uint32_t)((r >> 1) & 1), kLimitNs)) ok = false;
       if (__syncthreads_or(!ok)) { ok = false; break; }
-      // ---- OA = S0 Q^T and Delta^T = S0 (-W^T) ----
+      // ---- Delta^T = S0 (-W^T) (critical path) ----
       if (tid == 0) {
         tc_fence_after();
 #pragma unroll
@@ -575,6 +672,8 @@ __device__ void state_role(const PcParams& p, uint8_t* sm, int s) {
           mma_f16(tmem + ST_DT, a, sw128_desc(a_buf + SL_WN + kk * 2048, 16384, 1024), id_mnb,
                   kk > 0);
         }
+        mma_commit(&ss.bar_dt);
+        // OA = S0 Q^T runs while the Delta readout proceeds; P's commit covers it
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint64_t a = sw128_desc(a_s0 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
@@ -582,7 +681,6 @@ __device__ void state_role(const PcParams& p, uint8_t* sm, int s) {
                   sw128_desc(a_buf + SL_QF + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id_kk,
                   kk > 0);
         }
-        mma_commit(&ss.bar_dt);
       }
       if (!mbar_wait_bounded(&ss.bar_dt, par_dt, kLimitNs)) ok = false;
       par_dt ^= 1;
@@ -611,8 +709,8 @@ __device__ void state_role(const PcParams& p, uint8_t* sm, int s) {
       tc_fence_before();
       if (__syncthreads_or(!ok)) { ok = false; break; }
       // ---- P = Delta~^T K (critical), then OB = Delta^T M^T (hi/lo) ----
+      if (tid == 32) st_release(flags + kRing, r + 1);   // slot r fully read
       if (tid == 0) {
-        st_release(flags + kRing, r + 1);      // slot r fully read
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
@@ -628,8 +726,12 @@ __device__ void state_role(const PcParams& p, uint8_t* sm, int s) {
           mma_f16(tmem + ST_OB, sw128_desc(a_dth + ks * 32, 16, 1024), ml, id_kk, 1);
         }
         mma_commit(&ss.bar_o);
-        // prefetch the next step's slot into the other buffer if it is ready
-        if (issued == r + 1 && r + 1 < total && issue_copy(r + 1, false)) issued = r + 2;
+      }
+      // prefetch the next step's slot into the other buffer if it was ready
+      if (tid == 32 && issued == r + 1 && r + 1 < total && poll >= r + 2) {
+        fence_acq_rel_gpu();
+        issue_copy(r + 1, true);
+        issued = r + 2;
       }
       if (!mbar_wait_bounded(&ss.bar_p, par_p, kLimitNs)) ok = false;
       par_p ^= 1;
@@ -676,7 +778,7 @@ __device__ void state_role(const PcParams& p, uint8_t* sm, int s) {
   }
   if (!ok && tid == 0) atomicExch(&ctrl[1], 1);
   // drain our own copies before leaving (bounded)
-  if (tid == 0)
+  if (tid == 32)
     for (int st = r; st < issued; ++st)
       mbar_wait_bounded(&ss.bar_slot[st & 1], (uint32_t)((st >> 1) & 1), kLimitNs);
   tc_fence_before();

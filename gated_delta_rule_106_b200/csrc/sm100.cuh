@@ -108,6 +108,15 @@ __device__ __forceinline__ int ld_acquire(const int* p) {
   asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
+__device__ __forceinline__ int ld_relaxed(const int* p) {
+  int v;
+  asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+// Acquire side of a release store observed by a relaxed load.
+__device__ __forceinline__ void fence_acq_rel_gpu() {
+  asm volatile("fence.acq_rel.gpu;" ::: "memory");
+}
 // Spin until *p >= target, for at most limit_ns. Returns false on timeout or
 // when *abort becomes non-zero.
 __device__ __forceinline__ bool wait_flag_ge(const int* p, int target, const int* abort,
