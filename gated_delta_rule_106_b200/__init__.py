@@ -22,7 +22,8 @@ import torch
 
 __all__ = ["GDN_BF16", "GDN_F32", "GdnError", "library_path", "load",
            "gdn_conv1d_silu", "gdn_chunked_prefill",
-           "gdn_chunked_prefill_workspace", "gdn_decode_step",
+           "gdn_chunked_prefill_workspace", "gdn_chunked_prefill_noalloc",
+           "gdn_decode_step",
            "gdn_gated_rmsnorm", "gdn_status_string", "gdn_version",
            "H_K", "H_V", "HEAD_DIM", "CHUNK"]
 
@@ -51,6 +52,10 @@ _SIGNATURES = {
                                    _int, _f32, _vp, _int, _vp, ctypes.c_size_t,
                                    _vp]),
     "gdn_chunked_prefill_workspace": (ctypes.c_size_t, [_int, _i64, _int, _int]),
+    "gdn_chunked_prefill_noalloc": (_int, [_vp, _vp, _vp, _int, _i64, _i64, _i64, _vp,
+                                           _vp, _int, _vp, _vp, _vp, _int, _i64, _int,
+                                           _int, _f32, _vp, _int, _vp]),
+    "gdn_chunked_prefill_noalloc_scratch_bytes": (ctypes.c_size_t, []),
     "gdn_decode_step": (_int, [_vp, _vp, _vp, _int, _i64, _i64, _i64, _vp, _vp,
                                _int, _vp, _int, _int, _int, _f32, _vp, _int,
                                _vp]),
@@ -178,6 +183,25 @@ def gdn_chunked_prefill(q, k, v, g, beta, cu_seqlens, *, state_in=None,
         _ptr(state_in), _ptr(state_out), _ptr(cu_seqlens), N, T, H_k, H_v,
         scale, _ptr(o), _dtype_code(o.dtype), _ptr(workspace), ws_bytes,
         _stream(stream, v.device)))
+    return o
+
+
+def gdn_chunked_prefill_noalloc(q, k, v, g, beta, cu_seqlens, *, state_in=None,
+                                state_out=None, scale=1.0, o=None, o_dtype=None,
+                                stream=None):
+    """gdn_chunked_prefill working in the library's own static device scratch
+    instead of a caller-provided workspace (for callers that cannot allocate
+    at the call site). Calls that overlap on the GPU must not share it."""
+    T, H_k, _ = q.shape
+    H_v = v.shape[1]
+    N = cu_seqlens.numel() - 1
+    if o is None:
+        o = torch.empty((T, H_v, HEAD_DIM), dtype=o_dtype or v.dtype, device=v.device)
+    _check("gdn_chunked_prefill_noalloc", load().gdn_chunked_prefill_noalloc(
+        _ptr(q), _ptr(k), _ptr(v), _dtype_code(q.dtype), _row_stride(q),
+        _row_stride(k), _row_stride(v), _ptr(g), _ptr(beta), _dtype_code(g.dtype),
+        _ptr(state_in), _ptr(state_out), _ptr(cu_seqlens), N, T, H_k, H_v,
+        scale, _ptr(o), _dtype_code(o.dtype), _stream(stream, v.device)))
     return o
 
 

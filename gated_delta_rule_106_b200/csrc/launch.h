@@ -47,5 +47,8 @@ cudaError_t launch_prefill_stepwise(const RecurArgs& a);
 // kernel over all SMs; needs prefill_pc_workspace() bytes of workspace.
 cudaError_t launch_prefill_pc(const RecurArgs& a);
 size_t prefill_pc_workspace(int N, int64_t T_total, int H_v);
+// The same kernel on the library-owned static scratch (no workspace argument).
+cudaError_t launch_prefill_pc_noalloc(const RecurArgs& a);
+size_t prefill_noalloc_scratch_bytes();
 
 }  // namespace gdn

@@ -35,6 +35,8 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <mutex>
+
 #include "gdn_common.cuh"
 #include "launch.h"
 #include "sm100.cuh"
@@ -879,7 +881,47 @@ int state_ctas(int64_t items, int H_v, int nsm) {
   return base;
 }
 
+// ---- library-owned scratch for callers that cannot allocate --------------
+// Room for the rings of 49 state CTAs (a third of a 148-SM B200). Every GPU
+// that loads the library holds this array until the process exits.
+constexpr int kNoAllocStateCtas = 49;
+constexpr size_t kNoAllocScratchBytes =
+    CTRL_BYTES + (size_t)kNoAllocStateCtas * kRing * SLOT_BYTES;   // 14 617 600 B
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device (the host-side symbol is only a stand-in, never a device address).
+cudaError_t noalloc_scratch(void** out) {
+  static std::mutex mu;
+  static void* addr[256] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 256) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    addr[dev] = ptr;
+  }
+  *out = addr[dev];
+  return cudaSuccess;
+}
+
 }  // namespace
+
+size_t prefill_noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
+
+cudaError_t launch_prefill_pc_noalloc(const RecurArgs& args) {
+  void* scratch = nullptr;
+  cudaError_t e = noalloc_scratch(&scratch);
+  if (e != cudaSuccess) return e;
+  RecurArgs a = args;
+  a.workspace = scratch;
+  a.workspace_bytes = kNoAllocScratchBytes;
+  return launch_prefill_pc(a);
+}
 
 size_t prefill_pc_workspace(int N, int64_t T_total, int H_v) {
   const int nsm = sm_count();

@@ -147,6 +147,42 @@ gdn_status gdn_chunked_prefill(const void* q, const void* k, const void* v,
 size_t gdn_chunked_prefill_workspace(int N, int64_t T_total, int H_k, int H_v);
 
 /*
+ * gdn_chunked_prefill_noalloc -- gdn_chunked_prefill with no workspace
+ * argument: the library supplies the working memory itself. It is meant for
+ * callers that cannot hand the library device memory at the call site -- for
+ * example an operator plugged into a host framework whose allocator the plugin
+ * cannot reach, or a serving loop whose memory plan forbids any allocation
+ * after start-up. The pages have no counterpart to this call; it exists only
+ * for such callers.
+ *
+ * Arguments, results and numerics are those of gdn_chunked_prefill. The
+ * working memory is one static device array of
+ * gdn_chunked_prefill_noalloc_scratch_bytes() bytes (14 617 600: the chunk
+ * rings of 49 state CTAs) that every GPU which loads the library holds until
+ * the process exits. A problem whose working memory would exceed it returns
+ * GDN_ERR_UNSUPPORTED without launching (on a 148-SM B200 none does). The
+ * call itself never allocates or frees memory.
+ * The first call on a device looks up the array's device address with that
+ * device current; make that first call before any stream capture begins.
+ * Every call uses the same array and leaves its contents behind (the next
+ * call clears what must start at zero): calls whose executions overlap on the
+ * GPU -- on different streams or from different host threads -- race and give
+ * undefined results.
+ */
+gdn_status gdn_chunked_prefill_noalloc(const void* q, const void* k, const void* v,
+                                       gdn_dtype qkv_dtype, int64_t q_row_stride,
+                                       int64_t k_row_stride, int64_t v_row_stride,
+                                       const void* g, const void* beta,
+                                       gdn_dtype gate_dtype, const float* state_in,
+                                       float* state_out, const int32_t* cu_seqlens,
+                                       int N, int64_t T_total, int H_k, int H_v,
+                                       float scale, void* o, gdn_dtype o_dtype,
+                                       cudaStream_t stream);
+
+/* Bytes of the static device array gdn_chunked_prefill_noalloc works in. */
+size_t gdn_chunked_prefill_noalloc_scratch_bytes(void);
+
+/*
  * gdn_decode_step -- one stepwise update of the gated delta rule for N
  * sequences, one token each (the stepwise decode path of [P2 二.1]):
  *   S <- g S (I - beta k k^T) + beta v k^T ;  o = scale * S q
