@@ -14,15 +14,19 @@
 //
 // One cooperative launch, one CTA per SM, two roles:
 //  * state CTAs (about a third of the SMs) each own a list of (sequence,
-//    value head) items and run their chunks in order: per chunk two tcgen05
-//    MMAs on the critical path (Delta^T = U^T - S0 W^T, then P = Delta~^T K),
-//    the fp32 state in registers (four threads per row), outputs from
-//    S0 Q^T and Delta^T M^T.
+//    value head) items and run their chunks in order. Per chunk two wide
+//    tcgen05 MMAs form the critical path: D1 = S0 [-W ; Q]^T (N = 128: the
+//    S0 part of Delta and S0 Q^T together), then D2 = Delta^T [K~ | M^T]
+//    (N = 256: the state update P = Delta^T diag(e^{G_L-G}) K and the M Delta
+//    output term together); the fp32 state stays in registers (four threads
+//    per row). Few wide MMAs matter because each tcgen05.mma instruction
+//    costs about the same time whether N is 64 or 128.
 //  * prep CTAs claim (item, chunk) work in chunk order from a global counter
 //    and compute the state-free part: bf16 TMA tiles of K, Q, V; the Gram
-//    [K;Q] K^T on the tensor cores (bf16, exact products); decays; the UT
-//    solve in fp32; W and U as bf16 hi/lo MMAs (~17 significant bits, unit
-//    diagonal included); binary16 images of -W, K, Q and M (hi/lo). They
+//    [K;Q][K;Q]^T on the tensor cores (bf16, exact products: K K^T for A and
+//    K Q^T for M^T); decays; the UT solve in fp32; W and U as bf16 hi/lo MMAs
+//    (~17 significant bits, unit diagonal included); binary16 images of
+//    [-W ; Q], [K~ | M^T hi | M^T lo] and U^T in fp32. They
 //    publish one chunk per ring slot in the caller's workspace (3 slots per
 //    state CTA, ~97 KB each, L2-resident) with a release flag; the state CTA
 //    acquires it, bulk-copies the operand images into shared memory and
@@ -51,11 +55,13 @@ constexpr int kRing = 3;
 constexpr uint64_t kLimitNs = 2000000000ull;
 
 // ---- ring slot (global), 1024-aligned sections ---------------------------
-constexpr uint32_t SL_WN = 0;          // -W binary16, MN-major B image [128 d_k][64 t]
-constexpr uint32_t SL_KF = 16384;      // K binary16 image [2 blocks][64 t][64]
-constexpr uint32_t SL_QF = 32768;      // Q binary16 image [2 blocks][64 t][64]
-constexpr uint32_t SL_MH = 49152;      // M strictly lower, binary16 high part [64 t][64 s]
-constexpr uint32_t SL_ML = 57344;      // low part
+// B operand of S0 [-W ; Q]^T: K-major, [2 d_k blocks][128 rows][64], rows 0-63 = -W
+// (token t), rows 64-127 = Q (token t), binary16.
+constexpr uint32_t SL_WQ = 0;
+// B operand of Delta^T [K~ | M^T hi | M^T lo]: MN-major, four 64-column blocks of
+// [64 tokens s][64] at 8 KB stride: K~ = diag(e^{G_L-G}) K (d_k 0-63, 64-127), then the
+// strictly lower M transposed (M^T[s][t] = M_ts for t > s) as binary16 high and low parts.
+constexpr uint32_t SL_BKM = 32768;
 constexpr uint32_t SL_VEC = 65536;     // gamma[64] tail[64] mdiag[64] gL
 constexpr uint32_t SL_IMG = 66560;     // bytes of the shared-memory image above
 constexpr uint32_t SL_UT = 66560;      // U^T fp32 [64 t][128 i] (the consumer reads it from L2)
@@ -78,14 +84,17 @@ constexpr uint32_t S_BUF = 0;          // 2 x slot image
 constexpr uint32_t S_S0 = 133120;      // binary16 state, K-major [2 blocks][128 rows]
 constexpr uint32_t S_DTH = 165888;     // Delta^T high, K-major A [128][64 t]
 constexpr uint32_t S_DTL = 182272;     // Delta^T low
-constexpr uint32_t S_DKF = 198656;     // Delta~^T
 constexpr uint32_t S_SMALL = 215040;
-constexpr uint32_t PC_SMEM_BYTES = P_SMALL + 2048;
+constexpr uint32_t PC_SMEM_BYTES = P_SMALL + 4096;
 constexpr uint32_t PC_SMEM_ALLOC = PC_SMEM_BYTES + 1024;
 
 // TMEM columns
-constexpr uint32_t PT_GR = 0, PT_W = 64, PT_U = 128, PT_COLS = 256;      // prep
-constexpr uint32_t ST_DT = 0, ST_P = 64, ST_OA = 192, ST_OB = 256, ST_COLS = 512;  // state
+// prep: Gram [128 x 128]; W^T and U^T each as [hi part | lo part] column halves
+constexpr uint32_t PT_GR = 0, PT_W = 128, PT_U = 256, PT_COLS = 512;
+// state: D1 = S0 [-W ; Q]^T -> [Delta^T - U^T | S0 Q^T];
+//        D2 = Delta_hi^T [K~ | M^T hi | M^T lo] -> [P | OB_hh | OB_hl]; D3 = Delta_lo^T M^T hi
+constexpr uint32_t ST_D1 = 0, ST_OA = 64, ST_D2 = 128, ST_OBHH = 256, ST_OBHL = 320,
+                   ST_D3 = 384, ST_COLS = 512;
 
 struct PcParams {
   const void* g; const void* beta;
@@ -96,7 +105,9 @@ struct PcParams {
   int NS;               // state CTAs
 };
 
+constexpr int kCuCache = 513;   // sequences whose boundaries the prep CTAs keep on chip
 struct PrepSmall {
+  int cu[kCuCache];
   float G[64], beta[64], gamma[64], bg[64], tail[64], mdiag[64];
   float gL;
   int claim;
@@ -121,18 +132,44 @@ __device__ __forceinline__ uint4 pack_half8(const float* f) {
   for (int i = 0; i < 4; ++i) h[i] = __floats2half2_rn(f[2 * i], f[2 * i + 1]);
   return u;
 }
-__device__ __forceinline__ uint4 pack_bf8(const float* f) {
-  uint4 u;
-  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+// hi/lo splits without round trips through the conversion unit (its
+// throughput is a fraction of the ALU's): float(hi) is rebuilt from the bits.
+// bf16 round-to-nearest-even with integer operations (finite inputs).
+__device__ __forceinline__ uint32_t bf16_bits_rn(float x) {
+  uint32_t u = __float_as_uint(x);
+  u += 0x7fffu + ((u >> 16) & 1u);
+  return u >> 16;
+}
+// 8 values -> bf16 high parts and bf16 low parts (x - hi), packed
+__device__ __forceinline__ void split_bf8(const float* f, uint4& hi, uint4& lo) {
+  uint32_t h[8], l[8];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
-  return u;
+  for (int j = 0; j < 8; ++j) {
+    h[j] = bf16_bits_rn(f[j]);
+    l[j] = bf16_bits_rn(f[j] - __uint_as_float(h[j] << 16));
+  }
+  hi = make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16), h[6] | (h[7] << 16));
+  lo = make_uint4(l[0] | (l[1] << 16), l[2] | (l[3] << 16), l[4] | (l[5] << 16), l[6] | (l[7] << 16));
 }
-__device__ __forceinline__ float half_lo(float x) {
-  return x - __half2float(__float2half_rn(x));
+// value of a finite binary16 given by its bits (low 16 bits of hb); exact
+__device__ __forceinline__ float half_bits_value(uint32_t hb) {
+  const float mag = __uint_as_float((hb & 0x7fffu) << 13) * 5.192296858534828e33f;  // * 2^112
+  return __uint_as_float(__float_as_uint(mag) | ((hb & 0x8000u) << 16));
 }
-__device__ __forceinline__ float bf_lo(float x) {
-  return x - __bfloat162float(__float2bfloat16_rn(x));
+// 8 values -> binary16 high parts and binary16 low parts (x - hi), packed
+__device__ __forceinline__ void split_half8(const float* f, uint4& hi, uint4& lo) {
+  uint32_t hw[4], lw[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __half2 h2 = __floats2half2_rn(f[2 * i], f[2 * i + 1]);
+    const uint32_t hb = *reinterpret_cast<const uint32_t*>(&h2);
+    const __half2 l2 = __floats2half2_rn(f[2 * i] - half_bits_value(hb & 0xffffu),
+                                         f[2 * i + 1] - half_bits_value(hb >> 16));
+    hw[i] = hb;
+    lw[i] = *reinterpret_cast<const uint32_t*>(&l2);
+  }
+  hi = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+  lo = make_uint4(lw[0], lw[1], lw[2], lw[3]);
 }
 
 __device__ __forceinline__ int* flags_of(uint8_t* ws, int s) {
@@ -145,23 +182,23 @@ __device__ __forceinline__ uint8_t* slot_of(uint8_t* ws, int s, int r) {
 // chunks of sequence n (clamped cu_seqlens)
 __device__ __forceinline__ int seq_chunks(const int32_t* cu, int64_t T, int n, int64_t* s0,
                                           int64_t* s1) {
-  int64_t a = clamp_t(__ldg(cu + n), T), b = clamp_t(__ldg(cu + n + 1), T);
+  int64_t a = clamp_t(cu[n], T), b = clamp_t(cu[n + 1], T);
   if (b < a) b = a;
   *s0 = a;
   *s1 = b;
   return (int)((b - a + kChunk - 1) / kChunk);
 }
-__device__ int steps_of(const PcParams& p, int s) {
+__device__ int steps_of(const PcParams& p, const int32_t* cu, int s) {
   int total = 0;
   int64_t a, b;
-  for (int i = s; i < p.N * p.H_v; i += p.NS) total += seq_chunks(p.cu, p.T, i / p.H_v, &a, &b);
+  for (int i = s; i < p.N * p.H_v; i += p.NS) total += seq_chunks(cu, p.T, i / p.H_v, &a, &b);
   return total;
 }
 // step r of state CTA s -> item i and chunk c (false if r is past its steps)
-__device__ bool locate(const PcParams& p, int s, int r, int* item, int* chunk) {
+__device__ bool locate(const PcParams& p, const int32_t* cu, int s, int r, int* item, int* chunk) {
   int64_t a, b;
   for (int i = s; i < p.N * p.H_v; i += p.NS) {
-    const int nc = seq_chunks(p.cu, p.T, i / p.H_v, &a, &b);
+    const int nc = seq_chunks(cu, p.T, i / p.H_v, &a, &b);
     if (r < nc) {
       *item = i;
       *chunk = r;
@@ -179,52 +216,74 @@ __device__ bool locate(const PcParams& p, int s, int r, int* item, int* chunk) {
 // outputs.
 template <int b>
 __device__ __forceinline__ void merge_level(const float* Af, float* Tf, float* Xs, int tid) {
-  constexpr int bb = b * b, pairs = 64 / (2 * b), outs = pairs * bb;
-  constexpr int per = outs / kPcThreads > 0 ? outs / kPcThreads : 1;   // 1 or 2 adjacent columns
-  constexpr int threads = outs / per;
+  // Each active thread makes an RI x 2 block of outputs (rows i..i+RI-1,
+  // columns j, j+1): row segments of A / T are read four floats at a time and
+  // column pairs of T / X two at a time, so loads per FMA stay low.
+  constexpr int bb = b * b, pairs = 64 / (2 * b);
+  constexpr int RI = b >= 32 ? 4 : 2, RJ = 2;
+  constexpr int tiles_i = b / RI, tiles_j = b / RJ;
+  constexpr int threads = pairs * tiles_i * tiles_j;   // b=8: 64, 16: 128, 32: 128
+  static_assert(threads <= kPcThreads, "too many threads");
+  const int pr = tid / (tiles_i * tiles_j);
+  const int ti = (tid / tiles_j) % tiles_i, tj = tid % tiles_j;
+  const int i0 = ti * RI, j0 = tj * RJ, o = 2 * b * pr;
   if (tid < threads) {
-    const int idx = tid * per;
-    const int pr = idx / bb, i = (idx / b) % b, j = idx % b, o = 2 * b * pr;
-    const float4* arow = reinterpret_cast<const float4*>(Af + (o + b + i) * kLd + o);
-    float acc[per][2];
+    float acc[RI][RJ];
 #pragma unroll
-    for (int c = 0; c < per; ++c) acc[c][0] = acc[c][1] = 0.f;
+    for (int a = 0; a < RI; ++a)
+#pragma unroll
+      for (int c = 0; c < RJ; ++c) acc[a][c] = 0.f;
 #pragma unroll
     for (int m4 = 0; m4 < b / 4; ++m4) {
-      const float4 a = arow[m4];
-      const float av[4] = {a.x, a.y, a.z, a.w};
+      float av[RI][4];
+#pragma unroll
+      for (int a = 0; a < RI; ++a) {
+        const float4 v = reinterpret_cast<const float4*>(Af + (o + b + i0 + a) * kLd + o)[m4];
+        av[a][0] = v.x; av[a][1] = v.y; av[a][2] = v.z; av[a][3] = v.w;
+      }
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const float* tr = Tf + (o + 4 * m4 + u) * kLd + o + j;
+        const float2 t2 = *reinterpret_cast<const float2*>(Tf + (o + 4 * m4 + u) * kLd + o + j0);
 #pragma unroll
-        for (int c = 0; c < per; ++c) acc[c][u & 1] = fmaf(av[u], tr[c], acc[c][u & 1]);
+        for (int a = 0; a < RI; ++a) {
+          acc[a][0] = fmaf(av[a][u], t2.x, acc[a][0]);
+          acc[a][1] = fmaf(av[a][u], t2.y, acc[a][1]);
+        }
       }
     }
 #pragma unroll
-    for (int c = 0; c < per; ++c) Xs[idx + c] = acc[c][0] + acc[c][1];
+    for (int a = 0; a < RI; ++a)
+      *reinterpret_cast<float2*>(Xs + pr * bb + (i0 + a) * b + j0) = make_float2(acc[a][0], acc[a][1]);
   }
   __syncthreads();
   if (tid < threads) {
-    const int idx = tid * per;
-    const int pr = idx / bb, i = (idx / b) % b, j = idx % b, o = 2 * b * pr;
-    const float4* trow = reinterpret_cast<const float4*>(Tf + (o + b + i) * kLd + o + b);
-    const float* xcol = Xs + pr * bb + j;
-    float acc[per][2];
+    float acc[RI][RJ];
 #pragma unroll
-    for (int c = 0; c < per; ++c) acc[c][0] = acc[c][1] = 0.f;
+    for (int a = 0; a < RI; ++a)
+#pragma unroll
+      for (int c = 0; c < RJ; ++c) acc[a][c] = 0.f;
 #pragma unroll
     for (int m4 = 0; m4 < b / 4; ++m4) {
-      const float4 t4 = trow[m4];
-      const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
+      float tv[RI][4];
+#pragma unroll
+      for (int a = 0; a < RI; ++a) {
+        const float4 v = reinterpret_cast<const float4*>(Tf + (o + b + i0 + a) * kLd + o + b)[m4];
+        tv[a][0] = v.x; tv[a][1] = v.y; tv[a][2] = v.z; tv[a][3] = v.w;
+      }
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const float* xr = xcol + (4 * m4 + u) * b;
+        const float2 x2 = *reinterpret_cast<const float2*>(Xs + pr * bb + (4 * m4 + u) * b + j0);
 #pragma unroll
-        for (int c = 0; c < per; ++c) acc[c][u & 1] = fmaf(tv[u], xr[c], acc[c][u & 1]);
+        for (int a = 0; a < RI; ++a) {
+          acc[a][0] = fmaf(tv[a][u], x2.x, acc[a][0]);
+          acc[a][1] = fmaf(tv[a][u], x2.y, acc[a][1]);
+        }
       }
     }
 #pragma unroll
-    for (int c = 0; c < per; ++c) Tf[(o + b + i) * kLd + o + j + c] = -(acc[c][0] + acc[c][1]);
+    for (int a = 0; a < RI; ++a)
+      *reinterpret_cast<float2*>(Tf + (o + b + i0 + a) * kLd + o + j0) =
+          make_float2(-acc[a][0], -acc[a][1]);
   }
   __syncthreads();
 }
@@ -261,16 +320,22 @@ __device__ void prep_role(const PcParams& p, const CUtensorMap* tm_q, const CUte
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ss.tmem;
-  for (int s = tid; s < p.NS; s += kPcThreads) atomicMax(&ss.max_steps, steps_of(p, s));
+  const bool cu_on_chip = p.N + 1 <= kCuCache;
+  if (cu_on_chip)
+    for (int i = tid; i <= p.N; i += kPcThreads) ss.cu[i] = __ldg(p.cu + i);
+  __syncthreads();
+  const int32_t* cu = cu_on_chip ? ss.cu : p.cu;
+  for (int s = tid; s < p.NS; s += kPcThreads) atomicMax(&ss.max_steps, steps_of(p, cu, s));
   __syncthreads();
   const int64_t E = (int64_t)p.NS * ss.max_steps;
   // Claim the next (state CTA, step) that exists: thread 0 claims, all read.
+  int early = -1;   // thread 0: a claim taken ahead of its use (hides the atomic's latency)
   auto claim_valid = [&]() -> int {
     if (tid == 0) {
-      int x, it_, c_;
-      do {
-        x = atomicAdd(&ctrl[0], 1);
-      } while (x < E && !locate(p, x % p.NS, x / p.NS, &it_, &c_));
+      int x = early >= 0 ? early : atomicAdd(&ctrl[0], 1);
+      early = -1;
+      int it_, c_;
+      while (x < E && !locate(p, cu, x % p.NS, x / p.NS, &it_, &c_)) x = atomicAdd(&ctrl[0], 1);
       ss.claim = x;
     }
     __syncthreads();
@@ -282,10 +347,10 @@ __device__ void prep_role(const PcParams& p, const CUtensorMap* tm_q, const CUte
   auto issue_tiles = [&](int x) {
     if (tid != 0) return;
     int it_, c_;
-    locate(p, x % p.NS, x / p.NS, &it_, &c_);
+    locate(p, cu, x % p.NS, x / p.NS, &it_, &c_);
     const int n_ = it_ / p.H_v, h_ = it_ % p.H_v, kh_ = h_ / (p.H_v / p.H_k);
     int64_t a_, b_;
-    seq_chunks(p.cu, p.T, n_, &a_, &b_);
+    seq_chunks(cu, p.T, n_, &a_, &b_);
     const int y = (int)(a_ + (int64_t)c_ * kChunk);
     fence_proxy_async_smem();
     mbar_arrive_expect_tx(&ss.bar_tma, 6 * 8192);
@@ -314,18 +379,19 @@ __device__ void prep_role(const PcParams& p, const CUtensorMap* tm_q, const CUte
     tiles_pending = true;
   }
   const uint32_t a_kq = smem_u32(kq), a_v = smem_u32(vv), a_t = smem_u32(sm + P_T);
-  const uint32_t id_gram = idesc_bf16(128, 64, false, false);
-  const uint32_t id_mn = idesc_bf16(128, 64, true, false);
+  const uint32_t id_gram = idesc_bf16(128, 128, false, false);
+  const uint32_t id_mn = idesc_bf16(128, 128, true, false);
 
   while (e < E) {
     const int s = e % p.NS, r = e / p.NS;
     int item, c;
     int e_next = (int)E;
     bool ok = true;
-    if (locate(p, s, r, &item, &c)) {
+    if (tid == 0) early = atomicAdd(&ctrl[0], 1);
+    if (locate(p, cu, s, r, &item, &c)) {
       const int n = item / p.H_v, h = item % p.H_v, kh = h / (p.H_v / p.H_k);
       int64_t s0, s1;
-      seq_chunks(p.cu, p.T, n, &s0, &s1);
+      seq_chunks(cu, p.T, n, &s0, &s1);
       const int64_t t0 = s0 + (int64_t)c * kChunk;
       const int L = (int)((s1 - t0) < kChunk ? (s1 - t0) : kChunk);
 
@@ -383,7 +449,8 @@ __device__ void prep_role(const PcParams& p, const CUtensorMap* tm_q, const CUte
         fence_proxy_async_smem();
         __syncthreads();
       }
-      // ---- Gram [K;Q] K^T (bf16, exact products) ----
+      // ---- Gram [K;Q][K;Q]^T (bf16, exact products): rows 0-63 give K K^T and
+      //      K Q^T (the transposed query-key products) ----
       if (tid == 0) {
         tc_fence_after();
 #pragma unroll
@@ -394,45 +461,61 @@ __device__ void prep_role(const PcParams& p, const CUtensorMap* tm_q, const CUte
         }
         mma_commit(&ss.bar_mma);
       }
-      // K, Q -> binary16 images for the state CTA (overlaps the MMA)
-      for (int idx = tid; idx < 2048; idx += kPcThreads) {
-        const int which = idx >> 10, b = (idx >> 9) & 1, x = idx & 511;
-        const uint8_t* src = kq + b * 16384 + which * 8192 + x * 16;
-        float f[8];
-        load8(reinterpret_cast<const __nv_bfloat16*>(src), f);
-        *reinterpret_cast<uint4*>(stg + (which ? SL_QF : SL_KF) + b * 8192 + x * 16) =
-            pack_half8(f);
-      }
       ok = mbar_wait_bounded(&ss.bar_mma, mma_par, kLimitNs);
       mma_par ^= 1;
       tc_fence_after();
-      {
-        float v[16];
-        tmem_ld16(tmem + lane_base + PT_GR + 16 * cg, v);
-        if (row < 64) {
-          const int t = row;
-          const float Gt = ss.G[t], bt = ss.beta[t];
+      if (q4 < 2) {
+        // lanes 0-63 (key token s): A[s][x] = beta_s e^{G_s-G_x} k_s.k_x (x < s) from
+        // columns 0-63, and M^T[s][t] = e^{G_t-G_s} q_t.k_s (t > s) from columns 64-127
+        const int s2 = row, c0 = 32 * cg;
+        float v[32];
+        tmem_ld32(tmem + lane_base + PT_GR + c0, v);
+        const float Gs = ss.G[s2];
+        if (c0 < 64) {
+          const float bs = ss.beta[s2];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int s2 = 16 * cg + j;
-            Af[t * kLd + s2] = (s2 < t) ? bt * __expf(Gt - ss.G[s2]) * v[j] : 0.f;
+          for (int j = 0; j < 32; j += 4) {
+            float a4[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int x = c0 + j + u;
+              a4[u] = (x < s2) ? bs * __expf(Gs - ss.G[x]) * v[j + u] : 0.f;
+            }
+            *reinterpret_cast<float4*>(Af + s2 * kLd + c0 + j) = make_float4(a4[0], a4[1], a4[2], a4[3]);
           }
         } else {
-          const int t = row - 64;
-          const float Gt = ss.G[t];
-          float mh[16], ml[16];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int s2 = 16 * cg + j;
-            const float val = (s2 <= t) ? __expf(Gt - ss.G[s2]) * v[j] : 0.f;
-            if (s2 == t) ss.mdiag[t] = val;
-            mh[j] = (s2 < t) ? val : 0.f;
-            ml[j] = half_lo(mh[j]);
+          for (int q = 0; q < 4; ++q) {
+            float mh[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const int t = c0 - 64 + 8 * q + u;
+              const float val = (t >= s2) ? __expf(ss.G[t] - Gs) * v[8 * q + u] : 0.f;
+              if (t == s2) ss.mdiag[s2] = val;
+              mh[u] = (t > s2) ? val : 0.f;
+            }
+            const int c8 = (c0 - 64) / 8 + q;
+            uint4 hi, lo;
+            split_half8(mh, hi, lo);
+            *reinterpret_cast<uint4*>(stg + SL_BKM + 2 * 8192 + swz(s2, c8)) = hi;
+            *reinterpret_cast<uint4*>(stg + SL_BKM + 3 * 8192 + swz(s2, c8)) = lo;
           }
+        }
+      } else {
+        // the other warps: binary16 images of K~ = diag(tail) K and of Q
+        const int lt = ((warp >> 2) * 2 + (q4 - 2)) * 32 + lane;   // 0..255
+        for (int idx = lt; idx < 2048; idx += 256) {
+          const int which = idx >> 10, b = (idx >> 9) & 1, x = idx & 511;
+          const uint8_t* src = kq + b * 16384 + which * 8192 + x * 16;
+          float f[8];
+          load8(reinterpret_cast<const __nv_bfloat16*>(src), f);
+          if (which == 0) {
+            const float sc = ss.tail[x >> 3];
 #pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            *reinterpret_cast<uint4*>(stg + SL_MH + swz(t, 2 * cg + q)) = pack_half8(mh + 8 * q);
-            *reinterpret_cast<uint4*>(stg + SL_ML + swz(t, 2 * cg + q)) = pack_half8(ml + 8 * q);
+            for (int u = 0; u < 8; ++u) f[u] *= sc;
+            *reinterpret_cast<uint4*>(stg + SL_BKM + b * 8192 + x * 16) = pack_half8(f);
+          } else {
+            *reinterpret_cast<uint4*>(stg + SL_WQ + b * 16384 + 8192 + x * 16) = pack_half8(f);
           }
         }
       }
@@ -468,21 +551,24 @@ __device__ void prep_role(const PcParams& p, const CUtensorMap* tm_q, const CUte
       // bf16 hi/lo K-major B images [t][s]
       {
         const int t = tid >> 3, c8 = tid & 7;
-        float ph[8], pl[8], qh[8], ql[8];
+        float pa[8], pb[8];
+        const float4 t0v = *reinterpret_cast<const float4*>(Tf + t * kLd + c8 * 8);
+        const float4 t1v = *reinterpret_cast<const float4*>(Tf + t * kLd + c8 * 8 + 4);
+        const float tv[8] = {t0v.x, t0v.y, t0v.z, t0v.w, t1v.x, t1v.y, t1v.z, t1v.w};
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const int s2 = c8 * 8 + j;
-          const float val = (s2 < t) ? Tf[t * kLd + s2] : (s2 == t ? 1.f : 0.f);
-          const float a = val * ss.bg[s2], b = val * ss.beta[s2];
-          ph[j] = a;
-          pl[j] = bf_lo(a);
-          qh[j] = b;
-          ql[j] = bf_lo(b);
+          const float val = (s2 < t) ? tv[j] : (s2 == t ? 1.f : 0.f);
+          pa[j] = val * ss.bg[s2];
+          pb[j] = val * ss.beta[s2];
         }
-        *reinterpret_cast<uint4*>(sm + P_T + 0 * 8192 + swz(t, c8)) = pack_bf8(ph);
-        *reinterpret_cast<uint4*>(sm + P_T + 1 * 8192 + swz(t, c8)) = pack_bf8(pl);
-        *reinterpret_cast<uint4*>(sm + P_T + 2 * 8192 + swz(t, c8)) = pack_bf8(qh);
-        *reinterpret_cast<uint4*>(sm + P_T + 3 * 8192 + swz(t, c8)) = pack_bf8(ql);
+        uint4 hi, lo;
+        split_bf8(pa, hi, lo);
+        *reinterpret_cast<uint4*>(sm + P_T + 0 * 8192 + swz(t, c8)) = hi;
+        *reinterpret_cast<uint4*>(sm + P_T + 1 * 8192 + swz(t, c8)) = lo;
+        split_bf8(pb, hi, lo);
+        *reinterpret_cast<uint4*>(sm + P_T + 2 * 8192 + swz(t, c8)) = hi;
+        *reinterpret_cast<uint4*>(sm + P_T + 3 * 8192 + swz(t, c8)) = lo;
       }
       fence_proxy_async_smem();
       __syncthreads();
@@ -493,10 +579,9 @@ __device__ void prep_role(const PcParams& p, const CUtensorMap* tm_q, const CUte
         for (int ks = 0; ks < 4; ++ks) {
           const uint64_t ak = sw128_desc(a_kq + ks * 2048, 16384, 1024);
           const uint64_t av = sw128_desc(a_v + ks * 2048, 8192, 1024);
+          // B = [T'hi ; T'lo] (N = 128): columns 0-63 get K^T T'hi^T, 64-127 K^T T'lo^T
           mma_f16(tmem + PT_W, ak, sw128_desc(a_t + 0 * 8192 + ks * 32, 16, 1024), id_mn, ks > 0);
-          mma_f16(tmem + PT_W, ak, sw128_desc(a_t + 1 * 8192 + ks * 32, 16, 1024), id_mn, 1);
           mma_f16(tmem + PT_U, av, sw128_desc(a_t + 2 * 8192 + ks * 32, 16, 1024), id_mn, ks > 0);
-          mma_f16(tmem + PT_U, av, sw128_desc(a_t + 3 * 8192 + ks * 32, 16, 1024), id_mn, 1);
         }
         mma_commit(&ss.bar_mma);
       }
@@ -517,14 +602,28 @@ __device__ void prep_role(const PcParams& p, const CUtensorMap* tm_q, const CUte
       }
       {
         uint8_t* slot = slot_of(p.ws, s, r);
-        float v[16];
+        float v[16], vl[16];
         tmem_ld16(tmem + lane_base + PT_W + 16 * cg, v);
+        tmem_ld16(tmem + lane_base + PT_W + 64 + 16 * cg, vl);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) v[j] = -v[j];
+        for (int j = 0; j < 16; ++j) v[j] += vl[j];
+        {
+          // -W, K-major: row = token t, 64 d_k per block (this thread's column j = row)
+          uint8_t* blk = stg + SL_WQ + (row >> 6) * 16384;
 #pragma unroll
-        for (int q = 0; q < 2; ++q)
-          *reinterpret_cast<uint4*>(stg + SL_WN + swz(row, 2 * cg + q)) = pack_half8(v + 8 * q);
+          for (int j = 0; j < 16; j += 2) {
+            const int t = 16 * cg + j;
+            const __half2 h2 = __floats2half2_rn(-v[j], -v[j + 1]);
+            const uint32_t hb = *reinterpret_cast<const uint32_t*>(&h2);
+            const uint32_t col = (row & 7) * 2;
+            *reinterpret_cast<uint16_t*>(blk + swz(t, (row & 63) >> 3) + col) = (uint16_t)(hb & 0xffffu);
+            *reinterpret_cast<uint16_t*>(blk + swz(t + 1, (row & 63) >> 3) + col) = (uint16_t)(hb >> 16);
+          }
+        }
         tmem_ld16(tmem + lane_base + PT_U + 16 * cg, v);
+        tmem_ld16(tmem + lane_base + PT_U + 64 + 16 * cg, vl);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[j] += vl[j];
         float* ut = reinterpret_cast<float*>(stg + SL_UT);
 #pragma unroll
         for (int j = 0; j < 16; ++j) ut[(16 * cg + j) * kHeadDim + row] = v[j];
@@ -594,12 +693,12 @@ __device__ void state_role(const PcParams& p, uint8_t* sm, int s) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ss.tmem;
-  const int total = steps_of(p, s);
+  const int total = steps_of(p, p.cu, s);
   const uint32_t a_s0 = smem_u32(sm + S_S0), a_dth = smem_u32(sm + S_DTH);
-  const uint32_t a_dtl = smem_u32(sm + S_DTL), a_dkf = smem_u32(sm + S_DKF);
-  const uint32_t id_kk = idesc_f16(128, 64, false, false);
-  const uint32_t id_mnb = idesc_f16(128, 64, false, true);
-  const uint32_t id_p = idesc_f16(128, 128, false, true);
+  const uint32_t a_dtl = smem_u32(sm + S_DTL);
+  const uint32_t id_d1 = idesc_f16(128, 128, false, false);
+  const uint32_t id_d2 = idesc_f16(128, 256, false, true);
+  const uint32_t id_d3 = idesc_f16(128, 64, false, true);
 
   int issued = 0;                 // slot copies issued (thread 0's view)
   uint32_t par_dt = 0, par_p = 0, par_o = 0;
@@ -665,68 +764,52 @@ __device__ void state_role(const PcParams& p, uint8_t* sm, int s) {
       }
       if (!mbar_wait_bounded(&ss.bar_slot[b], (uint32_t)((r >> 1) & 1), kLimitNs)) ok = false;
       if (__syncthreads_or(!ok)) { ok = false; break; }
-      // ---- Delta^T = S0 (-W^T) (critical path) ----
+      // ---- D1 = S0 [-W ; Q]^T: Delta^T - U^T and S0 Q^T (critical path) ----
       if (tid == 0) {
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t a = sw128_desc(a_s0 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-          mma_f16(tmem + ST_DT, a, sw128_desc(a_buf + SL_WN + kk * 2048, 16384, 1024), id_mnb,
-                  kk > 0);
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_f16(tmem + ST_D1, sw128_desc(a_s0 + off, 16, 1024),
+                  sw128_desc(a_buf + SL_WQ + off, 16, 1024), id_d1, kk > 0);
         }
         mma_commit(&ss.bar_dt);
-        // OA = S0 Q^T runs while the Delta readout proceeds; P's commit covers it
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t a = sw128_desc(a_s0 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-          mma_f16(tmem + ST_OA, a,
-                  sw128_desc(a_buf + SL_QF + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id_kk,
-                  kk > 0);
-        }
       }
       if (!mbar_wait_bounded(&ss.bar_dt, par_dt, kLimitNs)) ok = false;
       par_dt ^= 1;
       tc_fence_after();
-      // ---- Delta = U + (-W S0^T): operands Delta^T (hi, lo) and Delta~^T ----
+      // ---- Delta = U - W S0^T as binary16 high and low parts ----
       const float* vec = reinterpret_cast<const float*>(buf + SL_VEC);
       float d[16];
       {
-        float v[16], dh[16], dl[16], dk[16];
-        tmem_ld16(tmem + lane_base + ST_DT + 16 * cg, v);
+        float v[16];
+        tmem_ld16(tmem + lane_base + ST_D1 + 16 * cg, v);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          d[j] = v[j] + ut[j];
-          dh[j] = d[j];
-          dl[j] = half_lo(d[j]);
-          dk[j] = d[j] * vec[64 + 16 * cg + j];
-        }
+        for (int j = 0; j < 16; ++j) d[j] = v[j] + ut[j];
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
-          *reinterpret_cast<uint4*>(sm + S_DTH + swz(row, 2 * cg + q)) = pack_half8(dh + 8 * q);
-          *reinterpret_cast<uint4*>(sm + S_DTL + swz(row, 2 * cg + q)) = pack_half8(dl + 8 * q);
-          *reinterpret_cast<uint4*>(sm + S_DKF + swz(row, 2 * cg + q)) = pack_half8(dk + 8 * q);
+          uint4 hi, lo;
+          split_half8(d + 8 * q, hi, lo);
+          *reinterpret_cast<uint4*>(sm + S_DTH + swz(row, 2 * cg + q)) = hi;
+          *reinterpret_cast<uint4*>(sm + S_DTL + swz(row, 2 * cg + q)) = lo;
         }
       }
       fence_proxy_async_smem();
       tc_fence_before();
       if (__syncthreads_or(!ok)) { ok = false; break; }
-      // ---- P = Delta~^T K (critical), then OB = Delta^T M^T (hi/lo) ----
+      // ---- D2 = Delta_hi^T [K~ | M^T hi | M^T lo] (critical), D3 = Delta_lo^T M^T hi ----
       if (tid == 32) st_release(flags + kRing, r + 1);   // slot r fully read
       if (tid == 0) {
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
-          mma_f16(tmem + ST_P, sw128_desc(a_dkf + ks * 32, 16, 1024),
-                  sw128_desc(a_buf + SL_KF + ks * 2048, 8192, 1024), id_p, ks > 0);
+          mma_f16(tmem + ST_D2, sw128_desc(a_dth + ks * 32, 16, 1024),
+                  sw128_desc(a_buf + SL_BKM + ks * 2048, 8192, 1024), id_d2, ks > 0);
         mma_commit(&ss.bar_p);
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-          const uint64_t mh = sw128_desc(a_buf + SL_MH + ks * 32, 16, 1024);
-          const uint64_t ml = sw128_desc(a_buf + SL_ML + ks * 32, 16, 1024);
-          mma_f16(tmem + ST_OB, sw128_desc(a_dth + ks * 32, 16, 1024), mh, id_kk, ks > 0);
-          mma_f16(tmem + ST_OB, sw128_desc(a_dtl + ks * 32, 16, 1024), mh, id_kk, 1);
-          mma_f16(tmem + ST_OB, sw128_desc(a_dth + ks * 32, 16, 1024), ml, id_kk, 1);
-        }
+        for (int ks = 0; ks < 4; ++ks)
+          mma_f16(tmem + ST_D3, sw128_desc(a_dtl + ks * 32, 16, 1024),
+                  sw128_desc(a_buf + SL_BKM + 2 * 8192 + ks * 2048, 8192, 1024), id_d3, ks > 0);
         mma_commit(&ss.bar_o);
       }
       // prefetch the next step's slot into the other buffer if it was ready
@@ -741,7 +824,7 @@ __device__ void state_role(const PcParams& p, uint8_t* sm, int s) {
       {
         const float gL = vec[192];
         float pv[32];
-        tmem_ld32(tmem + lane_base + ST_P + 32 * cg, pv);
+        tmem_ld32(tmem + lane_base + ST_D2 + 32 * cg, pv);
 #pragma unroll
         for (int j = 0; j < 32; ++j) S[j] = fmaf(gL, S[j], pv[j]);
 #pragma unroll
@@ -753,16 +836,24 @@ __device__ void state_role(const PcParams& p, uint8_t* sm, int s) {
       par_o ^= 1;
       tc_fence_after();
       {
-        float oa[16], ob[16];
-        tmem_ld16(tmem + lane_base + ST_OA + 16 * cg, oa);
-        tmem_ld16(tmem + lane_base + ST_OB + 16 * cg, ob);
+        // o_t = scale (e^{G_t} (S0 Q^T)_t + (M Delta)_t + M_tt Delta_t)
+        float acc[16], part[16];
+        tmem_ld16(tmem + lane_base + ST_OA + 16 * cg, part);
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          acc[j] = fmaf(vec[16 * cg + j], part[j], vec[128 + 16 * cg + j] * d[j]);
+        tmem_ld16(tmem + lane_base + ST_OBHH + 16 * cg, part);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) acc[j] += part[j];
+        tmem_ld16(tmem + lane_base + ST_OBHL + 16 * cg, part);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) acc[j] += part[j];
+        tmem_ld16(tmem + lane_base + ST_D3 + 16 * cg, part);
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const int t = 16 * cg + j;
-          if (t < L) {
-            const float val = p.scale * (vec[t] * oa[j] + ob[j] + vec[128 + t] * d[j]);
-            o[((t0 + t) * p.H_v + h) * kHeadDim + row] = from_f32<To>(val);
-          }
+          if (t < L)
+            o[((t0 + t) * p.H_v + h) * kHeadDim + row] = from_f32<To>(p.scale * (acc[j] + part[j]));
         }
       }
       fence_proxy_async_smem();
