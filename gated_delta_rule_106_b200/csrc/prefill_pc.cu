@@ -51,16 +51,16 @@ namespace {
 using namespace sm100;
 
 constexpr int kPcThreads = 512;
-constexpr int kRing = 3;
+constexpr int kRing = 6;            // slots per state CTA: how far prep may run ahead
 constexpr uint64_t kLimitNs = 2000000000ull;
 
 // ---- ring slot (global), 1024-aligned sections ---------------------------
 // B operand of S0 [-W ; Q]^T: K-major, [2 d_k blocks][128 rows][64], rows 0-63 = -W
 // (token t), rows 64-127 = Q (token t), binary16.
 constexpr uint32_t SL_WQ = 0;
-// B operand of Delta^T [K~ | M^T hi | M^T lo]: MN-major, four 64-column blocks of
-// [64 tokens s][64] at 8 KB stride: K~ = diag(e^{G_L-G}) K (d_k 0-63, 64-127), then the
-// strictly lower M transposed (M^T[s][t] = M_ts for t > s) as binary16 high and low parts.
+// B operands of Delta^T K~ and Delta^T M^T, four 8 KB blocks: K~ = diag(e^{G_L-G}) K,
+// MN-major [64 tokens s][64 d_k] (d_k 0-63, 64-127), then the strictly lower M
+// (M[t][s] = M_ts for s < t) as binary16 high and low parts, K-major [64 t][64 s].
 constexpr uint32_t SL_BKM = 32768;
 constexpr uint32_t SL_VEC = 65536;     // gamma[64] tail[64] mdiag[64] gL
 constexpr uint32_t SL_IMG = 66560;     // bytes of the shared-memory image above
@@ -71,28 +71,34 @@ constexpr uint32_t CTRL_BYTES = 16384; // counter, abort word, per-state-CTA fla
 constexpr int kFlagStride = 16;        // ints per state CTA: full[kRing], consumed
 
 // ---- prep CTA shared memory ---------------------------------------------
-constexpr uint32_t P_KQ = 0;           // [blk0: K 8K | Q 8K][blk1: K | Q] bf16, TMA 128B swizzle
-constexpr uint32_t P_V = 32768;        // [blk0 8K][blk1 8K] bf16
+// A prep CTA runs two independent pipelines of kPipeThreads threads (named
+// barriers 1 and 2), each working on its own item, so that one pipeline's
+// latency-bound phases overlap the other's. Per pipeline:
+constexpr int kPipeThreads = kPcThreads / 2;
+constexpr uint32_t PIPE_BYTES = 100352;
+constexpr uint32_t PP_TILES = 0;       // [K0 8K | Q0 8K | K1 8K | Q1 8K | V0 8K | V1 8K] bf16,
+                                       // TMA 128B swizzle; the solve scratch reuses Q0
 constexpr int kLd = 68;                // row stride (floats) of the fp32 A and T tiles
-constexpr uint32_t P_AF = 49152;       // fp32 A [64][kLd]
-constexpr uint32_t P_TF = 66560;       // fp32 T [64][kLd]
-constexpr uint32_t P_T = 86016;        // bf16 T'hi, T'lo, T''hi, T''lo [64][64] each
-constexpr uint32_t P_STG = 118784;     // whole-slot staging (SLOT_BYTES), one bulk store
-constexpr uint32_t P_SMALL = 218112;
+constexpr uint32_t PP_AF = 49152;      // fp32 A [64][kLd]; after the solve: bf16 T' hi | lo
+constexpr uint32_t PP_TF = 66560;      // fp32 T [64][kLd]
+constexpr uint32_t PP_T2 = 83968;      // bf16 T'' hi | lo [64][64] each
+constexpr uint32_t P_SMALL = 2 * PIPE_BYTES;
 // ---- state CTA shared memory --------------------------------------------
 constexpr uint32_t S_BUF = 0;          // 2 x slot image
 constexpr uint32_t S_S0 = 133120;      // binary16 state, K-major [2 blocks][128 rows]
 constexpr uint32_t S_DTH = 165888;     // Delta^T high, K-major A [128][64 t]
 constexpr uint32_t S_DTL = 182272;     // Delta^T low
 constexpr uint32_t S_SMALL = 215040;
-constexpr uint32_t PC_SMEM_BYTES = P_SMALL + 4096;
+constexpr uint32_t PC_SMEM_BYTES = S_SMALL + 1024;   // the state role needs the most
 constexpr uint32_t PC_SMEM_ALLOC = PC_SMEM_BYTES + 1024;
 
 // TMEM columns
-// prep: Gram [128 x 128]; W^T and U^T each as [hi part | lo part] column halves
-constexpr uint32_t PT_GR = 0, PT_W = 128, PT_U = 256, PT_COLS = 512;
+// prep, per pipeline (256 columns each): Gram [128 x 64] at 0, then W^T as
+// [hi part | lo part] column halves at 0 and U^T the same way at 128
+constexpr uint32_t PT_GR = 0, PT_W = 0, PT_U = 128, PT_PIPE = 256, PT_COLS = 512;
 // state: D1 = S0 [-W ; Q]^T -> [Delta^T - U^T | S0 Q^T];
-//        D2 = Delta_hi^T [K~ | M^T hi | M^T lo] -> [P | OB_hh | OB_hl]; D3 = Delta_lo^T M^T hi
+//        D2 = Delta_hi^T K~ -> P;  Delta_hi^T [M hi ; M lo]^T -> [OB_hh | OB_hl];
+//        D3 = Delta_lo^T M_hi^T
 constexpr uint32_t ST_D1 = 0, ST_OA = 64, ST_D2 = 128, ST_OBHH = 256, ST_OBHL = 320,
                    ST_D3 = 384, ST_COLS = 512;
 
@@ -106,15 +112,19 @@ struct PcParams {
 };
 
 constexpr int kCuCache = 513;   // sequences whose boundaries the prep CTAs keep on chip
-struct PrepSmall {
-  int cu[kCuCache];
+struct PipeSmall {
   float G[64], beta[64], gamma[64], bg[64], tail[64], mdiag[64];
   float gL;
   int claim;
-  int max_steps;
   int ok;
-  uint32_t tmem;
+  int abort;
   uint64_t bar_tma, bar_mma;
+};
+struct PrepSmall {
+  int cu[kCuCache];
+  int max_steps;
+  uint32_t tmem;
+  PipeSmall pipe[2];
 };
 struct StateSmall {
   uint32_t tmem;
@@ -215,7 +225,8 @@ __device__ bool locate(const PcParams& p, const int32_t* cu, int s, int r, int* 
 // X are read four floats at a time; at b = 32 each thread makes two adjacent
 // outputs.
 template <int b>
-__device__ __forceinline__ void merge_level(const float* Af, float* Tf, float* Xs, int tid) {
+__device__ __forceinline__ void merge_level(const float* Af, float* Tf, float* Xs, int tid,
+                                             uint32_t bar) {
   // Each active thread makes an RI x 2 block of outputs (rows i..i+RI-1,
   // columns j, j+1): row segments of A / T are read four floats at a time and
   // column pairs of T / X two at a time, so loads per FMA stay low.
@@ -223,7 +234,7 @@ __device__ __forceinline__ void merge_level(const float* Af, float* Tf, float* X
   constexpr int RI = b >= 32 ? 4 : 2, RJ = 2;
   constexpr int tiles_i = b / RI, tiles_j = b / RJ;
   constexpr int threads = pairs * tiles_i * tiles_j;   // b=8: 64, 16: 128, 32: 128
-  static_assert(threads <= kPcThreads, "too many threads");
+  static_assert(threads <= kPipeThreads, "too many threads");
   const int pr = tid / (tiles_i * tiles_j);
   const int ti = (tid / tiles_j) % tiles_i, tj = tid % tiles_j;
   const int i0 = ti * RI, j0 = tj * RJ, o = 2 * b * pr;
@@ -233,7 +244,7 @@ __device__ __forceinline__ void merge_level(const float* Af, float* Tf, float* X
     for (int a = 0; a < RI; ++a)
 #pragma unroll
       for (int c = 0; c < RJ; ++c) acc[a][c] = 0.f;
-#pragma unroll
+#pragma unroll 2
     for (int m4 = 0; m4 < b / 4; ++m4) {
       float av[RI][4];
 #pragma unroll
@@ -255,14 +266,14 @@ __device__ __forceinline__ void merge_level(const float* Af, float* Tf, float* X
     for (int a = 0; a < RI; ++a)
       *reinterpret_cast<float2*>(Xs + pr * bb + (i0 + a) * b + j0) = make_float2(acc[a][0], acc[a][1]);
   }
-  __syncthreads();
+  bar_sync_n(bar, kPipeThreads);
   if (tid < threads) {
     float acc[RI][RJ];
 #pragma unroll
     for (int a = 0; a < RI; ++a)
 #pragma unroll
       for (int c = 0; c < RJ; ++c) acc[a][c] = 0.f;
-#pragma unroll
+#pragma unroll 2
     for (int m4 = 0; m4 < b / 4; ++m4) {
       float tv[RI][4];
 #pragma unroll
@@ -285,67 +296,76 @@ __device__ __forceinline__ void merge_level(const float* Af, float* Tf, float* X
       *reinterpret_cast<float2*>(Tf + (o + b + i0 + a) * kLd + o + j0) =
           make_float2(-acc[a][0], -acc[a][1]);
   }
-  __syncthreads();
+  bar_sync_n(bar, kPipeThreads);
 }
 
 // ===================================================================== prep ==
 template <class Tg>
 __device__ void prep_role(const PcParams& p, const CUtensorMap* tm_q, const CUtensorMap* tm_k,
                           const CUtensorMap* tm_v, uint8_t* sm) {
-  PrepSmall& ss = *reinterpret_cast<PrepSmall*>(sm + P_SMALL);
-  float* Af = reinterpret_cast<float*>(sm + P_AF);
-  float* Tf = reinterpret_cast<float*>(sm + P_TF);
-  float* Xs = reinterpret_cast<float*>(sm + P_T);   // solve scratch (T' tiles are written after)
-  uint8_t* kq = sm + P_KQ;
-  uint8_t* vv = sm + P_V;
-  uint8_t* stg = sm + P_STG;
-  int* ctrl = reinterpret_cast<int*>(p.ws);   // [0] counter, [1] abort
+  PrepSmall& sh = *reinterpret_cast<PrepSmall*>(sm + P_SMALL);
+  int* ctrl = reinterpret_cast<int*>(p.ws);         // [0] claim counter, [1] abort word
 
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int q4 = warp & 3, cg = warp >> 2;          // TMEM lane quadrant, 16-column group
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int pl = tid / kPipeThreads;                // pipeline
+  const int ptid = tid % kPipeThreads, warp = ptid >> 5;
+  const int q4 = warp & 3, cg = warp >> 2;          // TMEM lane quadrant, column half
   const int row = (q4 << 5) | lane;
   const uint32_t lane_base = (uint32_t)(q4 << 5) << 16;
+  const uint32_t bar = 1 + pl;
+  // lane 0 of the pipeline's last warp claims the next item during the solve
+  // (where that warp is idle) and starts its tile loads once the current
+  // item's tiles are no longer read
+  constexpr int kIssuer = kPipeThreads - 32;
+  PipeSmall& ss = sh.pipe[pl];
+  uint8_t* pb = sm + pl * PIPE_BYTES;
+  float* Af = reinterpret_cast<float*>(pb + PP_AF);
+  float* Tf = reinterpret_cast<float*>(pb + PP_TF);
+  float* Xs = reinterpret_cast<float*>(pb + PP_TILES + 8192);   // over Q0 once it is dead
+  uint8_t* kq = pb + PP_TILES;                      // [K0 | Q0 | K1 | Q1]
+  uint8_t* vv = kq + 32768;                         // [V0 | V1]
 
-  if (warp == 0) {
-    tmem_alloc(&ss.tmem, PT_COLS);
+  if (tid < 32) {
+    tmem_alloc(&sh.tmem, PT_COLS);
     tmem_relinquish();
   }
   if (tid == 32) {
-    mbar_init(&ss.bar_tma, 1);
-    mbar_init(&ss.bar_mma, 1);
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sh.pipe[i].bar_tma, 1);
+      mbar_init(&sh.pipe[i].bar_mma, 1);
+    }
     fence_mbar_init();
   }
-  if (tid == 0) ss.max_steps = 0;
+  if (tid == 64) {
+    prefetch_tmap(tm_q);
+    prefetch_tmap(tm_k);
+    prefetch_tmap(tm_v);
+  }
+  if (tid == 0) sh.max_steps = 0;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = ss.tmem;
+  const uint32_t tmem = sh.tmem + pl * PT_PIPE;
   const bool cu_on_chip = p.N + 1 <= kCuCache;
   if (cu_on_chip)
-    for (int i = tid; i <= p.N; i += kPcThreads) ss.cu[i] = __ldg(p.cu + i);
+    for (int i = tid; i <= p.N; i += kPcThreads) sh.cu[i] = __ldg(p.cu + i);
   __syncthreads();
-  const int32_t* cu = cu_on_chip ? ss.cu : p.cu;
-  for (int s = tid; s < p.NS; s += kPcThreads) atomicMax(&ss.max_steps, steps_of(p, cu, s));
+  const int32_t* cu = cu_on_chip ? sh.cu : p.cu;
+  for (int s = tid; s < p.NS; s += kPcThreads) atomicMax(&sh.max_steps, steps_of(p, cu, s));
   __syncthreads();
-  const int64_t E = (int64_t)p.NS * ss.max_steps;
-  // Claim the next (state CTA, step) that exists: thread 0 claims, all read.
-  int early = -1;   // thread 0: a claim taken ahead of its use (hides the atomic's latency)
-  auto claim_valid = [&]() -> int {
-    if (tid == 0) {
-      int x = early >= 0 ? early : atomicAdd(&ctrl[0], 1);
-      early = -1;
-      int it_, c_;
-      while (x < E && !locate(p, cu, x % p.NS, x / p.NS, &it_, &c_)) x = atomicAdd(&ctrl[0], 1);
-      ss.claim = x;
-    }
-    __syncthreads();
-    const int x = ss.claim;
-    __syncthreads();
+  const int64_t E = (int64_t)p.NS * sh.max_steps;
+
+  // next existing (state CTA, step) item, in global claim order (one thread)
+  auto claim = [&]() -> int {
+    int x, it_, c_;
+    do {
+      x = atomicAdd(&ctrl[0], 1);
+    } while (x < E && !locate(p, cu, x % p.NS, x / p.NS, &it_, &c_));
     return x;
   };
-  // TMA of claim x's K, Q (key head) and V (value head) tiles.
+  // TMA of item x's K, Q (key head) and V (value head) tiles
   auto issue_tiles = [&](int x) {
-    if (tid != 0) return;
     int it_, c_;
     locate(p, cu, x % p.NS, x / p.NS, &it_, &c_);
     const int n_ = it_ / p.H_v, h_ = it_ % p.H_v, kh_ = h_ / (p.H_v / p.H_k);
@@ -361,307 +381,308 @@ __device__ void prep_role(const PcParams& p, const CUtensorMap* tm_q, const CUte
       tma_load_2d(vv + b * 8192, tm_v, h_ * kHeadDim + b * 64, y, &ss.bar_tma);
     }
   };
-  // Completion of the last bulk store, then the release of its slot's flag.
-  int* pend_flag = nullptr;   // thread 0 only
-  int pend_val = 0;
-  auto publish = [&](int*& flag, int val) {
-    if (!flag) return;
-    bulk_wait_all();
-    fence_proxy_async_all();
-    st_release(flag, val);
-    flag = nullptr;
-  };
-  uint32_t tma_par = 0, mma_par = 0;
-  int e = claim_valid();
-  bool tiles_pending = false;
-  if (e < E) {
-    issue_tiles(e);
-    tiles_pending = true;
+  bool pend = false;   // kIssuer: tile loads in flight that no item has waited on
+  int next = 0;        // kIssuer: the claimed next item
+  if (ptid == kIssuer) {
+    const int x = claim();
+    ss.claim = x;
+    if (x < E) {
+      issue_tiles(x);
+      pend = true;
+    }
   }
-  const uint32_t a_kq = smem_u32(kq), a_v = smem_u32(vv), a_t = smem_u32(sm + P_T);
-  const uint32_t id_gram = idesc_bf16(128, 128, false, false);
+  bar_sync_n(bar, kPipeThreads);
+  int e = ss.claim;
+  uint32_t tma_par = 0, mma_par = 0;
+  const uint32_t a_kq = smem_u32(kq), a_v = smem_u32(vv);
+  const uint32_t a_t1 = smem_u32(pb + PP_AF), a_t2 = smem_u32(pb + PP_T2);
+  const uint32_t id_gram = idesc_bf16(128, 64, false, false);
   const uint32_t id_mn = idesc_bf16(128, 128, true, false);
 
   while (e < E) {
     const int s = e % p.NS, r = e / p.NS;
-    int item, c;
-    int e_next = (int)E;
+    int item = 0, c = 0;
+    locate(p, cu, s, r, &item, &c);
+    const int n = item / p.H_v, h = item % p.H_v;
+    int64_t s0, s1;
+    seq_chunks(cu, p.T, n, &s0, &s1);
+    const int64_t t0 = s0 + (int64_t)c * kChunk;
+    const int L = (int)((s1 - t0) < kChunk ? (s1 - t0) : kChunk);
+    uint8_t* slot = slot_of(p.ws, s, r);
     bool ok = true;
-    if (tid == 0) early = atomicAdd(&ctrl[0], 1);
-    if (locate(p, cu, s, r, &item, &c)) {
-      const int n = item / p.H_v, h = item % p.H_v, kh = h / (p.H_v / p.H_k);
-      int64_t s0, s1;
-      seq_chunks(cu, p.T, n, &s0, &s1);
-      const int64_t t0 = s0 + (int64_t)c * kChunk;
-      const int L = (int)((s1 - t0) < kChunk ? (s1 - t0) : kChunk);
 
-      (void)kh;
-      if (warp == 1) {   // gates: cumulative log-decay and derived vectors
-        const Tg* g = static_cast<const Tg*>(p.g);
-        const Tg* bt = static_cast<const Tg*>(p.beta);
-        float lg[2], be[2];
+    // the slot is written directly: wait until step r - kRing has been consumed
+    if (ptid == 0)
+      ss.ok = wait_flag_ge(flags_of(p.ws, s) + kRing, r + 1 - kRing, &ctrl[1], kLimitNs);
+    if (warp == 1) {   // gates: cumulative log-decay and derived vectors
+      const Tg* g = static_cast<const Tg*>(p.g);
+      const Tg* bt = static_cast<const Tg*>(p.beta);
+      float lg[2], be[2];
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const int t = 2 * lane + j;
-          lg[j] = 0.f;
-          be[j] = 0.f;
-          if (t < L) {
-            const int64_t idx = (t0 + t) * p.H_v + h;
-            lg[j] = logf(fmaxf(to_f32(g[idx]), 1.17549435e-38f));
-            be[j] = to_f32(bt[idx]);
-          }
+      for (int j = 0; j < 2; ++j) {
+        const int t = 2 * lane + j;
+        lg[j] = 0.f;
+        be[j] = 0.f;
+        if (t < L) {
+          const int64_t idx = (t0 + t) * p.H_v + h;
+          lg[j] = logf(fmaxf(to_f32(g[idx]), 1.17549435e-38f));
+          be[j] = to_f32(bt[idx]);
         }
-        float incl = lg[0] + lg[1];
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-          const float y = __shfl_up_sync(0xffffffffu, incl, off);
-          if (lane >= off) incl += y;
-        }
-        const float excl = incl - (lg[0] + lg[1]);
-        const float Gl = __shfl_sync(0xffffffffu, incl, 31);
-        const float Gt[2] = {excl + lg[0], excl + lg[0] + lg[1]};
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const int t = 2 * lane + j;
-          const float gam = __expf(Gt[j]);
-          ss.G[t] = Gt[j];
-          ss.beta[t] = be[j];
-          ss.gamma[t] = gam;
-          ss.bg[t] = be[j] * gam;
-          ss.tail[t] = __expf(Gl - Gt[j]);
-        }
-        if (lane == 0) ss.gL = __expf(Gl);
       }
-      ok = mbar_wait_bounded(&ss.bar_tma, tma_par, kLimitNs);
+      float incl = lg[0] + lg[1];
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
+      }
+      const float excl = incl - (lg[0] + lg[1]);
+      const float Gl = __shfl_sync(0xffffffffu, incl, 31);
+      const float Gt[2] = {excl + lg[0], excl + lg[0] + lg[1]};
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int t = 2 * lane + j;
+        const float gam = __expf(Gt[j]);
+        ss.G[t] = Gt[j];
+        ss.beta[t] = be[j];
+        ss.gamma[t] = gam;
+        ss.bg[t] = be[j] * gam;
+        ss.tail[t] = __expf(Gl - Gt[j]);
+      }
+      if (lane == 0) ss.gL = __expf(Gl);
+    }
+    ok = mbar_wait_bounded(&ss.bar_tma, tma_par, kLimitNs);
+    if (ok) {   // a phase seen complete by this thread
       tma_par ^= 1;
-      if (ok) tiles_pending = false;
-      if (tid == 0) publish(pend_flag, pend_val);   // previous item's slot
-      if (__syncthreads_or(!ok)) goto fail;
+      if (ptid == kIssuer) pend = false;
+    }
+    bar_sync_n(bar, kPipeThreads);
+    ok = ok && ss.ok;
+    if (bar_or_n(bar, kPipeThreads, !ok)) goto fail;
 
-      if (L < kChunk) {   // rows past the sequence end hold other data: zero them
-        for (int idx = tid; idx < 3072; idx += kPcThreads) {
-          const int rr = (idx & 511) >> 3;
-          if (rr >= L) {
-            uint8_t* ptr = idx < 2048 ? kq + idx * 16 : vv + (idx - 2048) * 16;
-            *reinterpret_cast<uint4*>(ptr) = make_uint4(0, 0, 0, 0);
-          }
+    if (L < kChunk) {   // rows past the sequence end hold other data: zero them
+      for (int idx = ptid; idx < 3072; idx += kPipeThreads) {
+        const int rr = (idx & 511) >> 3;
+        if (rr >= L) {
+          uint8_t* ptr = idx < 2048 ? kq + idx * 16 : vv + (idx - 2048) * 16;
+          *reinterpret_cast<uint4*>(ptr) = make_uint4(0, 0, 0, 0);
         }
-        fence_proxy_async_smem();
-        __syncthreads();
-      }
-      // ---- Gram [K;Q][K;Q]^T (bf16, exact products): rows 0-63 give K K^T and
-      //      K Q^T (the transposed query-key products) ----
-      if (tid == 0) {
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_f16(tmem + PT_GR, sw128_desc(a_kq + off, 16, 1024),
-                  sw128_desc(a_kq + off, 16, 1024), id_gram, kk > 0);
-        }
-        mma_commit(&ss.bar_mma);
-      }
-      ok = mbar_wait_bounded(&ss.bar_mma, mma_par, kLimitNs);
-      mma_par ^= 1;
-      tc_fence_after();
-      if (q4 < 2) {
-        // lanes 0-63 (key token s): A[s][x] = beta_s e^{G_s-G_x} k_s.k_x (x < s) from
-        // columns 0-63, and M^T[s][t] = e^{G_t-G_s} q_t.k_s (t > s) from columns 64-127
-        const int s2 = row, c0 = 32 * cg;
-        float v[32];
-        tmem_ld32(tmem + lane_base + PT_GR + c0, v);
-        const float Gs = ss.G[s2];
-        if (c0 < 64) {
-          const float bs = ss.beta[s2];
-#pragma unroll
-          for (int j = 0; j < 32; j += 4) {
-            float a4[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const int x = c0 + j + u;
-              a4[u] = (x < s2) ? bs * __expf(Gs - ss.G[x]) * v[j + u] : 0.f;
-            }
-            *reinterpret_cast<float4*>(Af + s2 * kLd + c0 + j) = make_float4(a4[0], a4[1], a4[2], a4[3]);
-          }
-        } else {
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            float mh[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              const int t = c0 - 64 + 8 * q + u;
-              const float val = (t >= s2) ? __expf(ss.G[t] - Gs) * v[8 * q + u] : 0.f;
-              if (t == s2) ss.mdiag[s2] = val;
-              mh[u] = (t > s2) ? val : 0.f;
-            }
-            const int c8 = (c0 - 64) / 8 + q;
-            uint4 hi, lo;
-            split_half8(mh, hi, lo);
-            *reinterpret_cast<uint4*>(stg + SL_BKM + 2 * 8192 + swz(s2, c8)) = hi;
-            *reinterpret_cast<uint4*>(stg + SL_BKM + 3 * 8192 + swz(s2, c8)) = lo;
-          }
-        }
-      } else {
-        // the other warps: binary16 images of K~ = diag(tail) K and of Q
-        const int lt = ((warp >> 2) * 2 + (q4 - 2)) * 32 + lane;   // 0..255
-        for (int idx = lt; idx < 2048; idx += 256) {
-          const int which = idx >> 10, b = (idx >> 9) & 1, x = idx & 511;
-          const uint8_t* src = kq + b * 16384 + which * 8192 + x * 16;
-          float f[8];
-          load8(reinterpret_cast<const __nv_bfloat16*>(src), f);
-          if (which == 0) {
-            const float sc = ss.tail[x >> 3];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) f[u] *= sc;
-            *reinterpret_cast<uint4*>(stg + SL_BKM + b * 8192 + x * 16) = pack_half8(f);
-          } else {
-            *reinterpret_cast<uint4*>(stg + SL_WQ + b * 16384 + 8192 + x * 16) = pack_half8(f);
-          }
-        }
-      }
-      tc_fence_before();
-      if (__syncthreads_or(!ok)) goto fail;
-
-      // ---- T = (I + A)^{-1}: 8x8 diagonal blocks by forward substitution,
-      //      then pairwise merges 8 -> 16 -> 32 -> 64:  T21 = -T22 A21 T11 ----
-      for (int idx = tid; idx < 64 * kLd; idx += kPcThreads) Tf[idx] = 0.f;
-      __syncthreads();
-      if (tid < 64) {
-        const int B = tid >> 3, j = tid & 7;
-        float a[8][8], x[8];
-#pragma unroll
-        for (int rr = 1; rr < 8; ++rr)
-#pragma unroll
-          for (int m = 0; m < rr; ++m) a[rr][m] = Af[(8 * B + rr) * kLd + 8 * B + m];
-#pragma unroll
-        for (int rr = 0; rr < 8; ++rr) {
-          float acc = (rr == j) ? 1.f : 0.f;
-#pragma unroll
-          for (int m = 0; m < rr; ++m) acc = fmaf(-a[rr][m], x[m], acc);
-          x[rr] = acc;
-        }
-#pragma unroll
-        for (int rr = 0; rr < 8; ++rr) Tf[(8 * B + rr) * kLd + 8 * B + j] = x[rr];
-      }
-      __syncthreads();
-      merge_level<8>(Af, Tf, Xs, tid);
-      merge_level<16>(Af, Tf, Xs, tid);
-      merge_level<32>(Af, Tf, Xs, tid);
-      // T' = T diag(beta e^G), T'' = T diag(beta) (unit diagonal included) as
-      // bf16 hi/lo K-major B images [t][s]
-      {
-        const int t = tid >> 3, c8 = tid & 7;
-        float pa[8], pb[8];
-        const float4 t0v = *reinterpret_cast<const float4*>(Tf + t * kLd + c8 * 8);
-        const float4 t1v = *reinterpret_cast<const float4*>(Tf + t * kLd + c8 * 8 + 4);
-        const float tv[8] = {t0v.x, t0v.y, t0v.z, t0v.w, t1v.x, t1v.y, t1v.z, t1v.w};
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int s2 = c8 * 8 + j;
-          const float val = (s2 < t) ? tv[j] : (s2 == t ? 1.f : 0.f);
-          pa[j] = val * ss.bg[s2];
-          pb[j] = val * ss.beta[s2];
-        }
-        uint4 hi, lo;
-        split_bf8(pa, hi, lo);
-        *reinterpret_cast<uint4*>(sm + P_T + 0 * 8192 + swz(t, c8)) = hi;
-        *reinterpret_cast<uint4*>(sm + P_T + 1 * 8192 + swz(t, c8)) = lo;
-        split_bf8(pb, hi, lo);
-        *reinterpret_cast<uint4*>(sm + P_T + 2 * 8192 + swz(t, c8)) = hi;
-        *reinterpret_cast<uint4*>(sm + P_T + 3 * 8192 + swz(t, c8)) = lo;
       }
       fence_proxy_async_smem();
-      __syncthreads();
-      // ---- W^T = K^T T'^T, U^T = V^T T''^T (bf16 hi + lo) ----
-      if (tid == 0) {
-        tc_fence_after();
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-          const uint64_t ak = sw128_desc(a_kq + ks * 2048, 16384, 1024);
-          const uint64_t av = sw128_desc(a_v + ks * 2048, 8192, 1024);
-          // B = [T'hi ; T'lo] (N = 128): columns 0-63 get K^T T'hi^T, 64-127 K^T T'lo^T
-          mma_f16(tmem + PT_W, ak, sw128_desc(a_t + 0 * 8192 + ks * 32, 16, 1024), id_mn, ks > 0);
-          mma_f16(tmem + PT_U, av, sw128_desc(a_t + 2 * 8192 + ks * 32, 16, 1024), id_mn, ks > 0);
-        }
-        mma_commit(&ss.bar_mma);
-      }
-      // the slot must be free before anything is written to it
-      if (tid == 0)
-        ss.ok = wait_flag_ge(flags_of(p.ws, s) + kRing, r + 1 - kRing, &ctrl[1], kLimitNs);
-      ok = mbar_wait_bounded(&ss.bar_mma, mma_par, kLimitNs);
-      mma_par ^= 1;
+      bar_sync_n(bar, kPipeThreads);
+    }
+    // ---- Gram [K;Q] K^T (bf16, exact products): rows 0-63 give K K^T, rows
+    //      64-127 the query-key products Q K^T ----
+    if (ptid == 0) {
       tc_fence_after();
-      __syncthreads();
-      ok = ok && ss.ok;
-      if (__syncthreads_or(!ok)) goto fail;
-      // the tiles are no longer read: prefetch the next claim's tiles
-      e_next = claim_valid();
-      if (e_next < E) {
-        issue_tiles(e_next);
-        tiles_pending = true;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+        mma_f16(tmem + PT_GR, sw128_desc(a_kq + off, 16, 1024),
+                sw128_desc(a_kq + off, 16, 1024), id_gram, kk > 0);
       }
-      {
-        uint8_t* slot = slot_of(p.ws, s, r);
-        float v[16], vl[16];
-        tmem_ld16(tmem + lane_base + PT_W + 16 * cg, v);
-        tmem_ld16(tmem + lane_base + PT_W + 64 + 16 * cg, vl);
+      mma_commit(&ss.bar_mma);
+    }
+    // meanwhile: binary16 images of K~ = diag(tail) K and of Q, straight to the slot
+#pragma unroll 2
+    for (int idx = ptid; idx < 2048; idx += kPipeThreads) {
+      const int which = idx >> 10, b = (idx >> 9) & 1, x = idx & 511;
+      const uint8_t* src = kq + b * 16384 + which * 8192 + x * 16;
+      float f[8];
+      load8(reinterpret_cast<const __nv_bfloat16*>(src), f);
+      const float sc = which == 0 ? ss.tail[x >> 3] : 1.f;
 #pragma unroll
-        for (int j = 0; j < 16; ++j) v[j] += vl[j];
-        {
-          // -W, K-major: row = token t, 64 d_k per block (this thread's column j = row)
-          uint8_t* blk = stg + SL_WQ + (row >> 6) * 16384;
+      for (int u = 0; u < 8; ++u) f[u] *= sc;
+      uint8_t* dst = which == 0 ? slot + SL_BKM + b * 8192 + x * 16
+                                : slot + SL_WQ + b * 16384 + 8192 + x * 16;
+      *reinterpret_cast<uint4*>(dst) = pack_half8(f);
+    }
+    ok = mbar_wait_bounded(&ss.bar_mma, mma_par, kLimitNs);
+    mma_par ^= 1;
+    tc_fence_after();
+    if (q4 < 2) {
+      // lanes 0-63 (key token s = row), columns x = 32cg..32cg+31:
+      // A[s][x] = beta_s e^{G_s-G_x} k_s.k_x for x < s (the solve reads no other entry)
+      const int s2 = row, c0 = 32 * cg;
+      if (!(q4 == 0 && cg == 1)) {
+        const float Gs = ss.G[s2], bs = ss.beta[s2];
+        float v[32];
+        tmem_ld32(tmem + lane_base + PT_GR + c0, v);
 #pragma unroll
-          for (int j = 0; j < 16; j += 2) {
-            const int t = 16 * cg + j;
-            const __half2 h2 = __floats2half2_rn(-v[j], -v[j + 1]);
-            const uint32_t hb = *reinterpret_cast<const uint32_t*>(&h2);
-            const uint32_t col = (row & 7) * 2;
-            *reinterpret_cast<uint16_t*>(blk + swz(t, (row & 63) >> 3) + col) = (uint16_t)(hb & 0xffffu);
-            *reinterpret_cast<uint16_t*>(blk + swz(t + 1, (row & 63) >> 3) + col) = (uint16_t)(hb >> 16);
+        for (int q = 0; q < 8; ++q) {
+          float a4[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int x = c0 + 4 * q + u;
+            a4[u] = (x < s2) ? bs * __expf(Gs - ss.G[x]) * v[4 * q + u] : 0.f;
           }
+          *reinterpret_cast<float4*>(Af + s2 * kLd + c0 + 4 * q) = make_float4(a4[0], a4[1], a4[2], a4[3]);
         }
-        tmem_ld16(tmem + lane_base + PT_U + 16 * cg, v);
-        tmem_ld16(tmem + lane_base + PT_U + 64 + 16 * cg, vl);
+      }
+    } else {
+      // lanes 64-127 (query token t = row - 64), columns s = 32cg..32cg+31:
+      // M[t][s] = e^{G_t-G_s} q_t.k_s for s < t as binary16 high and low parts, and
+      // the diagonal M_tt = q_t.k_t
+      const int t = row - 64, c0 = 32 * cg;
+      uint8_t* mh = slot + SL_BKM + 2 * 8192;
+      uint8_t* ml = slot + SL_BKM + 3 * 8192;
+      if (q4 == 2 && cg == 1) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) v[j] += vl[j];
-        float* ut = reinterpret_cast<float*>(stg + SL_UT);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) ut[(16 * cg + j) * kHeadDim + row] = v[j];
-        float* vec = reinterpret_cast<float*>(stg + SL_VEC);
-        if (tid < 64) {
-          vec[tid] = ss.gamma[tid];
-          vec[64 + tid] = ss.tail[tid];
-          vec[128 + tid] = ss.mdiag[tid];
+        for (int q = 0; q < 4; ++q) {
+          *reinterpret_cast<uint4*>(mh + swz(t, 4 * cg + q)) = make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(ml + swz(t, 4 * cg + q)) = make_uint4(0, 0, 0, 0);
         }
-        if (tid == 64) vec[192] = ss.gL;
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        // one bulk store of the whole slot; its completion and the release of
-        // the slot's flag happen at the next item, after that item's tiles land
-        if (tid == 0) {
-          bulk_s2g(slot, stg, SLOT_BYTES);
-          bulk_commit();
-          pend_flag = flags_of(p.ws, s) + (r % kRing);
-          pend_val = r + 1;
+      } else {
+        const float Gt = ss.G[t];
+        float v[32];
+        tmem_ld32(tmem + lane_base + PT_GR + c0, v);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          float m8[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int s2 = c0 + 8 * q + u;
+            if (s2 == t) ss.mdiag[t] = v[8 * q + u];
+            m8[u] = (s2 < t) ? __expf(Gt - ss.G[s2]) * v[8 * q + u] : 0.f;
+          }
+          uint4 hi, lo;
+          split_half8(m8, hi, lo);
+          *reinterpret_cast<uint4*>(mh + swz(t, 4 * cg + q)) = hi;
+          *reinterpret_cast<uint4*>(ml + swz(t, 4 * cg + q)) = lo;
         }
       }
     }
-    e = e_next;
-    if (ld_acquire(&ctrl[1]) != 0) break;
+    tc_fence_before();
+    if (bar_or_n(bar, kPipeThreads, !ok)) goto fail;
+
+    if (ptid == kIssuer) {
+      next = claim();
+      ss.claim = next;
+    }
+    // ---- T = (I + A)^{-1}: 8x8 diagonal blocks by forward substitution,
+    //      then pairwise merges 8 -> 16 -> 32 -> 64:  T21 = -T22 A21 T11 ----
+    for (int idx = ptid; idx < 16 * kLd; idx += kPipeThreads)
+      reinterpret_cast<float4*>(Tf)[idx] = make_float4(0.f, 0.f, 0.f, 0.f);
+    bar_sync_n(bar, kPipeThreads);
+    if (ptid < 64) {
+      const int B = ptid >> 3, j = ptid & 7;
+      float a[8][8], x[8];
+#pragma unroll
+      for (int rr = 1; rr < 8; ++rr)
+#pragma unroll
+        for (int m = 0; m < rr; ++m) a[rr][m] = Af[(8 * B + rr) * kLd + 8 * B + m];
+#pragma unroll
+      for (int rr = 0; rr < 8; ++rr) {
+        float acc = (rr == j) ? 1.f : 0.f;
+#pragma unroll
+        for (int m = 0; m < rr; ++m) acc = fmaf(-a[rr][m], x[m], acc);
+        x[rr] = acc;
+      }
+#pragma unroll
+      for (int rr = 0; rr < 8; ++rr) Tf[(8 * B + rr) * kLd + 8 * B + j] = x[rr];
+    }
+    bar_sync_n(bar, kPipeThreads);
+    merge_level<8>(Af, Tf, Xs, ptid, bar);
+    merge_level<16>(Af, Tf, Xs, ptid, bar);
+    merge_level<32>(Af, Tf, Xs, ptid, bar);
+    // T' = T diag(beta e^G) (over A, which is no longer read), T'' = T diag(beta)
+    // (unit diagonal included) as bf16 hi/lo K-major B images [t][s]
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+      const int t = (ptid >> 3) + 32 * h2, c8 = ptid & 7;
+      float pa[8], pb2[8];
+      const float4 t0v = *reinterpret_cast<const float4*>(Tf + t * kLd + c8 * 8);
+      const float4 t1v = *reinterpret_cast<const float4*>(Tf + t * kLd + c8 * 8 + 4);
+      const float tv[8] = {t0v.x, t0v.y, t0v.z, t0v.w, t1v.x, t1v.y, t1v.z, t1v.w};
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int s2 = c8 * 8 + j;
+        const float val = (s2 < t) ? tv[j] : (s2 == t ? 1.f : 0.f);
+        pa[j] = val * ss.bg[s2];
+        pb2[j] = val * ss.beta[s2];
+      }
+      uint4 hi, lo;
+      split_bf8(pa, hi, lo);
+      *reinterpret_cast<uint4*>(pb + PP_AF + swz(t, c8)) = hi;
+      *reinterpret_cast<uint4*>(pb + PP_AF + 8192 + swz(t, c8)) = lo;
+      split_bf8(pb2, hi, lo);
+      *reinterpret_cast<uint4*>(pb + PP_T2 + swz(t, c8)) = hi;
+      *reinterpret_cast<uint4*>(pb + PP_T2 + 8192 + swz(t, c8)) = lo;
+    }
+    fence_proxy_async_smem();
+    bar_sync_n(bar, kPipeThreads);
+    // ---- W^T = K^T T'^T, U^T = V^T T''^T: B = [hi ; lo] stacked (N = 128), the
+    //      two column halves are summed in the readout ----
+    if (ptid == 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks) {
+        const uint64_t ak = sw128_desc(a_kq + ks * 2048, 16384, 1024);
+        const uint64_t av = sw128_desc(a_v + ks * 2048, 8192, 1024);
+        mma_f16(tmem + PT_W, ak, sw128_desc(a_t1 + ks * 32, 16, 1024), id_mn, ks > 0);
+        mma_f16(tmem + PT_U, av, sw128_desc(a_t2 + ks * 32, 16, 1024), id_mn, ks > 0);
+      }
+      mma_commit(&ss.bar_mma);
+    }
+    ok = mbar_wait_bounded(&ss.bar_mma, mma_par, kLimitNs);
+    mma_par ^= 1;
+    tc_fence_after();
+    // the tiles are free: start the next item's loads
+    if (ptid == kIssuer && ok && next < E) {
+      issue_tiles(next);
+      pend = true;
+    }
+    {
+      float* ut = reinterpret_cast<float*>(slot + SL_UT);
+      // -W, K-major: row = token t, 64 d_k per block (this thread's d_k column = row)
+      uint8_t* blk = slot + SL_WQ + (row >> 6) * 16384;
+      const uint32_t col = (row & 7) * 2;
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int tb0 = 32 * cg + 16 * hh;
+        float v[16], vl[16];
+        tmem_ld16(tmem + lane_base + PT_W + tb0, v);
+        tmem_ld16(tmem + lane_base + PT_W + 64 + tb0, vl);
+#pragma unroll
+        for (int j = 0; j < 16; j += 2) {
+          const int t = tb0 + j;
+          const __half2 h2 = __floats2half2_rn(-(v[j] + vl[j]), -(v[j + 1] + vl[j + 1]));
+          const uint32_t hb = *reinterpret_cast<const uint32_t*>(&h2);
+          *reinterpret_cast<uint16_t*>(blk + swz(t, (row & 63) >> 3) + col) = (uint16_t)(hb & 0xffffu);
+          *reinterpret_cast<uint16_t*>(blk + swz(t + 1, (row & 63) >> 3) + col) = (uint16_t)(hb >> 16);
+        }
+        tmem_ld16(tmem + lane_base + PT_U + tb0, v);
+        tmem_ld16(tmem + lane_base + PT_U + 64 + tb0, vl);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) ut[(tb0 + j) * kHeadDim + row] = v[j] + vl[j];
+      }
+      float* vec = reinterpret_cast<float*>(slot + SL_VEC);
+      if (ptid < 64) {
+        vec[ptid] = ss.gamma[ptid];
+        vec[64 + ptid] = ss.tail[ptid];
+        vec[128 + ptid] = ss.mdiag[ptid];
+      }
+      if (ptid == 64) vec[192] = ss.gL;
+    }
+    fence_proxy_async_all();   // the state CTA reads the slot with a bulk copy
+    tc_fence_before();
+    if (ptid == 0) ss.abort = ld_acquire(&ctrl[1]);
+    if (bar_or_n(bar, kPipeThreads, !ok)) goto fail;
+    // every thread's slot writes precede this release (barrier, then gpu fence)
+    if (ptid == 0) {
+      __threadfence();
+      st_release(flags_of(p.ws, s) + (r % kRing), r + 1);
+    }
+    e = ss.claim;
+    if (ss.abort != 0) break;
     continue;
   fail:
-    if (tid == 0) atomicExch(&ctrl[1], 1);
+    if (ptid == 0) atomicExch(&ctrl[1], 1);
     break;
   }
-  if (tid == 0) {
-    if (tiles_pending) mbar_wait_bounded(&ss.bar_tma, tma_par, kLimitNs);
-    if (ld_acquire(&ctrl[1]) == 0) publish(pend_flag, pend_val);
-    else bulk_wait_all();
-  }
+  if (ptid == kIssuer && pend) mbar_wait_bounded(&ss.bar_tma, tma_par, kLimitNs);
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, PT_COLS);
+  if (tid < 32) tmem_dealloc(sh.tmem, PT_COLS);
 }
 
 // ==================================================================== state ==
@@ -697,8 +718,9 @@ __device__ void state_role(const PcParams& p, uint8_t* sm, int s) {
   const uint32_t a_s0 = smem_u32(sm + S_S0), a_dth = smem_u32(sm + S_DTH);
   const uint32_t a_dtl = smem_u32(sm + S_DTL);
   const uint32_t id_d1 = idesc_f16(128, 128, false, false);
-  const uint32_t id_d2 = idesc_f16(128, 256, false, true);
-  const uint32_t id_d3 = idesc_f16(128, 64, false, true);
+  const uint32_t id_p = idesc_f16(128, 128, false, true);
+  const uint32_t id_ob = idesc_f16(128, 128, false, false);
+  const uint32_t id_d3 = idesc_f16(128, 64, false, false);
 
   int issued = 0;                 // slot copies issued (thread 0's view)
   uint32_t par_dt = 0, par_p = 0, par_o = 0;
@@ -797,19 +819,22 @@ __device__ void state_role(const PcParams& p, uint8_t* sm, int s) {
       fence_proxy_async_smem();
       tc_fence_before();
       if (__syncthreads_or(!ok)) { ok = false; break; }
-      // ---- D2 = Delta_hi^T [K~ | M^T hi | M^T lo] (critical), D3 = Delta_lo^T M^T hi ----
+      // ---- P = Delta_hi^T K~ (critical path), then Delta_hi^T [M hi ; M lo]^T and
+      //      Delta_lo^T M_hi^T for the output ----
       if (tid == 32) st_release(flags + kRing, r + 1);   // slot r fully read
       if (tid == 0) {
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
           mma_f16(tmem + ST_D2, sw128_desc(a_dth + ks * 32, 16, 1024),
-                  sw128_desc(a_buf + SL_BKM + ks * 2048, 8192, 1024), id_d2, ks > 0);
+                  sw128_desc(a_buf + SL_BKM + ks * 2048, 8192, 1024), id_p, ks > 0);
         mma_commit(&ss.bar_p);
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-          mma_f16(tmem + ST_D3, sw128_desc(a_dtl + ks * 32, 16, 1024),
-                  sw128_desc(a_buf + SL_BKM + 2 * 8192 + ks * 2048, 8192, 1024), id_d3, ks > 0);
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint64_t bm = sw128_desc(a_buf + SL_BKM + 2 * 8192 + ks * 32, 16, 1024);
+          mma_f16(tmem + ST_OBHH, sw128_desc(a_dth + ks * 32, 16, 1024), bm, id_ob, ks > 0);
+          mma_f16(tmem + ST_D3, sw128_desc(a_dtl + ks * 32, 16, 1024), bm, id_d3, ks > 0);
+        }
         mma_commit(&ss.bar_o);
       }
       // prefetch the next step's slot into the other buffer if it was ready
@@ -831,6 +856,7 @@ __device__ void state_role(const PcParams& p, uint8_t* sm, int s) {
         for (int q = 0; q < 4; ++q)
           *reinterpret_cast<uint4*>(sm + S_S0 + (cg >> 1) * 16384 + swz(row, (cg & 1) * 4 + q)) =
               pack_half8(S + 8 * q);
+        fence_proxy_async_smem();   // the next step's D1 reads S0
       }
       if (!mbar_wait_bounded(&ss.bar_o, par_o, kLimitNs)) ok = false;
       par_o ^= 1;
@@ -856,7 +882,6 @@ __device__ void state_role(const PcParams& p, uint8_t* sm, int s) {
             o[((t0 + t) * p.H_v + h) * kHeadDim + row] = from_f32<To>(p.scale * (acc[j] + part[j]));
         }
       }
-      fence_proxy_async_smem();
       tc_fence_before();
       if (__syncthreads_or(!ok)) { ok = false; break; }
     }
@@ -977,7 +1002,7 @@ int state_ctas(int64_t items, int H_v, int nsm) {
 // that loads the library holds this array until the process exits.
 constexpr int kNoAllocStateCtas = 49;
 constexpr size_t kNoAllocScratchBytes =
-    CTRL_BYTES + (size_t)kNoAllocStateCtas * kRing * SLOT_BYTES;   // 14 617 600 B
+    CTRL_BYTES + (size_t)kNoAllocStateCtas * kRing * SLOT_BYTES;   // 29 218 816 B
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
 // Device address of g_noalloc_scratch on the current device, looked up once

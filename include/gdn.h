@@ -157,7 +157,7 @@ size_t gdn_chunked_prefill_workspace(int N, int64_t T_total, int H_k, int H_v);
  *
  * Arguments, results and numerics are those of gdn_chunked_prefill. The
  * working memory is one static device array of
- * gdn_chunked_prefill_noalloc_scratch_bytes() bytes (14 617 600: the chunk
+ * gdn_chunked_prefill_noalloc_scratch_bytes() bytes (29 218 816: the chunk
  * rings of 49 state CTAs) that every GPU which loads the library holds until
  * the process exits. A problem whose working memory would exceed it returns
  * GDN_ERR_UNSUPPORTED without launching (on a 148-SM B200 none does). The
