@@ -875,15 +875,37 @@ __device__ void state_role(const PcParams& p, uint8_t* sm, int s) {
 #pragma unroll
         for (int j = 0; j < 16; ++j) acc[j] += part[j];
         tmem_ld16(tmem + lane_base + ST_D3 + 16 * cg, part);
+        // stage o (fp32 [64 t][128 rows]) over Delta^T hi/lo, which the output
+        // MMAs no longer read
+        float* stg = reinterpret_cast<float*>(sm + S_DTH);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int t = 16 * cg + j;
-          if (t < L)
-            o[((t0 + t) * p.H_v + h) * kHeadDim + row] = from_f32<To>(p.scale * (acc[j] + part[j]));
-        }
+        for (int j = 0; j < 16; ++j) stg[(16 * cg + j) * kHeadDim + row] = p.scale * (acc[j] + part[j]);
       }
       tc_fence_before();
       if (__syncthreads_or(!ok)) { ok = false; break; }
+      {
+        // rows t < L of the staged tile, 16 output bytes per store
+        constexpr int kPer = 16 / (int)sizeof(To);          // outputs per 16-byte chunk
+        constexpr int kRowChunks = kHeadDim / kPer;
+        const float* stg = reinterpret_cast<const float*>(sm + S_DTH);
+#pragma unroll
+        for (int ci = tid; ci < kChunk * kRowChunks; ci += kPcThreads) {
+          const int t = ci / kRowChunks, part = ci % kRowChunks;
+          if (t < L) {
+            uint4 v;
+            if constexpr (sizeof(To) == 2) {
+              const float4 a = *reinterpret_cast<const float4*>(stg + t * kHeadDim + part * 8);
+              const float4 b = *reinterpret_cast<const float4*>(stg + t * kHeadDim + part * 8 + 4);
+              __nv_bfloat162 h2[4] = {__floats2bfloat162_rn(a.x, a.y), __floats2bfloat162_rn(a.z, a.w),
+                                      __floats2bfloat162_rn(b.x, b.y), __floats2bfloat162_rn(b.z, b.w)};
+              v = *reinterpret_cast<const uint4*>(h2);
+            } else {
+              v = *reinterpret_cast<const uint4*>(stg + t * kHeadDim + part * 4);
+            }
+            *reinterpret_cast<uint4*>(o + ((t0 + t) * p.H_v + h) * kHeadDim + part * kPer) = v;
+          }
+        }
+      }
     }
     if (p.state_out) {
       float* dst = p.state_out + (nh * kHeadDim + row) * kHeadDim + cg * 32;
