@@ -129,6 +129,7 @@ struct PrepSmall {
 struct StateSmall {
   uint32_t tmem;
   int ok;
+  int pf;     // step r+1's slot was seen released (acquire) during step r
   uint64_t bar_slot[2], bar_dt, bar_p, bar_o;
 };
 
@@ -765,15 +766,12 @@ __device__ void state_role(const PcParams& p, uint8_t* sm, int s) {
       const uint32_t a_buf = smem_u32(buf);
       const int64_t t0 = s0 + (int64_t)c * kChunk;
       const int L = (int)((s1 - t0) < kChunk ? (s1 - t0) : kChunk);
-      int poll = 0;
       if (tid == 32) {
         ss.ok = 1;
         if (issued == r) {
           if (issue_copy(r, false)) issued = r + 1;
           else ss.ok = 0;
         }
-        // early, non-blocking look at the next slot's flag (consumed after the readout)
-        if (issued == r + 1 && r + 1 < total) poll = ld_relaxed(flags + ((r + 1) % kRing));
       }
       __syncthreads();
       if (!ss.ok) { ok = false; break; }
@@ -797,6 +795,13 @@ __device__ void state_role(const PcParams& p, uint8_t* sm, int s) {
         }
         mma_commit(&ss.bar_dt);
       }
+      // gpu-scope flag work, in the shadow of D1 (each access costs a memory
+      // round trip): release slot r (its image is in shared memory, its U^T loads
+      // were issued above) and look, with acquire, whether step r+1 is published;
+      // the barrier after the readout carries that to thread 32, which copies
+      if (tid == 64) st_release(flags + kRing, r + 1);
+      if (tid == 96)
+        ss.pf = (r + 1 < total && ld_acquire(flags + ((r + 1) % kRing)) >= r + 2) ? 1 : 0;
       if (!mbar_wait_bounded(&ss.bar_dt, par_dt, kLimitNs)) ok = false;
       par_dt ^= 1;
       tc_fence_after();
@@ -821,7 +826,6 @@ __device__ void state_role(const PcParams& p, uint8_t* sm, int s) {
       if (__syncthreads_or(!ok)) { ok = false; break; }
       // ---- P = Delta_hi^T K~ (critical path), then Delta_hi^T [M hi ; M lo]^T and
       //      Delta_lo^T M_hi^T for the output ----
-      if (tid == 32) st_release(flags + kRing, r + 1);   // slot r fully read
       if (tid == 0) {
         tc_fence_after();
 #pragma unroll
@@ -837,9 +841,9 @@ __device__ void state_role(const PcParams& p, uint8_t* sm, int s) {
         }
         mma_commit(&ss.bar_o);
       }
-      // prefetch the next step's slot into the other buffer if it was ready
-      if (tid == 32 && issued == r + 1 && r + 1 < total && poll >= r + 2) {
-        fence_acq_rel_gpu();
+      // copy step r+1's slot into the other buffer (free since step r-1 ended)
+      // if it was seen published, in the shadow of P
+      if (tid == 32 && issued == r + 1 && ss.pf) {
         issue_copy(r + 1, true);
         issued = r + 2;
       }
