@@ -55,17 +55,20 @@ constexpr int kRing = 6;            // slots per state CTA: how far prep may run
 constexpr uint64_t kLimitNs = 2000000000ull;
 
 // ---- ring slot (global), 1024-aligned sections ---------------------------
-// B operand of S0 [-W ; Q]^T: K-major, [2 d_k blocks][128 rows][64], rows 0-63 = -W
-// (token t), rows 64-127 = Q (token t), binary16.
+// B operand of S0 [-W ; Q~]^T: K-major, [2 d_k blocks][128 rows][64], rows 0-63 = -W
+// (token t), rows 64-127 = Q~ = diag(e^G) Q (token t), binary16.
 constexpr uint32_t SL_WQ = 0;
 // B operands of Delta^T K~ and Delta^T M^T, four 8 KB blocks: K~ = diag(e^{G_L-G}) K,
-// MN-major [64 tokens s][64 d_k] (d_k 0-63, 64-127), then the strictly lower M
-// (M[t][s] = M_ts for s < t) as binary16 high and low parts, K-major [64 t][64 s].
+// MN-major [64 tokens s][64 d_k] (d_k 0-63, 64-127), then the lower triangle of M
+// (M[t][s] = M_ts for s <= t) as binary16 high and low parts, K-major [64 t][64 s].
 constexpr uint32_t SL_BKM = 32768;
-constexpr uint32_t SL_VEC = 65536;     // gamma[64] tail[64] mdiag[64] gL
+constexpr uint32_t SL_VEC = 65536;     // gL (the chunk's total decay)
 constexpr uint32_t SL_IMG = 66560;     // bytes of the shared-memory image above
 constexpr uint32_t SL_UT = 66560;      // U^T fp32 [64 t][128 i] (the consumer reads it from L2)
 constexpr uint32_t SLOT_BYTES = 99328;
+// state CTA use of a slot image buffer once its MMAs are done: the [-W ; Q] area
+// stages that step's fp32 outputs, the K~/M area receives the next step's U^T
+constexpr uint32_t S_STG_OFF = SL_WQ, S_UT_OFF = SL_BKM;
 
 constexpr uint32_t CTRL_BYTES = 16384; // counter, abort word, per-state-CTA flags
 constexpr int kFlagStride = 16;        // ints per state CTA: full[kRing], consumed
@@ -96,11 +99,11 @@ constexpr uint32_t PC_SMEM_ALLOC = PC_SMEM_BYTES + 1024;
 // prep, per pipeline (256 columns each): Gram [128 x 64] at 0, then W^T as
 // [hi part | lo part] column halves at 0 and U^T the same way at 128
 constexpr uint32_t PT_GR = 0, PT_W = 0, PT_U = 128, PT_PIPE = 256, PT_COLS = 512;
-// state: D1 = S0 [-W ; Q]^T -> [Delta^T - U^T | S0 Q^T];
-//        D2 = Delta_hi^T K~ -> P;  Delta_hi^T [M hi ; M lo]^T -> [OB_hh | OB_hl];
-//        D3 = Delta_lo^T M_hi^T
-constexpr uint32_t ST_D1 = 0, ST_OA = 64, ST_D2 = 128, ST_OBHH = 256, ST_OBHL = 320,
-                   ST_D3 = 384, ST_COLS = 512;
+// state: D1 = S0 [-W ; Q~]^T -> [Delta^T - U^T | OA = S0 Q~^T], in one of two column
+//        sets by step parity (a step's OA outlives the next step's D1), and
+//        Delta_lo^T M_hi^T accumulated onto OA;  P = Delta_hi^T K~;
+//        OB = Delta_hi^T [M hi ; M lo]^T -> [OB_hh | OB_hl].  o^T = scale (OA + OB_hh + OB_hl)
+constexpr uint32_t ST_D1A = 0, ST_P = 128, ST_D1B = 256, ST_OB = 384, ST_COLS = 512;
 
 struct PcParams {
   const void* g; const void* beta;
@@ -113,7 +116,7 @@ struct PcParams {
 
 constexpr int kCuCache = 513;   // sequences whose boundaries the prep CTAs keep on chip
 struct PipeSmall {
-  float G[64], beta[64], gamma[64], bg[64], tail[64], mdiag[64];
+  float G[64], beta[64], gamma[64], bg[64], tail[64];
   float gL;
   int claim;
   int ok;
@@ -130,7 +133,7 @@ struct StateSmall {
   uint32_t tmem;
   int ok;
   int pf;     // step r+1's slot was seen released (acquire) during step r
-  uint64_t bar_slot[2], bar_dt, bar_p, bar_o;
+  uint64_t bar_slot[2], bar_ut[2], bar_dt, bar_p, bar_o;
 };
 
 __device__ __forceinline__ uint32_t swz(int r, int c) {
@@ -483,14 +486,15 @@ __device__ void prep_role(const PcParams& p, const CUtensorMap* tm_q, const CUte
       }
       mma_commit(&ss.bar_mma);
     }
-    // meanwhile: binary16 images of K~ = diag(tail) K and of Q, straight to the slot
+    // meanwhile: binary16 images of K~ = diag(tail) K and Q~ = diag(gamma) Q, straight
+    // to the slot
 #pragma unroll 2
     for (int idx = ptid; idx < 2048; idx += kPipeThreads) {
       const int which = idx >> 10, b = (idx >> 9) & 1, x = idx & 511;
       const uint8_t* src = kq + b * 16384 + which * 8192 + x * 16;
       float f[8];
       load8(reinterpret_cast<const __nv_bfloat16*>(src), f);
-      const float sc = which == 0 ? ss.tail[x >> 3] : 1.f;
+      const float sc = which == 0 ? ss.tail[x >> 3] : ss.gamma[x >> 3];
 #pragma unroll
       for (int u = 0; u < 8; ++u) f[u] *= sc;
       uint8_t* dst = which == 0 ? slot + SL_BKM + b * 8192 + x * 16
@@ -521,8 +525,7 @@ __device__ void prep_role(const PcParams& p, const CUtensorMap* tm_q, const CUte
       }
     } else {
       // lanes 64-127 (query token t = row - 64), columns s = 32cg..32cg+31:
-      // M[t][s] = e^{G_t-G_s} q_t.k_s for s < t as binary16 high and low parts, and
-      // the diagonal M_tt = q_t.k_t
+      // M[t][s] = e^{G_t-G_s} q_t.k_s for s <= t as binary16 high and low parts
       const int t = row - 64, c0 = 32 * cg;
       uint8_t* mh = slot + SL_BKM + 2 * 8192;
       uint8_t* ml = slot + SL_BKM + 3 * 8192;
@@ -542,8 +545,7 @@ __device__ void prep_role(const PcParams& p, const CUtensorMap* tm_q, const CUte
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
             const int s2 = c0 + 8 * q + u;
-            if (s2 == t) ss.mdiag[t] = v[8 * q + u];
-            m8[u] = (s2 < t) ? __expf(Gt - ss.G[s2]) * v[8 * q + u] : 0.f;
+            m8[u] = (s2 <= t) ? __expf(Gt - ss.G[s2]) * v[8 * q + u] : 0.f;
           }
           uint4 hi, lo;
           split_half8(m8, hi, lo);
@@ -657,12 +659,7 @@ __device__ void prep_role(const PcParams& p, const CUtensorMap* tm_q, const CUte
         for (int j = 0; j < 16; ++j) ut[(tb0 + j) * kHeadDim + row] = v[j] + vl[j];
       }
       float* vec = reinterpret_cast<float*>(slot + SL_VEC);
-      if (ptid < 64) {
-        vec[ptid] = ss.gamma[ptid];
-        vec[64 + ptid] = ss.tail[ptid];
-        vec[128 + ptid] = ss.mdiag[ptid];
-      }
-      if (ptid == 64) vec[192] = ss.gL;
+      if (ptid == 0) vec[0] = ss.gL;
     }
     fence_proxy_async_all();   // the state CTA reads the slot with a bulk copy
     tc_fence_before();
@@ -706,6 +703,8 @@ __device__ void state_role(const PcParams& p, uint8_t* sm, int s) {
   if (tid == 32) {
     mbar_init(&ss.bar_slot[0], 1);
     mbar_init(&ss.bar_slot[1], 1);
+    mbar_init(&ss.bar_ut[0], 1);
+    mbar_init(&ss.bar_ut[1], 1);
     mbar_init(&ss.bar_dt, 1);
     mbar_init(&ss.bar_p, 1);
     mbar_init(&ss.bar_o, 1);
@@ -723,7 +722,8 @@ __device__ void state_role(const PcParams& p, uint8_t* sm, int s) {
   const uint32_t id_ob = idesc_f16(128, 128, false, false);
   const uint32_t id_d3 = idesc_f16(128, 64, false, false);
 
-  int issued = 0;                 // slot copies issued (thread 0's view)
+  int issued = 0;                 // slot image copies issued (thread 32's view)
+  int ut_issued = 0;              // U^T copies issued (thread 32's view)
   uint32_t par_dt = 0, par_p = 0, par_o = 0;
   bool ok = true;
   int r = 0;
@@ -738,6 +738,58 @@ __device__ void state_role(const PcParams& p, uint8_t* sm, int s) {
     bulk_g2s(sm + S_BUF + (step & 1) * SL_IMG, slot_of(p.ws, s, step), SL_IMG, bar);
     return true;
   };
+  // U^T of `step` goes to the other buffer's K~/M area, free once step-1's output
+  // MMAs are done (the caller has acquired the slot and fenced the async proxy)
+  auto issue_ut = [&](int step) {
+    const int ub = (step + 1) & 1;
+    mbar_arrive_expect_tx(&ss.bar_ut[ub], 32768);
+    bulk_g2s(sm + S_BUF + ub * SL_IMG + S_UT_OFF, slot_of(p.ws, s, step) + SL_UT, 32768,
+             &ss.bar_ut[ub]);
+  };
+  // staged outputs of an earlier step: rows t < L, 16 output bytes per store
+  auto copy_out = [&](const uint8_t* stage, int64_t ot0, int oL, int oh) {
+    constexpr int kPer = 16 / (int)sizeof(To);          // outputs per 16-byte chunk
+    constexpr int kRowChunks = kHeadDim / kPer;
+    const float* stg = reinterpret_cast<const float*>(stage);
+#pragma unroll
+    for (int ci = tid; ci < kChunk * kRowChunks; ci += kPcThreads) {
+      const int t = ci / kRowChunks, part = ci % kRowChunks;
+      if (t < oL) {
+        uint4 v;
+        if constexpr (sizeof(To) == 2) {
+          const float4 a = *reinterpret_cast<const float4*>(stg + t * kHeadDim + part * 8);
+          const float4 b = *reinterpret_cast<const float4*>(stg + t * kHeadDim + part * 8 + 4);
+          __nv_bfloat162 h2[4] = {__floats2bfloat162_rn(a.x, a.y), __floats2bfloat162_rn(a.z, a.w),
+                                  __floats2bfloat162_rn(b.x, b.y), __floats2bfloat162_rn(b.z, b.w)};
+          v = *reinterpret_cast<const uint4*>(h2);
+        } else {
+          v = *reinterpret_cast<const uint4*>(stg + t * kHeadDim + part * 4);
+        }
+        *reinterpret_cast<uint4*>(o + ((ot0 + t) * p.H_v + oh) * kHeadDim + part * kPer) = v;
+      }
+    }
+  };
+  // this thread's 16 outputs (row, tokens 16cg..16cg+15) of the step whose D1
+  // went to column set d1c: o^T = scale (OA + OB_hh + OB_hl)
+  auto load_out = [&](uint32_t d1c, float (&ov)[16]) {
+    float part[16];
+    tmem_ld16(tmem + lane_base + d1c + 64 + 16 * cg, ov);
+    tmem_ld16(tmem + lane_base + ST_OB + 16 * cg, part);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) ov[j] += part[j];
+    tmem_ld16(tmem + lane_base + ST_OB + 64 + 16 * cg, part);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) ov[j] = p.scale * (ov[j] + part[j]);
+  };
+  // fp32 [64 t][128 rows] stage over a buffer's [-W ; Q~] area
+  auto stage_out = [&](uint8_t* sbuf, const float (&ov)[16]) {
+    float* stg = reinterpret_cast<float*>(sbuf + S_STG_OFF);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) stg[(16 * cg + j) * kHeadDim + row] = ov[j];
+  };
+  bool pend = false;              // a step's outputs wait in TMEM
+  int64_t pend_t0 = 0;
+  int pend_L = 0, pend_h = 0;
 
   for (int i = s; i < p.N * p.H_v && ok; i += p.NS) {
     const int n = i / p.H_v, h = i % p.H_v;
@@ -772,25 +824,25 @@ __device__ void state_role(const PcParams& p, uint8_t* sm, int s) {
           if (issue_copy(r, false)) issued = r + 1;
           else ss.ok = 0;
         }
+        if (ss.ok && ut_issued == r) {
+          issue_ut(r);
+          ut_issued = r + 1;
+        }
       }
       __syncthreads();
       if (!ss.ok) { ok = false; break; }
-      // U^T values of this thread (row, tokens 16cg..16cg+15), straight from L2
-      float ut[16];
-      {
-        const float* src = reinterpret_cast<const float*>(slot_of(p.ws, s, r) + SL_UT);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) ut[j] = __ldcg(src + (16 * cg + j) * kHeadDim + row);
-      }
+      uint8_t* ubuf = sm + S_BUF + ((r + 1) & 1) * SL_IMG;   // U^T of step r
+      const uint32_t d1 = (r & 1) ? ST_D1B : ST_D1A;
+      const uint32_t ut_par = (uint32_t)((r >> 1) & 1);        // step r is its r>>1-th use
       if (!mbar_wait_bounded(&ss.bar_slot[b], (uint32_t)((r >> 1) & 1), kLimitNs)) ok = false;
       if (__syncthreads_or(!ok)) { ok = false; break; }
-      // ---- D1 = S0 [-W ; Q]^T: Delta^T - U^T and S0 Q^T (critical path) ----
+      // ---- D1 = S0 [-W ; Q~]^T: Delta^T - U^T and OA (critical path) ----
       if (tid == 0) {
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_f16(tmem + ST_D1, sw128_desc(a_s0 + off, 16, 1024),
+          mma_f16(tmem + d1, sw128_desc(a_s0 + off, 16, 1024),
                   sw128_desc(a_buf + SL_WQ + off, 16, 1024), id_d1, kk > 0);
         }
         mma_commit(&ss.bar_dt);
@@ -799,20 +851,32 @@ __device__ void state_role(const PcParams& p, uint8_t* sm, int s) {
       // round trip): release slot r (its image is in shared memory, its U^T loads
       // were issued above) and look, with acquire, whether step r+1 is published;
       // the barrier after the readout carries that to thread 32, which copies
-      if (tid == 64) st_release(flags + kRing, r + 1);
+      if (tid == 64) {
+        if (mbar_wait_bounded(&ss.bar_ut[(r + 1) & 1], ut_par, kLimitNs))
+          st_release(flags + kRing, r + 1);
+        else
+          ok = false;
+      }
       if (tid == 96)
         ss.pf = (r + 1 < total && ld_acquire(flags + ((r + 1) % kRing)) >= r + 2) ? 1 : 0;
+      // step r-1's outputs (its MMAs completed before the last barrier)
+      float ov[16];
+      if (pend) {
+        tc_fence_after();
+        load_out((r & 1) ? ST_D1A : ST_D1B, ov);
+      }
+      if (!mbar_wait_bounded(&ss.bar_ut[(r + 1) & 1], ut_par, kLimitNs)) ok = false;
       if (!mbar_wait_bounded(&ss.bar_dt, par_dt, kLimitNs)) ok = false;
       par_dt ^= 1;
       tc_fence_after();
       // ---- Delta = U - W S0^T as binary16 high and low parts ----
       const float* vec = reinterpret_cast<const float*>(buf + SL_VEC);
-      float d[16];
       {
-        float v[16];
-        tmem_ld16(tmem + lane_base + ST_D1 + 16 * cg, v);
+        float v[16], d[16];
+        tmem_ld16(tmem + lane_base + d1 + 16 * cg, v);
+        const float* ut = reinterpret_cast<const float*>(ubuf + S_UT_OFF);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) d[j] = v[j] + ut[j];
+        for (int j = 0; j < 16; ++j) d[j] = v[j] + ut[(16 * cg + j) * kHeadDim + row];
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
           uint4 hi, lo;
@@ -821,39 +885,46 @@ __device__ void state_role(const PcParams& p, uint8_t* sm, int s) {
           *reinterpret_cast<uint4*>(sm + S_DTL + swz(row, 2 * cg + q)) = lo;
         }
       }
+      // stage step r-1's outputs over this step's [-W ; Q~] image (D1 is done)
+      if (pend) stage_out(buf, ov);
       fence_proxy_async_smem();
       tc_fence_before();
       if (__syncthreads_or(!ok)) { ok = false; break; }
       // ---- P = Delta_hi^T K~ (critical path), then Delta_hi^T [M hi ; M lo]^T and
-      //      Delta_lo^T M_hi^T for the output ----
+      //      Delta_lo^T M_hi^T (onto OA) for the output, read during the next step ----
       if (tid == 0) {
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
-          mma_f16(tmem + ST_D2, sw128_desc(a_dth + ks * 32, 16, 1024),
+          mma_f16(tmem + ST_P, sw128_desc(a_dth + ks * 32, 16, 1024),
                   sw128_desc(a_buf + SL_BKM + ks * 2048, 8192, 1024), id_p, ks > 0);
         mma_commit(&ss.bar_p);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
           const uint64_t bm = sw128_desc(a_buf + SL_BKM + 2 * 8192 + ks * 32, 16, 1024);
-          mma_f16(tmem + ST_OBHH, sw128_desc(a_dth + ks * 32, 16, 1024), bm, id_ob, ks > 0);
-          mma_f16(tmem + ST_D3, sw128_desc(a_dtl + ks * 32, 16, 1024), bm, id_d3, ks > 0);
+          mma_f16(tmem + ST_OB, sw128_desc(a_dth + ks * 32, 16, 1024), bm, id_ob, ks > 0);
+          mma_f16(tmem + d1 + 64, sw128_desc(a_dtl + ks * 32, 16, 1024), bm, id_d3, true);
         }
         mma_commit(&ss.bar_o);
       }
-      // copy step r+1's slot into the other buffer (free since step r-1 ended)
-      // if it was seen published, in the shadow of P
+      // copy step r+1's slot into the other buffer (its stage was copied out and its
+      // U^T read before the barrier above) if it was seen published, in the shadow of P
       if (tid == 32 && issued == r + 1 && ss.pf) {
         issue_copy(r + 1, true);
         issued = r + 2;
+      }
+      // and step r-1's outputs leave from the stage
+      if (pend) {
+        copy_out(buf + S_STG_OFF, pend_t0, pend_L, pend_h);
+        pend = false;
       }
       if (!mbar_wait_bounded(&ss.bar_p, par_p, kLimitNs)) ok = false;
       par_p ^= 1;
       tc_fence_after();
       {
-        const float gL = vec[192];
+        const float gL = vec[0];
         float pv[32];
-        tmem_ld32(tmem + lane_base + ST_D2 + 32 * cg, pv);
+        tmem_ld32(tmem + lane_base + ST_P + 32 * cg, pv);
 #pragma unroll
         for (int j = 0; j < 32; ++j) S[j] = fmaf(gL, S[j], pv[j]);
 #pragma unroll
@@ -865,51 +936,18 @@ __device__ void state_role(const PcParams& p, uint8_t* sm, int s) {
       if (!mbar_wait_bounded(&ss.bar_o, par_o, kLimitNs)) ok = false;
       par_o ^= 1;
       tc_fence_after();
-      {
-        // o_t = scale (e^{G_t} (S0 Q^T)_t + (M Delta)_t + M_tt Delta_t)
-        float acc[16], part[16];
-        tmem_ld16(tmem + lane_base + ST_OA + 16 * cg, part);
-#pragma unroll
-        for (int j = 0; j < 16; ++j)
-          acc[j] = fmaf(vec[16 * cg + j], part[j], vec[128 + 16 * cg + j] * d[j]);
-        tmem_ld16(tmem + lane_base + ST_OBHH + 16 * cg, part);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) acc[j] += part[j];
-        tmem_ld16(tmem + lane_base + ST_OBHL + 16 * cg, part);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) acc[j] += part[j];
-        tmem_ld16(tmem + lane_base + ST_D3 + 16 * cg, part);
-        // stage o (fp32 [64 t][128 rows]) over Delta^T hi/lo, which the output
-        // MMAs no longer read
-        float* stg = reinterpret_cast<float*>(sm + S_DTH);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) stg[(16 * cg + j) * kHeadDim + row] = p.scale * (acc[j] + part[j]);
+      // step r+1's U^T into this buffer's K~/M area, which the output MMAs have
+      // finished reading
+      if (tid == 32 && issued == r + 2 && ut_issued == r + 1) {
+        issue_ut(r + 1);
+        ut_issued = r + 2;
       }
       tc_fence_before();
       if (__syncthreads_or(!ok)) { ok = false; break; }
-      {
-        // rows t < L of the staged tile, 16 output bytes per store
-        constexpr int kPer = 16 / (int)sizeof(To);          // outputs per 16-byte chunk
-        constexpr int kRowChunks = kHeadDim / kPer;
-        const float* stg = reinterpret_cast<const float*>(sm + S_DTH);
-#pragma unroll
-        for (int ci = tid; ci < kChunk * kRowChunks; ci += kPcThreads) {
-          const int t = ci / kRowChunks, part = ci % kRowChunks;
-          if (t < L) {
-            uint4 v;
-            if constexpr (sizeof(To) == 2) {
-              const float4 a = *reinterpret_cast<const float4*>(stg + t * kHeadDim + part * 8);
-              const float4 b = *reinterpret_cast<const float4*>(stg + t * kHeadDim + part * 8 + 4);
-              __nv_bfloat162 h2[4] = {__floats2bfloat162_rn(a.x, a.y), __floats2bfloat162_rn(a.z, a.w),
-                                      __floats2bfloat162_rn(b.x, b.y), __floats2bfloat162_rn(b.z, b.w)};
-              v = *reinterpret_cast<const uint4*>(h2);
-            } else {
-              v = *reinterpret_cast<const uint4*>(stg + t * kHeadDim + part * 4);
-            }
-            *reinterpret_cast<uint4*>(o + ((t0 + t) * p.H_v + h) * kHeadDim + part * kPer) = v;
-          }
-        }
-      }
+      pend = true;
+      pend_t0 = t0;
+      pend_L = L;
+      pend_h = h;
     }
     if (p.state_out) {
       float* dst = p.state_out + (nh * kHeadDim + row) * kHeadDim + cg * 32;
@@ -920,11 +958,23 @@ __device__ void state_role(const PcParams& p, uint8_t* sm, int s) {
             ok ? make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]) : make_float4(qnan, qnan, qnan, qnan);
     }
   }
+  if (ok && pend) {   // the last step's outputs
+    float ov[16];
+    tc_fence_after();
+    load_out(((r - 1) & 1) ? ST_D1B : ST_D1A, ov);
+    uint8_t* lbuf = sm + S_BUF + ((r - 1) & 1) * SL_IMG;
+    stage_out(lbuf, ov);
+    __syncthreads();
+    copy_out(lbuf + S_STG_OFF, pend_t0, pend_L, pend_h);
+  }
   if (!ok && tid == 0) atomicExch(&ctrl[1], 1);
   // drain our own copies before leaving (bounded)
-  if (tid == 32)
+  if (tid == 32) {
     for (int st = r; st < issued; ++st)
       mbar_wait_bounded(&ss.bar_slot[st & 1], (uint32_t)((st >> 1) & 1), kLimitNs);
+    for (int st = r; st < ut_issued; ++st)
+      mbar_wait_bounded(&ss.bar_ut[(st + 1) & 1], (uint32_t)((st >> 1) & 1), kLimitNs);
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, ST_COLS);
