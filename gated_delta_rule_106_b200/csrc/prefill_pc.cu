@@ -685,7 +685,7 @@ __device__ void prep_role(const PcParams& p, const CUtensorMap* tm_q, const CUte
 
 // ==================================================================== state ==
 template <class To>
-__device__ void state_role(const PcParams& p, uint8_t* sm, int s) {
+__device__ void state_role(const PcParams& p, const CUtensorMap* tm_o, uint8_t* sm, int s) {
   StateSmall& ss = *reinterpret_cast<StateSmall*>(sm + S_SMALL);
   int* ctrl = reinterpret_cast<int*>(p.ws);
   int* flags = flags_of(p.ws, s);
@@ -733,6 +733,7 @@ __device__ void state_role(const PcParams& p, uint8_t* sm, int s) {
     int* full = flags + (step % kRing);
     if (!acquired && !wait_flag_ge(full, step + 1, &ctrl[1], kLimitNs)) return false;
     fence_proxy_async_all();
+    bulk_wait_read_all();   // an output store of this thread may still read the buffer
     uint64_t* bar = &ss.bar_slot[step & 1];
     mbar_arrive_expect_tx(bar, SL_IMG);
     bulk_g2s(sm + S_BUF + (step & 1) * SL_IMG, slot_of(p.ws, s, step), SL_IMG, bar);
@@ -746,27 +747,25 @@ __device__ void state_role(const PcParams& p, uint8_t* sm, int s) {
     bulk_g2s(sm + S_BUF + ub * SL_IMG + S_UT_OFF, slot_of(p.ws, s, step) + SL_UT, 32768,
              &ss.bar_ut[ub]);
   };
-  // staged outputs of an earlier step: rows t < L, 16 output bytes per store
-  auto copy_out = [&](const uint8_t* stage, int64_t ot0, int oL, int oh) {
-    constexpr int kPer = 16 / (int)sizeof(To);          // outputs per 16-byte chunk
-    constexpr int kRowChunks = kHeadDim / kPer;
-    const float* stg = reinterpret_cast<const float*>(stage);
+  // staged outputs of an earlier step (o's dtype, [64 t][128 rows] over a buffer's
+  // [-W ; Q~] area): a whole bf16 chunk leaves as one tensor store issued by thread
+  // 32, which waits for its read before it next copies into that buffer; a ragged
+  // chunk (whose box would reach the next sequence) or fp32 goes as 16-byte rows
+  auto emit_out = [&](const uint8_t* stage, int64_t ot0, int oL, int oh) {
+    if (sizeof(To) == 2 && oL == kChunk) {
+      if (tid == 32) {
+        tma_store_2d(tm_o, oh * kHeadDim, (int)ot0, stage);
+        bulk_commit();
+      }
+      return;
+    }
+    constexpr int kRowChunks = kHeadDim * (int)sizeof(To) / 16;
 #pragma unroll
     for (int ci = tid; ci < kChunk * kRowChunks; ci += kPcThreads) {
       const int t = ci / kRowChunks, part = ci % kRowChunks;
-      if (t < oL) {
-        uint4 v;
-        if constexpr (sizeof(To) == 2) {
-          const float4 a = *reinterpret_cast<const float4*>(stg + t * kHeadDim + part * 8);
-          const float4 b = *reinterpret_cast<const float4*>(stg + t * kHeadDim + part * 8 + 4);
-          __nv_bfloat162 h2[4] = {__floats2bfloat162_rn(a.x, a.y), __floats2bfloat162_rn(a.z, a.w),
-                                  __floats2bfloat162_rn(b.x, b.y), __floats2bfloat162_rn(b.z, b.w)};
-          v = *reinterpret_cast<const uint4*>(h2);
-        } else {
-          v = *reinterpret_cast<const uint4*>(stg + t * kHeadDim + part * 4);
-        }
-        *reinterpret_cast<uint4*>(o + ((ot0 + t) * p.H_v + oh) * kHeadDim + part * kPer) = v;
-      }
+      if (t < oL)
+        *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(o + ((ot0 + t) * p.H_v + oh) * kHeadDim) +
+                                  part * 16) = *reinterpret_cast<const uint4*>(stage + ci * 16);
     }
   };
   // this thread's 16 outputs (row, tokens 16cg..16cg+15) of the step whose D1
@@ -781,11 +780,22 @@ __device__ void state_role(const PcParams& p, uint8_t* sm, int s) {
 #pragma unroll
     for (int j = 0; j < 16; ++j) ov[j] = p.scale * (ov[j] + part[j]);
   };
-  // fp32 [64 t][128 rows] stage over a buffer's [-W ; Q~] area
+  // [64 t][128 rows] stage in o's dtype over a buffer's [-W ; Q~] area
   auto stage_out = [&](uint8_t* sbuf, const float (&ov)[16]) {
-    float* stg = reinterpret_cast<float*>(sbuf + S_STG_OFF);
+    if constexpr (sizeof(To) == 2) {
+      uint16_t* stg = reinterpret_cast<uint16_t*>(sbuf + S_STG_OFF);
 #pragma unroll
-    for (int j = 0; j < 16; ++j) stg[(16 * cg + j) * kHeadDim + row] = ov[j];
+      for (int j = 0; j < 16; j += 2) {
+        const __nv_bfloat162 h2 = __floats2bfloat162_rn(ov[j], ov[j + 1]);
+        const uint32_t hb = *reinterpret_cast<const uint32_t*>(&h2);
+        stg[(16 * cg + j) * kHeadDim + row] = (uint16_t)(hb & 0xffffu);
+        stg[(16 * cg + j + 1) * kHeadDim + row] = (uint16_t)(hb >> 16);
+      }
+    } else {
+      float* stg = reinterpret_cast<float*>(sbuf + S_STG_OFF);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) stg[(16 * cg + j) * kHeadDim + row] = ov[j];
+    }
   };
   bool pend = false;              // a step's outputs wait in TMEM
   int64_t pend_t0 = 0;
@@ -915,7 +925,7 @@ __device__ void state_role(const PcParams& p, uint8_t* sm, int s) {
       }
       // and step r-1's outputs leave from the stage
       if (pend) {
-        copy_out(buf + S_STG_OFF, pend_t0, pend_L, pend_h);
+        emit_out(buf + S_STG_OFF, pend_t0, pend_L, pend_h);
         pend = false;
       }
       if (!mbar_wait_bounded(&ss.bar_p, par_p, kLimitNs)) ok = false;
@@ -964,8 +974,9 @@ __device__ void state_role(const PcParams& p, uint8_t* sm, int s) {
     load_out(((r - 1) & 1) ? ST_D1B : ST_D1A, ov);
     uint8_t* lbuf = sm + S_BUF + ((r - 1) & 1) * SL_IMG;
     stage_out(lbuf, ov);
+    fence_proxy_async_smem();
     __syncthreads();
-    copy_out(lbuf + S_STG_OFF, pend_t0, pend_L, pend_h);
+    emit_out(lbuf + S_STG_OFF, pend_t0, pend_L, pend_h);
   }
   if (!ok && tid == 0) atomicExch(&ctrl[1], 1);
   // drain our own copies before leaving (bounded)
@@ -974,6 +985,7 @@ __device__ void state_role(const PcParams& p, uint8_t* sm, int s) {
       mbar_wait_bounded(&ss.bar_slot[st & 1], (uint32_t)((st >> 1) & 1), kLimitNs);
     for (int st = r; st < ut_issued; ++st)
       mbar_wait_bounded(&ss.bar_ut[(st + 1) & 1], (uint32_t)((st >> 1) & 1), kLimitNs);
+    bulk_wait_all();   // output stores complete
   }
   tc_fence_before();
   __syncthreads();
@@ -984,11 +996,12 @@ template <class Tg, class To>
 __global__ void __launch_bounds__(kPcThreads, 1)
 prefill_pc_kernel(const __grid_constant__ CUtensorMap tm_q,
                   const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v, const PcParams p) {
+                  const __grid_constant__ CUtensorMap tm_v,
+                  const __grid_constant__ CUtensorMap tm_o, const PcParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  if ((int)blockIdx.x < p.NS) state_role<To>(p, sm, blockIdx.x);
+  if ((int)blockIdx.x < p.NS) state_role<To>(p, &tm_o, sm, blockIdx.x);
   else prep_role<Tg>(p, &tm_q, &tm_k, &tm_v, sm);
 }
 
@@ -1019,6 +1032,19 @@ bool make_map(CUtensorMap* m, const void* base, int64_t cols, int64_t rows, int6
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// bf16 output [rows][cols] (dense), 128 x 64 boxes, unswizzled
+bool make_out_map(CUtensorMap* m, void* base, int64_t cols, int64_t rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(cols * 2)};
+  cuuint32_t box[2] = {(cuuint32_t)kHeadDim, (cuuint32_t)kChunk};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int sm_count() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
@@ -1028,11 +1054,16 @@ int sm_count() {
 
 template <class Tg, class To>
 cudaError_t launch_typed(const RecurArgs& a, int nsm, int NS) {
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo;
   if (!make_map(&mq, a.q, (int64_t)a.H_k * kHeadDim, a.T_total, a.q_row_stride) ||
       !make_map(&mk, a.k, (int64_t)a.H_k * kHeadDim, a.T_total, a.k_row_stride) ||
       !make_map(&mv, a.v, (int64_t)a.H_v * kHeadDim, a.T_total, a.v_row_stride))
     return cudaErrorInvalidValue;
+  if (sizeof(To) == 2) {   // whole-chunk output tiles [64 tokens][128] leave by TMA
+    if (!make_out_map(&mo, a.o, (int64_t)a.H_v * kHeadDim, a.T_total)) return cudaErrorInvalidValue;
+  } else {
+    mo = mv;   // unused: fp32 outputs are stored by the threads
+  }
   auto kern = prefill_pc_kernel<Tg, To>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)PC_SMEM_ALLOC);
@@ -1051,7 +1082,7 @@ cudaError_t launch_typed(const RecurArgs& a, int nsm, int NS) {
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, p);
+  e = cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, mo, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
