@@ -5,12 +5,16 @@
 // q and k channels are L2-normalised per 128-channel head before they enter
 // the recurrence.
 //
-// HBM-bound: each token row is read once (plus a 3-row halo per tile, served
-// from L2) and written once. A thread owns 8 consecutive channels (one 16-byte
-// bf16 vector) for a run of kRowsPerTile tokens and keeps the last three
-// pre-conv rows in registers as a sliding window; 16 threads cover one
-// 128-channel head, so the L2 norm is a 16-lane shuffle reduction. A warp
-// reads/writes 512 contiguous bytes of a row per access.
+// HBM-bound: each token row is read from HBM once and written once. A thread
+// owns 8 consecutive channels (one 16-byte bf16 vector) of a tile of tokens and
+// issues every load its outputs need before it computes, so that many loads
+// are in flight. A tile whose tokens and their three predecessors all lie in
+// one sequence (the common case in prefill) loads that window of rows once; a
+// tile that meets a sequence start takes each token's predecessors from x inside
+// its sequence and from the conv cache (or zeros) before its start. All threads
+// of a block work on the same tokens, so the sequence bookkeeping is uniform;
+// 16 threads cover one 128-channel head, so the L2 norm is a 16-lane shuffle
+// reduction.
 #include "gdn_common.cuh"
 #include "launch.h"
 
@@ -18,8 +22,27 @@ namespace gdn {
 namespace {
 
 constexpr int kConvThreads = 128;
-constexpr int kRowsPerTile = 16;
+// tokens per tile (window path), and per batch of the per-token-source path;
+// either way the loaded vectors of a thread stay in registers
+template <class Tx> __host__ __device__ constexpr int conv_tile() { return sizeof(Tx) == 2 ? 8 : 4; }
+template <class Tx> __host__ __device__ constexpr int conv_batch() { return sizeof(Tx) == 2 ? 4 : 2; }
 
+template <class Tw>
+__device__ __forceinline__ void load_taps(const Tw* w, int c, float (&wt)[4][8]);
+template <class Tw>
+__device__ __forceinline__ void load_taps_bias(const Tw* w, const Tw* bias, int c, bool active,
+                                               float (&wt)[4][8], float (&b)[8]) {
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    b[e] = 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) wt[j][e] = 0.f;
+  }
+  if (active) {
+    load_taps(w, c, wt);
+    if (bias) load8(bias + c, b);
+  }
+}
 template <class Tw>
 __device__ __forceinline__ void load_taps(const Tw* w, int c, float (&wt)[4][8]) {
   // w is [C, 4]: the 8 channels' taps are 32 consecutive values.
@@ -35,15 +58,43 @@ __device__ __forceinline__ void load_taps(const Tw* w, int c, float (&wt)[4][8])
   }
 }
 
-template <class Tx>
-__device__ __forceinline__ void load_hist(const Tx* cs_in, int n, int C, int r,
-                                          int c, float (&h)[8]) {
-  if (cs_in) {
-    load8(cs_in + ((int64_t)n * 3 + r) * C + c, h);
-  } else {
+// one output token: taps over its four pre-conv inputs (oldest first), SiLU, and
+// the per-head L2 norm for the leading l2c channels
+template <class Tx, class Ty>
+__device__ __forceinline__ void conv_token(const Raw8<Tx>& s0, const Raw8<Tx>& s1,
+                                           const Raw8<Tx>& s2, const Raw8<Tx>& s3,
+                                           const float (&wt)[4][8], const float (&b)[8],
+                                           int c, int l2c, float eps, bool store, Ty* dst) {
+  float a[8], f[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) h[e] = 0.f;
+  for (int e = 0; e < 8; ++e) a[e] = b[e];
+  s0.to_f32(f);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) a[e] = fmaf(wt[0][e], f[e], a[e]);
+  s1.to_f32(f);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) a[e] = fmaf(wt[1][e], f[e], a[e]);
+  s2.to_f32(f);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) a[e] = fmaf(wt[2][e], f[e], a[e]);
+  s3.to_f32(f);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) a[e] = fmaf(wt[3][e], f[e], a[e]);
+  float out[8], ss = 0.f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    out[e] = silu(a[e]);
+    ss = fmaf(out[e], out[e], ss);
   }
+  // 16 lanes = one 128-channel head
+#pragma unroll
+  for (int off = 8; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+  if (c < l2c) {
+    const float inv = rsqrtf(ss + eps);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) out[e] *= inv;
+  }
+  if (store) store8(dst, out);
 }
 
 template <class Tx, class Tw, class Ty>
@@ -52,79 +103,64 @@ conv_silu_kernel(const Tx* __restrict__ x, int64_t xs, const Tw* __restrict__ w,
                  const Tw* __restrict__ bias, int C, int l2c, float eps,
                  const int32_t* __restrict__ cu, int N, int64_t T,
                  const Tx* __restrict__ cs_in, Ty* __restrict__ y, int64_t ys) {
+  constexpr int R = conv_tile<Tx>(), RB = conv_batch<Tx>();
   const int c = (blockIdx.x * kConvThreads + threadIdx.x) * 8;
   const bool active = c < C;
-  const int64_t t0 = (int64_t)blockIdx.y * kRowsPerTile;
-  const int64_t t1 = t0 + kRowsPerTile < T ? t0 + kRowsPerTile : T;
-
-  float wt[4][8], b[8], h[3][8];   // h[j] = pre-conv row t-3+j
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    b[e] = 0.f;
-#pragma unroll
-    for (int j = 0; j < 3; ++j) h[j][e] = 0.f;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) wt[j][e] = 0.f;
-  }
-  if (active) {
-    load_taps(w, c, wt);
-    if (bias) load8(bias + c, b);
-  }
+  const int64_t t0 = (int64_t)blockIdx.y * R;
 
   int n = seq_of(cu, N, t0);
   int64_t s_start = clamp_t(__ldg(cu + n), T);
   int64_t s_end = clamp_t(__ldg(cu + n + 1), T);
-  if (active) {
+
+  if (t0 - 3 >= s_start && t0 + R <= s_end) {
+    // window path: rows t0-3 .. t0+R-1, each loaded once
+    Raw8<Tx> win[R + 3];
 #pragma unroll
-    for (int j = 0; j < 3; ++j) {
-      const int64_t p = t0 - 3 + j;
-      if (p >= s_start) load8(x + p * xs + c, h[j]);
-      else load_hist(cs_in, n, C, (int)(3 + (p - s_start)), c, h[j]);
+    for (int j = 0; j < R + 3; ++j) {
+      win[j].zero();
+      if (active) win[j].load(x + (t0 - 3 + j) * xs + c);
     }
+    float wt[4][8], b[8];
+    load_taps_bias(w, bias, c, active, wt, b);
+#pragma unroll
+    for (int i = 0; i < R; ++i)
+      conv_token<Tx, Ty>(win[i], win[i + 1], win[i + 2], win[i + 3], wt, b, c, l2c, eps, active,
+                         y + (t0 + i) * ys + c);
+    return;
   }
 
-  for (int64_t t = t0; t < t1; ++t) {
-    if (t >= s_end) {
-      // enter the sequence that starts at t (skipping empty ones)
-      while (n < N - 1 && t >= s_end) {
+  float wt[4][8], b[8];
+  load_taps_bias(w, bias, c, active, wt, b);
+  // per-token sources, RB tokens at a time: src[i][k] = pre-conv input of token
+  // t at lag 3-k (k = 3: the token itself)
+#pragma unroll 1
+  for (int i0 = 0; i0 < R; i0 += RB) {
+    Raw8<Tx> src[RB][4];
+#pragma unroll
+    for (int i = 0; i < RB; ++i) {
+      const int64_t t = t0 + i0 + i;
+      while (n < N - 1 && t >= s_end) {   // enter the sequence holding t (skip empty ones)
         ++n;
         s_start = clamp_t(__ldg(cu + n), T);
         s_end = clamp_t(__ldg(cu + n + 1), T);
       }
-      if (active) {
+      // a token past the last sequence is treated as the start of one
+      const int64_t st = t >= s_end ? t : s_start;
 #pragma unroll
-        for (int j = 0; j < 3; ++j) load_hist(cs_in, n, C, j, c, h[j]);
+      for (int k = 0; k < 4; ++k) {
+        const int64_t pr = t - 3 + k;
+        src[i][k].zero();
+        if (active && t < T) {
+          if (pr >= st) src[i][k].load(x + pr * xs + c);
+          else if (cs_in) src[i][k].load(cs_in + ((int64_t)n * 3 + (3 + (pr - st))) * C + c);
+        }
       }
     }
-    float cur[8], out[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) cur[e] = 0.f;
-    if (active) load8(x + t * xs + c, cur);
-    float ss = 0.f;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      float a = b[e];
-      a = fmaf(wt[0][e], h[0][e], a);
-      a = fmaf(wt[1][e], h[1][e], a);
-      a = fmaf(wt[2][e], h[2][e], a);
-      a = fmaf(wt[3][e], cur[e], a);
-      out[e] = silu(a);
-      ss = fmaf(out[e], out[e], ss);
-    }
-    // 16 lanes = one 128-channel head
-#pragma unroll
-    for (int off = 8; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-    if (c < l2c) {
-      const float inv = 1.0f / sqrtf(ss + eps);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) out[e] *= inv;
-    }
-    if (active) store8(y + t * ys + c, out);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      h[0][e] = h[1][e];
-      h[1][e] = h[2][e];
-      h[2][e] = cur[e];
+    for (int i = 0; i < RB; ++i) {
+      const int64_t t = t0 + i0 + i;
+      conv_token<Tx, Ty>(src[i][0], src[i][1], src[i][2], src[i][3], wt, b, c, l2c, eps,
+                         active && t < T, y + t * ys + c);
     }
   }
 }
@@ -167,8 +203,9 @@ __global__ void conv_state_kernel(const char* __restrict__ x, int64_t xs_bytes,
 template <class Tx, class Tw, class Ty>
 cudaError_t launch_typed(const ConvArgs& a) {
   if (a.T_total > 0) {
+    constexpr int R = conv_tile<Tx>();
     dim3 grid((unsigned)((a.channels / 8 + kConvThreads - 1) / kConvThreads),
-              (unsigned)((a.T_total + kRowsPerTile - 1) / kRowsPerTile));
+              (unsigned)((a.T_total + R - 1) / R));
     conv_silu_kernel<Tx, Tw, Ty><<<grid, kConvThreads, 0, a.stream>>>(
         static_cast<const Tx*>(a.x), a.x_row_stride,
         static_cast<const Tw*>(a.w), static_cast<const Tw*>(a.bias), a.channels,
