@@ -58,37 +58,29 @@ __device__ __forceinline__ void load_taps(const Tw* w, int c, float (&wt)[4][8])
   }
 }
 
-// one output token: taps over its four pre-conv inputs (oldest first), SiLU, and
-// the per-head L2 norm for the leading l2c channels
-template <class Tx, class Ty>
-__device__ __forceinline__ void conv_token(const Raw8<Tx>& s0, const Raw8<Tx>& s1,
-                                           const Raw8<Tx>& s2, const Raw8<Tx>& s3,
+// one output token from its four pre-conv inputs (oldest first, as floats):
+// taps, SiLU, and the per-head L2 norm for the leading l2c channels
+template <class Ty>
+__device__ __forceinline__ void conv_token(const float (&f0)[8], const float (&f1)[8],
+                                           const float (&f2)[8], const float (&f3)[8],
                                            const float (&wt)[4][8], const float (&b)[8],
-                                           int c, int l2c, float eps, bool store, Ty* dst) {
-  float a[8], f[8];
+                                           int c, int l2c, bool any_l2, float eps, bool store,
+                                           Ty* dst) {
+  float a[8];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) a[e] = b[e];
-  s0.to_f32(f);
-#pragma unroll
-  for (int e = 0; e < 8; ++e) a[e] = fmaf(wt[0][e], f[e], a[e]);
-  s1.to_f32(f);
-#pragma unroll
-  for (int e = 0; e < 8; ++e) a[e] = fmaf(wt[1][e], f[e], a[e]);
-  s2.to_f32(f);
-#pragma unroll
-  for (int e = 0; e < 8; ++e) a[e] = fmaf(wt[2][e], f[e], a[e]);
-  s3.to_f32(f);
-#pragma unroll
-  for (int e = 0; e < 8; ++e) a[e] = fmaf(wt[3][e], f[e], a[e]);
+  for (int e = 0; e < 8; ++e)
+    a[e] = fmaf(wt[3][e], f3[e], fmaf(wt[2][e], f2[e], fmaf(wt[1][e], f1[e], fmaf(wt[0][e], f0[e], b[e]))));
   float out[8], ss = 0.f;
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
     out[e] = silu(a[e]);
     ss = fmaf(out[e], out[e], ss);
   }
-  // 16 lanes = one 128-channel head
+  if (any_l2) {   // block-uniform: some channel of the block is L2-normalised
+    // 16 lanes = one 128-channel head
 #pragma unroll
-  for (int off = 8; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    for (int off = 8; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+  }
   if (c < l2c) {
     const float inv = rsqrtf(ss + eps);
 #pragma unroll
@@ -106,6 +98,7 @@ conv_silu_kernel(const Tx* __restrict__ x, int64_t xs, const Tw* __restrict__ w,
   constexpr int R = conv_tile<Tx>(), RB = conv_batch<Tx>();
   const int c = (blockIdx.x * kConvThreads + threadIdx.x) * 8;
   const bool active = c < C;
+  const bool any_l2 = (int)blockIdx.x * kConvThreads * 8 < l2c;
   const int64_t t0 = (int64_t)blockIdx.y * R;
 
   int n = seq_of(cu, N, t0);
@@ -122,10 +115,23 @@ conv_silu_kernel(const Tx* __restrict__ x, int64_t xs, const Tw* __restrict__ w,
     }
     float wt[4][8], b[8];
     load_taps_bias(w, bias, c, active, wt, b);
+    // each row converted once; the last three stay as floats
+    float h0[8], h1[8], h2[8], h3[8];
+    win[0].to_f32(h0);
+    win[1].to_f32(h1);
+    win[2].to_f32(h2);
+    Ty* dst = y + t0 * ys + c;
 #pragma unroll
-    for (int i = 0; i < R; ++i)
-      conv_token<Tx, Ty>(win[i], win[i + 1], win[i + 2], win[i + 3], wt, b, c, l2c, eps, active,
-                         y + (t0 + i) * ys + c);
+    for (int i = 0; i < R; ++i, dst += ys) {
+      win[i + 3].to_f32(h3);
+      conv_token<Ty>(h0, h1, h2, h3, wt, b, c, l2c, any_l2, eps, active, dst);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        h0[e] = h1[e];
+        h1[e] = h2[e];
+        h2[e] = h3[e];
+      }
+    }
     return;
   }
 
@@ -159,8 +165,12 @@ conv_silu_kernel(const Tx* __restrict__ x, int64_t xs, const Tw* __restrict__ w,
 #pragma unroll
     for (int i = 0; i < RB; ++i) {
       const int64_t t = t0 + i0 + i;
-      conv_token<Tx, Ty>(src[i][0], src[i][1], src[i][2], src[i][3], wt, b, c, l2c, eps,
-                         active && t < T, y + t * ys + c);
+      float f0[8], f1[8], f2[8], f3[8];
+      src[i][0].to_f32(f0);
+      src[i][1].to_f32(f1);
+      src[i][2].to_f32(f2);
+      src[i][3].to_f32(f3);
+      conv_token<Ty>(f0, f1, f2, f3, wt, b, c, l2c, any_l2, eps, active && t < T, y + t * ys + c);
     }
   }
 }
