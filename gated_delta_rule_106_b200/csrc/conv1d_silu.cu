@@ -6,15 +6,15 @@
 // the recurrence.
 //
 // HBM-bound: each token row is read from HBM once and written once. A thread
-// owns 8 consecutive channels (one 16-byte bf16 vector) of a tile of tokens and
+// owns 4 consecutive channels (one 8-byte bf16 vector) of a tile of tokens and
 // issues every load its outputs need before it computes, so that many loads
-// are in flight. A tile whose tokens and their three predecessors all lie in
+// are in flight; 4 channels (not 8) keep the register count low enough for
+// 7 CTAs per SM. A tile whose tokens and their three predecessors all lie in
 // one sequence (the common case in prefill) loads that window of rows once; a
 // tile that meets a sequence start takes each token's predecessors from x inside
 // its sequence and from the conv cache (or zeros) before its start. All threads
-// of a block work on the same tokens, so the sequence bookkeeping is uniform;
-// 16 threads cover one 128-channel head, so the L2 norm is a 16-lane shuffle
-// reduction.
+// of a block work on the same tokens, so the sequence bookkeeping is uniform; a
+// warp covers one 128-channel head, so the L2 norm is a warp shuffle reduction.
 #include "gdn_common.cuh"
 #include "launch.h"
 
@@ -22,71 +22,122 @@ namespace gdn {
 namespace {
 
 constexpr int kConvThreads = 128;
+constexpr int kV = 4;                    // channels per thread
+constexpr int kHeadLanes = kHeadDim / kV; // lanes per 128-channel head
 // tokens per tile (window path), and per batch of the per-token-source path;
 // either way the loaded vectors of a thread stay in registers
 template <class Tx> __host__ __device__ constexpr int conv_tile() { return sizeof(Tx) == 2 ? 8 : 4; }
 template <class Tx> __host__ __device__ constexpr int conv_batch() { return sizeof(Tx) == 2 ? 4 : 2; }
 
-template <class Tw>
-__device__ __forceinline__ void load_taps(const Tw* w, int c, float (&wt)[4][8]);
+// kV consecutive elements kept as loaded
+template <class Tx> struct RawV {
+  static constexpr int kBytes = kV * (int)sizeof(Tx);
+  static constexpr int kWords = kBytes / 4;
+  uint32_t u[kWords];
+  __device__ __forceinline__ void zero() {
+#pragma unroll
+    for (int i = 0; i < kWords; ++i) u[i] = 0u;
+  }
+  __device__ __forceinline__ void load(const Tx* p) {
+    if constexpr (kBytes == 8) {
+      const uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
+      u[0] = v.x; u[1] = v.y;
+    } else {
+#pragma unroll
+      for (int i = 0; i < kBytes / 16; ++i) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(p) + i);
+        u[4 * i] = v.x; u[4 * i + 1] = v.y; u[4 * i + 2] = v.z; u[4 * i + 3] = v.w;
+      }
+    }
+  }
+  __device__ __forceinline__ void to_f32(float (&f)[kV]) const {
+    if constexpr (sizeof(Tx) == 2) {
+#pragma unroll
+      for (int i = 0; i < kWords; ++i) {
+        const float2 t = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u[i]));
+        f[2 * i] = t.x;
+        f[2 * i + 1] = t.y;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < kV; ++i) f[i] = __uint_as_float(u[i]);
+    }
+  }
+};
+template <class T>
+__device__ __forceinline__ void loadV(const T* p, float (&f)[kV]) {
+  RawV<T> r;
+  r.load(p);
+  r.to_f32(f);
+}
+template <class Ty>
+__device__ __forceinline__ void storeV(Ty* p, const float (&f)[kV]) {
+  if constexpr (sizeof(Ty) == 2) {
+    uint32_t u[kV / 2];
+#pragma unroll
+    for (int i = 0; i < kV / 2; ++i) {
+      const __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+      u[i] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+    if constexpr (kV == 4) *reinterpret_cast<uint2*>(p) = make_uint2(u[0], u[1]);
+    else *reinterpret_cast<uint4*>(p) = make_uint4(u[0], u[1], u[2], u[3]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < kV / 4; ++i)
+      reinterpret_cast<float4*>(p)[i] = make_float4(f[4 * i], f[4 * i + 1], f[4 * i + 2], f[4 * i + 3]);
+  }
+}
+
 template <class Tw>
 __device__ __forceinline__ void load_taps_bias(const Tw* w, const Tw* bias, int c, bool active,
-                                               float (&wt)[4][8], float (&b)[8]) {
+                                               float (&wt)[4][kV], float (&b)[kV]) {
 #pragma unroll
-  for (int e = 0; e < 8; ++e) {
+  for (int e = 0; e < kV; ++e) {
     b[e] = 0.f;
 #pragma unroll
     for (int j = 0; j < 4; ++j) wt[j][e] = 0.f;
   }
   if (active) {
-    load_taps(w, c, wt);
-    if (bias) load8(bias + c, b);
-  }
-}
-template <class Tw>
-__device__ __forceinline__ void load_taps(const Tw* w, int c, float (&wt)[4][8]) {
-  // w is [C, 4]: the 8 channels' taps are 32 consecutive values.
-  float f[8];
+    // w is [C, 4]: the kV channels' taps are 4 kV consecutive values
+    float f[kV];
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    load8(w + (int64_t)c * 4 + q * 8, f);
+    for (int q = 0; q < 4; ++q) {
+      loadV(w + (int64_t)c * 4 + q * kV, f);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      int flat = q * 8 + e;          // = (channel - c) * 4 + tap
-      wt[flat & 3][flat >> 2] = f[e];
+      for (int e = 0; e < kV; ++e) {
+        const int flat = q * kV + e;          // = (channel - c) * 4 + tap
+        wt[flat & 3][flat >> 2] = f[e];
+      }
     }
+    if (bias) loadV(bias + c, b);
   }
 }
 
 // one output token from its four pre-conv inputs (oldest first, as floats):
 // taps, SiLU, and the per-head L2 norm for the leading l2c channels
 template <class Ty>
-__device__ __forceinline__ void conv_token(const float (&f0)[8], const float (&f1)[8],
-                                           const float (&f2)[8], const float (&f3)[8],
-                                           const float (&wt)[4][8], const float (&b)[8],
+__device__ __forceinline__ void conv_token(const float (&f0)[kV], const float (&f1)[kV],
+                                           const float (&f2)[kV], const float (&f3)[kV],
+                                           const float (&wt)[4][kV], const float (&b)[kV],
                                            int c, int l2c, bool any_l2, float eps, bool store,
                                            Ty* dst) {
-  float a[8];
+  float out[kV], ss = 0.f;
 #pragma unroll
-  for (int e = 0; e < 8; ++e)
-    a[e] = fmaf(wt[3][e], f3[e], fmaf(wt[2][e], f2[e], fmaf(wt[1][e], f1[e], fmaf(wt[0][e], f0[e], b[e]))));
-  float out[8], ss = 0.f;
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    out[e] = silu(a[e]);
+  for (int e = 0; e < kV; ++e) {
+    const float a = fmaf(wt[3][e], f3[e], fmaf(wt[2][e], f2[e], fmaf(wt[1][e], f1[e], fmaf(wt[0][e], f0[e], b[e]))));
+    out[e] = silu(a);
     ss = fmaf(out[e], out[e], ss);
   }
   if (any_l2) {   // block-uniform: some channel of the block is L2-normalised
-    // 16 lanes = one 128-channel head
 #pragma unroll
-    for (int off = 8; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    for (int off = kHeadLanes / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
   }
   if (c < l2c) {
     const float inv = rsqrtf(ss + eps);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) out[e] *= inv;
+    for (int e = 0; e < kV; ++e) out[e] *= inv;
   }
-  if (store) store8(dst, out);
+  if (store) storeV(dst, out);
 }
 
 template <class Tx, class Tw, class Ty>
@@ -96,27 +147,27 @@ conv_silu_kernel(const Tx* __restrict__ x, int64_t xs, const Tw* __restrict__ w,
                  const int32_t* __restrict__ cu, int N, int64_t T,
                  const Tx* __restrict__ cs_in, Ty* __restrict__ y, int64_t ys) {
   constexpr int R = conv_tile<Tx>(), RB = conv_batch<Tx>();
-  const int c = (blockIdx.x * kConvThreads + threadIdx.x) * 8;
+  const int c = (blockIdx.x * kConvThreads + threadIdx.x) * kV;
   const bool active = c < C;
-  const bool any_l2 = (int)blockIdx.x * kConvThreads * 8 < l2c;
+  const bool any_l2 = (int)blockIdx.x * kConvThreads * kV < l2c;
   const int64_t t0 = (int64_t)blockIdx.y * R;
 
   int n = seq_of(cu, N, t0);
   int64_t s_start = clamp_t(__ldg(cu + n), T);
   int64_t s_end = clamp_t(__ldg(cu + n + 1), T);
 
+  float wt[4][kV], b[kV];
   if (t0 - 3 >= s_start && t0 + R <= s_end) {
     // window path: rows t0-3 .. t0+R-1, each loaded once
-    Raw8<Tx> win[R + 3];
+    RawV<Tx> win[R + 3];
 #pragma unroll
     for (int j = 0; j < R + 3; ++j) {
       win[j].zero();
       if (active) win[j].load(x + (t0 - 3 + j) * xs + c);
     }
-    float wt[4][8], b[8];
     load_taps_bias(w, bias, c, active, wt, b);
     // each row converted once; the last three stay as floats
-    float h0[8], h1[8], h2[8], h3[8];
+    float h0[kV], h1[kV], h2[kV], h3[kV];
     win[0].to_f32(h0);
     win[1].to_f32(h1);
     win[2].to_f32(h2);
@@ -126,7 +177,7 @@ conv_silu_kernel(const Tx* __restrict__ x, int64_t xs, const Tw* __restrict__ w,
       win[i + 3].to_f32(h3);
       conv_token<Ty>(h0, h1, h2, h3, wt, b, c, l2c, any_l2, eps, active, dst);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
+      for (int e = 0; e < kV; ++e) {
         h0[e] = h1[e];
         h1[e] = h2[e];
         h2[e] = h3[e];
@@ -135,13 +186,12 @@ conv_silu_kernel(const Tx* __restrict__ x, int64_t xs, const Tw* __restrict__ w,
     return;
   }
 
-  float wt[4][8], b[8];
   load_taps_bias(w, bias, c, active, wt, b);
   // per-token sources, RB tokens at a time: src[i][k] = pre-conv input of token
   // t at lag 3-k (k = 3: the token itself)
 #pragma unroll 1
   for (int i0 = 0; i0 < R; i0 += RB) {
-    Raw8<Tx> src[RB][4];
+    RawV<Tx> src[RB][4];
 #pragma unroll
     for (int i = 0; i < RB; ++i) {
       const int64_t t = t0 + i0 + i;
@@ -165,7 +215,7 @@ conv_silu_kernel(const Tx* __restrict__ x, int64_t xs, const Tw* __restrict__ w,
 #pragma unroll
     for (int i = 0; i < RB; ++i) {
       const int64_t t = t0 + i0 + i;
-      float f0[8], f1[8], f2[8], f3[8];
+      float f0[kV], f1[kV], f2[kV], f3[kV];
       src[i][0].to_f32(f0);
       src[i][1].to_f32(f1);
       src[i][2].to_f32(f2);
@@ -214,7 +264,7 @@ template <class Tx, class Tw, class Ty>
 cudaError_t launch_typed(const ConvArgs& a) {
   if (a.T_total > 0) {
     constexpr int R = conv_tile<Tx>();
-    dim3 grid((unsigned)((a.channels / 8 + kConvThreads - 1) / kConvThreads),
+    dim3 grid((unsigned)((a.channels / kV + kConvThreads - 1) / kConvThreads),
               (unsigned)((a.T_total + R - 1) / R));
     conv_silu_kernel<Tx, Tw, Ty><<<grid, kConvThreads, 0, a.stream>>>(
         static_cast<const Tx*>(a.x), a.x_row_stride,

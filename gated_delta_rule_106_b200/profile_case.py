@@ -4,6 +4,7 @@
     python -m gated_delta_rule_106_b200.profile_case prefill [--t 8192] [--launches 4]
     python -m gated_delta_rule_106_b200.profile_case conv    [--t 8192] [--launches 4]
     python -m gated_delta_rule_106_b200.profile_case norm    [--t 8192] [--launches 4]
+    python -m gated_delta_rule_106_b200.profile_case dconv   [--n 64]   [--launches 4]
 
 Each case allocates its inputs (synthetic, seeded; larger than the 126 MB L2
 at the defaults so DRAM counters are meaningful, and a few GB at most), runs
@@ -68,8 +69,19 @@ def case_norm(a):
     return lambda: gdn.gdn_gated_rmsnorm(x, z, w, eps=1e-6, y=y)
 
 
+def case_dconv(a):
+    """The decode step's conv: --n one-token sequences, 3-row cache rolled in place."""
+    N = a.n
+    cache = gi.to_bf16(gi.normal(0, "dconv", (N, 3, gi.CONV_CHANNELS))).to(DEV)
+    x = gi.decode_step_inputs(0, N, 0)["x_pre"].to(DEV)
+    w = gi.conv_weight(0).to(DEV)
+    cu = torch.arange(N + 1, dtype=torch.int32, device=DEV)
+    y = torch.empty((N, gi.CONV_CHANNELS), dtype=torch.bfloat16, device=DEV)
+    return lambda: gdn.gdn_conv1d_silu(x, w, cu, conv_state_in=cache, conv_state_out=cache, y=y)
+
+
 CASES = {"decode": case_decode, "prefill": case_prefill, "conv": case_conv,
-         "norm": case_norm}
+         "norm": case_norm, "dconv": case_dconv}
 
 
 def main():
