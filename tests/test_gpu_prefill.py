@@ -138,6 +138,21 @@ def test_bf16_output_and_long_memory_gates():
     check(o, S, o_ref, S_ref, torch.bfloat16, o_dtype=torch.bfloat16)
 
 
+@pytest.mark.parametrize("lens", [[65, 130, 64, 1], [200, 7, 129]])
+def test_bf16_output_ragged_sequences(lens):
+    """bf16 outputs over several sequences: whole chunks leave as tensor-store
+    tiles, a sequence's ragged last chunk as row stores that must stop at the
+    sequence end (the next sequence's rows follow it)."""
+    cu = cu_of(lens)
+    T = int(cu[-1])
+    q, k, v, g, b = random_qkv(15, T, torch.bfloat16)
+    S0 = gi.initial_states(15, len(lens))
+    o_ref, S_ref = oracle.recurrence(f64(q), f64(k), f64(v), f64(g), f64(b),
+                                     f64(S0), cu.numpy())
+    o, S = run_prefill(q, k, v, g, b, cu, state_in=S0, o_dtype=torch.bfloat16)
+    check(o, S, o_ref, S_ref, torch.bfloat16, o_dtype=torch.bfloat16)
+
+
 # ---- layer workloads at full size, checked on sampled head groups ----------
 
 def conv_gpu(x_pre, conv_w, cu, conv_state=None):
