@@ -25,9 +25,12 @@ constexpr int kConvThreads = 128;
 constexpr int kV = 4;                    // channels per thread
 constexpr int kHeadLanes = kHeadDim / kV; // lanes per 128-channel head
 // tokens per tile (window path), and per batch of the per-token-source path;
-// either way the loaded vectors of a thread stay in registers
+// either way the loaded vectors of a thread stay in registers. Calls whose
+// sequences average at most kShortLen tokens (decode) use tiles of 2 tokens:
+// more CTAs, one short batch each.
 template <class Tx> __host__ __device__ constexpr int conv_tile() { return sizeof(Tx) == 2 ? 8 : 4; }
 template <class Tx> __host__ __device__ constexpr int conv_batch() { return sizeof(Tx) == 2 ? 4 : 2; }
+constexpr int kShortLen = 4;
 
 // kV consecutive elements kept as loaded
 template <class Tx> struct RawV {
@@ -140,19 +143,20 @@ __device__ __forceinline__ void conv_token(const float (&f0)[kV], const float (&
   if (store) storeV(dst, out);
 }
 
-template <class Tx, class Tw, class Ty>
+template <class Tx, class Tw, class Ty, int R, int RB>
 __global__ void __launch_bounds__(kConvThreads)
 conv_silu_kernel(const Tx* __restrict__ x, int64_t xs, const Tw* __restrict__ w,
                  const Tw* __restrict__ bias, int C, int l2c, float eps,
                  const int32_t* __restrict__ cu, int N, int64_t T,
                  const Tx* __restrict__ cs_in, Ty* __restrict__ y, int64_t ys) {
-  constexpr int R = conv_tile<Tx>(), RB = conv_batch<Tx>();
   const int c = (blockIdx.x * kConvThreads + threadIdx.x) * kV;
   const bool active = c < C;
   const bool any_l2 = (int)blockIdx.x * kConvThreads * kV < l2c;
   const int64_t t0 = (int64_t)blockIdx.y * R;
 
-  int n = seq_of(cu, N, t0);
+  // short-sequence tiles guess the sequence from equal lengths (one round of loads
+  // for one token per sequence); long ones search
+  int n = R == 2 ? seq_locate(cu, N, T, t0) : seq_of(cu, N, t0);
   int64_t s_start = clamp_t(__ldg(cu + n), T);
   int64_t s_end = clamp_t(__ldg(cu + n + 1), T);
 
@@ -263,10 +267,13 @@ __global__ void conv_state_kernel(const char* __restrict__ x, int64_t xs_bytes,
 template <class Tx, class Tw, class Ty>
 cudaError_t launch_typed(const ConvArgs& a) {
   if (a.T_total > 0) {
-    constexpr int R = conv_tile<Tx>();
+    const bool short_seqs = (int64_t)a.N * kShortLen >= a.T_total;
+    const int R = short_seqs ? 2 : conv_tile<Tx>();
     dim3 grid((unsigned)((a.channels / kV + kConvThreads - 1) / kConvThreads),
               (unsigned)((a.T_total + R - 1) / R));
-    conv_silu_kernel<Tx, Tw, Ty><<<grid, kConvThreads, 0, a.stream>>>(
+    auto kern = short_seqs ? conv_silu_kernel<Tx, Tw, Ty, 2, 2>
+                           : conv_silu_kernel<Tx, Tw, Ty, conv_tile<Tx>(), conv_batch<Tx>()>;
+    kern<<<grid, kConvThreads, 0, a.stream>>>(
         static_cast<const Tx*>(a.x), a.x_row_stride,
         static_cast<const Tw*>(a.w), static_cast<const Tw*>(a.bias), a.channels,
         a.l2norm_channels, a.l2_eps, a.cu_seqlens, a.N, a.T_total,

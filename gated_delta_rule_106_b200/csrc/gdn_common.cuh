@@ -108,4 +108,15 @@ __device__ __forceinline__ int64_t clamp_t(int64_t v, int64_t T) {
   return v < 0 ? 0 : (v > T ? T : v);
 }
 
+// seq_of, starting from the guess that sequences are of equal length: when the
+// guessed sequence brackets t (always, for equal lengths, e.g. one token per
+// sequence) this is one round of two independent loads instead of a chain
+__device__ __forceinline__ int seq_locate(const int32_t* cu, int N, int64_t T, int64_t t) {
+  int n = T > 0 ? (int)((t * N) / T) : 0;
+  n = n < 0 ? 0 : (n > N - 1 ? N - 1 : n);
+  const int64_t a = __ldg(cu + n), b = __ldg(cu + n + 1);
+  if (a <= t && (t < b || n == N - 1)) return n;
+  return seq_of(cu, N, t);
+}
+
 }  // namespace gdn
