@@ -14,23 +14,24 @@
 //
 // One cooperative launch, one CTA per SM, two roles:
 //  * state CTAs (about a third of the SMs) each own a list of (sequence,
-//    value head) items and run their chunks in order. Per chunk two wide
-//    tcgen05 MMAs form the critical path: D1 = S0 [-W ; Q]^T (N = 128: the
-//    S0 part of Delta and S0 Q^T together), then D2 = Delta^T [K~ | M^T]
-//    (N = 256: the state update P = Delta^T diag(e^{G_L-G}) K and the M Delta
-//    output term together); the fp32 state stays in registers (four threads
-//    per row). Few wide MMAs matter because each tcgen05.mma instruction
-//    costs about the same time whether N is 64 or 128.
-//  * prep CTAs claim (item, chunk) work in chunk order from a global counter
-//    and compute the state-free part: bf16 TMA tiles of K, Q, V; the Gram
-//    [K;Q][K;Q]^T on the tensor cores (bf16, exact products: K K^T for A and
-//    K Q^T for M^T); decays; the UT solve in fp32; W and U as bf16 hi/lo MMAs
-//    (~17 significant bits, unit diagonal included); binary16 images of
-//    [-W ; Q], [K~ | M^T hi | M^T lo] and U^T in fp32. They
-//    publish one chunk per ring slot in the caller's workspace (3 slots per
-//    state CTA, ~97 KB each, L2-resident) with a release flag; the state CTA
-//    acquires it, bulk-copies the operand images into shared memory and
-//    releases the slot once read.
+//    value head) items and run their chunks in order. Per chunk: D1 = S0
+//    [-W ; Q~]^T (N = 128: the S0 part of Delta and S0 q~ per token together,
+//    Q~ = diag(e^G) Q), the Delta readout, then P = Delta_hi^T K~ (the state
+//    update, K~ = diag(e^{G_L-G}) K) and the M Delta products, which accumulate
+//    onto S0 q~ in TMEM; the fp32 state stays in registers (four threads per
+//    row). Few wide MMAs matter because each tcgen05.mma instruction costs
+//    about the same time whether N is 64 or 128. A chunk's outputs are read
+//    during the next chunk and leave as one TMA tensor store.
+//  * prep CTAs run two independent 256-thread pipelines each; a pipeline claims
+//    (item, chunk) work in chunk order from a global counter and computes the
+//    state-free part: bf16 TMA tiles of K, Q, V; the Gram [K;Q] K^T on the
+//    tensor cores (bf16, exact products: K K^T for A, Q K^T for M); decays; the
+//    UT solve in fp32; W and U as bf16 hi/lo MMAs (~17 significant bits, unit
+//    diagonal included); it writes binary16 images of [-W ; Q~] and
+//    [K~ | M hi | M lo] and U in fp32 straight into a ring slot in the caller's
+//    workspace (6 slots per state CTA, ~97 KB each, L2-resident) and releases
+//    its flag; the state CTA acquires it, bulk-copies the operand images into
+//    shared memory and releases the slot once read.
 // Deadlock freedom: all CTAs are co-resident (cooperative launch); a prep CTA
 // works on claims in increasing order and a claim only waits on the
 // consumption of an earlier step of the same state CTA. Every wait is
@@ -58,16 +59,17 @@ constexpr uint64_t kLimitNs = 2000000000ull;
 // B operand of S0 [-W ; Q~]^T: K-major, [2 d_k blocks][128 rows][64], rows 0-63 = -W
 // (token t), rows 64-127 = Q~ = diag(e^G) Q (token t), binary16.
 constexpr uint32_t SL_WQ = 0;
-// B operands of Delta^T K~ and Delta^T M^T, four 8 KB blocks: K~ = diag(e^{G_L-G}) K,
-// MN-major [64 tokens s][64 d_k] (d_k 0-63, 64-127), then the lower triangle of M
-// (M[t][s] = M_ts for s <= t) as binary16 high and low parts, K-major [64 t][64 s].
+// Four 8 KB blocks: K~ = diag(e^{G_L-G}) K, MN-major [64 tokens s][64 d_k] (d_k 0-63,
+// 64-127; the B operand of P = Delta^T K~), then the lower triangle of M
+// (M[t][s] = M_ts for s <= t) as binary16 high and low parts, K-major [64 t][64 s]
+// (the B operands of the M Delta products).
 constexpr uint32_t SL_BKM = 32768;
 constexpr uint32_t SL_VEC = 65536;     // gL (the chunk's total decay)
 constexpr uint32_t SL_IMG = 66560;     // bytes of the shared-memory image above
-constexpr uint32_t SL_UT = 66560;      // U^T fp32 [64 t][128 i] (the consumer reads it from L2)
+constexpr uint32_t SL_UT = 66560;      // U fp32 [64 t][128 i] (copied to shared memory separately)
 constexpr uint32_t SLOT_BYTES = 99328;
-// state CTA use of a slot image buffer once its MMAs are done: the [-W ; Q] area
-// stages that step's fp32 outputs, the K~/M area receives the next step's U^T
+// state CTA use of a slot image buffer once its MMAs are done: the [-W ; Q~] area
+// stages that step's outputs (o's dtype), the K~/M area receives the next step's U
 constexpr uint32_t S_STG_OFF = SL_WQ, S_UT_OFF = SL_BKM;
 
 constexpr uint32_t CTRL_BYTES = 16384; // counter, abort word, per-state-CTA flags
@@ -89,7 +91,7 @@ constexpr uint32_t P_SMALL = 2 * PIPE_BYTES;
 // ---- state CTA shared memory --------------------------------------------
 constexpr uint32_t S_BUF = 0;          // 2 x slot image
 constexpr uint32_t S_S0 = 133120;      // binary16 state, K-major [2 blocks][128 rows]
-constexpr uint32_t S_DTH = 165888;     // Delta^T high, K-major A [128][64 t]
+constexpr uint32_t S_DTH = 165888;     // Delta^T high, K-major A [128 d_v][64 t]
 constexpr uint32_t S_DTL = 182272;     // Delta^T low
 constexpr uint32_t S_SMALL = 215040;
 constexpr uint32_t PC_SMEM_BYTES = S_SMALL + 1024;   // the state role needs the most
@@ -100,9 +102,10 @@ constexpr uint32_t PC_SMEM_ALLOC = PC_SMEM_BYTES + 1024;
 // [hi part | lo part] column halves at 0 and U^T the same way at 128
 constexpr uint32_t PT_GR = 0, PT_W = 0, PT_U = 128, PT_PIPE = 256, PT_COLS = 512;
 // state: D1 = S0 [-W ; Q~]^T -> [Delta^T - U^T | OA = S0 Q~^T], in one of two column
-//        sets by step parity (a step's OA outlives the next step's D1), and
+//        sets by step parity (a step's outputs outlive the next step's D1), and
 //        Delta_lo^T M_hi^T accumulated onto OA;  P = Delta_hi^T K~;
-//        OB = Delta_hi^T [M hi ; M lo]^T -> [OB_hh | OB_hl].  o^T = scale (OA + OB_hh + OB_hl)
+//        OB = Delta_hi^T [M hi ; M lo]^T -> [OB_hh | OB_hl] (M with its diagonal).
+//        o^T = scale (OA + OB_hh + OB_hl)
 constexpr uint32_t ST_D1A = 0, ST_P = 128, ST_D1B = 256, ST_OB = 384, ST_COLS = 512;
 
 struct PcParams {
