@@ -53,6 +53,15 @@ template <class Tx> struct RawV {
       }
     }
   }
+  __device__ __forceinline__ void store(Tx* p) const {
+    if constexpr (kBytes == 8) {
+      *reinterpret_cast<uint2*>(p) = make_uint2(u[0], u[1]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < kBytes / 16; ++i)
+        reinterpret_cast<uint4*>(p)[i] = make_uint4(u[4 * i], u[4 * i + 1], u[4 * i + 2], u[4 * i + 3]);
+    }
+  }
   __device__ __forceinline__ void to_f32(float (&f)[kV]) const {
     if constexpr (sizeof(Tx) == 2) {
 #pragma unroll
@@ -148,7 +157,7 @@ __global__ void __launch_bounds__(kConvThreads)
 conv_silu_kernel(const Tx* __restrict__ x, int64_t xs, const Tw* __restrict__ w,
                  const Tw* __restrict__ bias, int C, int l2c, float eps,
                  const int32_t* __restrict__ cu, int N, int64_t T,
-                 const Tx* __restrict__ cs_in, Ty* __restrict__ y, int64_t ys) {
+                 const Tx* __restrict__ cs_in, Tx* cs_out, Ty* __restrict__ y, int64_t ys) {
   const int c = (blockIdx.x * kConvThreads + threadIdx.x) * kV;
   const bool active = c < C;
   const bool any_l2 = (int)blockIdx.x * kConvThreads * kV < l2c;
@@ -196,6 +205,8 @@ conv_silu_kernel(const Tx* __restrict__ x, int64_t xs, const Tw* __restrict__ w,
 #pragma unroll 1
   for (int i0 = 0; i0 < R; i0 += RB) {
     RawV<Tx> src[RB][4];
+    int nn[RB];
+    int64_t s_lo[RB], s_hi[RB];
 #pragma unroll
     for (int i = 0; i < RB; ++i) {
       const int64_t t = t0 + i0 + i;
@@ -206,6 +217,9 @@ conv_silu_kernel(const Tx* __restrict__ x, int64_t xs, const Tw* __restrict__ w,
       }
       // a token past the last sequence is treated as the start of one
       const int64_t st = t >= s_end ? t : s_start;
+      nn[i] = n;
+      s_lo[i] = s_start;
+      s_hi[i] = s_end;
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const int64_t pr = t - 3 + k;
@@ -225,6 +239,14 @@ conv_silu_kernel(const Tx* __restrict__ x, int64_t xs, const Tw* __restrict__ w,
       src[i][2].to_f32(f2);
       src[i][3].to_f32(f3);
       conv_token<Ty>(f0, f1, f2, f3, wt, b, c, l2c, any_l2, eps, active && t < T, y + t * ys + c);
+      // a sequence that lies whole in this batch (this thread alone read its cache
+      // rows) gets its new cache here: its last three pre-conv rows, oldest first
+      if constexpr (R == 2) {   // only the short-sequence tiles are given cs_out
+        if (cs_out && active && t < T && t == s_hi[i] - 1 && s_lo[i] >= t0 + i0) {
+#pragma unroll
+          for (int r = 0; r < 3; ++r) src[i][r + 1].store(cs_out + ((int64_t)nn[i] * 3 + r) * C + c);
+        }
+      }
     }
   }
 }
@@ -233,10 +255,12 @@ conv_silu_kernel(const Tx* __restrict__ x, int64_t xs, const Tw* __restrict__ w,
 // from conv_state_in when the sequence is shorter than 3. One thread per
 // (sequence, 16-byte column chunk) reads its three rows before writing any,
 // so conv_state_out may alias conv_state_in.
+// Sequences that lie whole in one fused_rb-token batch of the conv kernel had
+// their cache written there (fused_rb = 0: none did).
 __global__ void conv_state_kernel(const char* __restrict__ x, int64_t xs_bytes,
                                   int row_bytes, const int32_t* __restrict__ cu,
                                   int N, int64_t T, const char* cs_in,
-                                  char* cs_out) {
+                                  char* cs_out, int fused_rb) {
   const int chunks = row_bytes / 16;
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= (int64_t)N * chunks) return;
@@ -245,6 +269,7 @@ __global__ void conv_state_kernel(const char* __restrict__ x, int64_t xs_bytes,
   const int64_t s = clamp_t(__ldg(cu + n), T);
   int64_t e = clamp_t(__ldg(cu + n + 1), T);
   if (e < s) e = s;
+  if (fused_rb > 0 && e > s && s / fused_rb == (e - 1) / fused_rb) return;
   const int64_t len = e - s;
   uint4 v[3];
 #pragma unroll
@@ -266,6 +291,7 @@ __global__ void conv_state_kernel(const char* __restrict__ x, int64_t xs_bytes,
 
 template <class Tx, class Tw, class Ty>
 cudaError_t launch_typed(const ConvArgs& a) {
+  int fused_rb = 0;
   if (a.T_total > 0) {
     const bool short_seqs = (int64_t)a.N * kShortLen >= a.T_total;
     const int R = short_seqs ? 2 : conv_tile<Tx>();
@@ -273,11 +299,14 @@ cudaError_t launch_typed(const ConvArgs& a) {
               (unsigned)((a.T_total + R - 1) / R));
     auto kern = short_seqs ? conv_silu_kernel<Tx, Tw, Ty, 2, 2>
                            : conv_silu_kernel<Tx, Tw, Ty, conv_tile<Tx>(), conv_batch<Tx>()>;
+    // the short-sequence tiles write the new cache of the sequences they hold whole
+    fused_rb = short_seqs && a.conv_state_out ? 2 : 0;
     kern<<<grid, kConvThreads, 0, a.stream>>>(
         static_cast<const Tx*>(a.x), a.x_row_stride,
         static_cast<const Tw*>(a.w), static_cast<const Tw*>(a.bias), a.channels,
         a.l2norm_channels, a.l2_eps, a.cu_seqlens, a.N, a.T_total,
-        static_cast<const Tx*>(a.conv_state_in), static_cast<Ty*>(a.y),
+        static_cast<const Tx*>(a.conv_state_in),
+        fused_rb ? static_cast<Tx*>(a.conv_state_out) : nullptr, static_cast<Ty*>(a.y),
         a.y_row_stride);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -291,7 +320,7 @@ cudaError_t launch_typed(const ConvArgs& a) {
           static_cast<const char*>(a.x), a.x_row_stride * eb, row_bytes,
           a.cu_seqlens, a.N, a.T_total,
           static_cast<const char*>(a.conv_state_in),
-          static_cast<char*>(a.conv_state_out));
+          static_cast<char*>(a.conv_state_out), fused_rb);
       return cudaGetLastError();
     }
   }

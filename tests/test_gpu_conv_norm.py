@@ -69,6 +69,22 @@ def test_conv_decode_in_place_roll():
     conv_case([1] * 64, in_place=True)
 
 
+def test_conv_short_sequences_cache_out():
+    """Sequences of 0-3 tokens take the decode-shaped tiling: the conv kernel
+    writes the caches of sequences held whole by one 2-token batch, the roll
+    kernel the others (here some 2-token sequences straddle two batches)."""
+    conv_case([1, 2, 1, 0, 2, 3, 1, 1, 2, 1], hist=True)
+
+
+def test_conv_short_sequences_in_place():
+    conv_case([1, 2, 1, 2, 2, 1, 1, 3, 0, 1], in_place=True)
+
+
+def test_conv_short_sequences_fp32_no_history():
+    conv_case([2, 1, 1, 3, 0, 1, 2], x_dtype=torch.float32, y_dtype=torch.float32,
+              hist=False)
+
+
 def test_conv_zero_tokens_only_copies_state():
     C = 256
     h = torch.randn(3, 3, C, dtype=torch.bfloat16, device=DEV)
