@@ -204,6 +204,33 @@ class DecodeWorkload:
         g.gdn_gated_rmsnorm(self.o, st["z"], self.nw, eps=1e-6, y=self.out)
 
 
+class RankGroup:
+    """Barrier and max-over-ranks around the timed regions; no-ops at one rank.
+    `dist` is torch.distributed with an initialised process group (NCCL on the
+    GPUs; gloo works the same on CPU tensors) and `device` where its reductions
+    run."""
+
+    def __init__(self, dist=None, device=None):
+        self.dist, self.device = dist, device
+
+    def barrier(self):
+        if self.dist is not None:
+            self.dist.barrier()
+
+    def max(self, v):
+        if self.dist is None:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=self.device)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+
+def throughput(units_per_rank, world, max_ms):
+    """Whole-job units per second: the units every rank processed over the
+    slowest rank's time."""
+    return units_per_rank * world / (max_ms * 1e-3)
+
+
 def timed_loop(step_fn, steps, warmup, dist_barrier):
     """Warm up, then time exactly `steps` back-to-back steps. Each step's
     region and its dominant kernel are bracketed by CUDA events on the
@@ -301,17 +328,8 @@ def gpu_arm(args):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
-
-    def barrier():
-        if dist is not None:
-            dist.barrier()
-
-    def max_over_ranks(v):
-        if dist is None:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    group = RankGroup(dist, dev)
+    barrier, max_over_ranks = group.barrier, group.max
 
     import gated_delta_rule_106_b200 as gdn
     gdn.load()
@@ -333,7 +351,6 @@ def gpu_arm(args):
     d_ms = max_over_ranks(statistics.mean(d_step_ms))
     d_kms = max_over_ranks(statistics.mean(d_kern_ms))
 
-    tokens = T_PREFILL * world
     flops = PREFILL_FLOP_PER_TOKEN * T_PREFILL
     pre_ach = flops / (kms * 1e-3) / 1e12
     dec_bytes = DECODE_BYTES_PER_TOKEN * N_DECODE
@@ -342,7 +359,7 @@ def gpu_arm(args):
     dtr = kernel_traffic("decode")
     line = {
         "metric": METRIC,
-        "value": tokens / (ms * 1e-3),
+        "value": throughput(T_PREFILL, world, ms),
         "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms,
@@ -369,7 +386,7 @@ def gpu_arm(args):
             "algorithmic_flop_per_launch": flops,
             "kernel_ms": kms,
         },
-        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
+        "e2e": {"value": throughput(T_PREFILL, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms},
         "gpu_launches": pre.launches_per_step * args.steps,
@@ -377,7 +394,7 @@ def gpu_arm(args):
         "decode": {
             "workload": "decode: 256 sequences x 128 steps, 1 token each, fp32 state "
                         "[256,48,128,128]; conv (cache roll) -> decode step -> gated RMSNorm",
-            "value": N_DECODE * world / (d_ms * 1e-3), "unit": "tokens/s",
+            "value": throughput(N_DECODE, world, d_ms), "unit": "tokens/s",
             "ms_per_step": d_ms,
             "roofline": {"kernel": "gdn_decode_step", "bound": "hbm",
                          "achieved": dec_ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",

@@ -1,0 +1,90 @@
+"""Host-side logic of bench.py on CPU: the reference arm's JSON line, the
+two-rank launch (only rank 0 prints), and the barrier / max-over-ranks /
+whole-job throughput used around the timed regions, on two gloo ranks."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+def free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def json_lines(out):
+    return [json.loads(l) for l in out.splitlines() if l.startswith("{")]
+
+
+def test_throughput_counts_every_rank_over_the_slowest():
+    assert bench.throughput(8192, 1, 1.0) == pytest.approx(8192e3)
+    assert bench.throughput(8192, 4, 2.0) == pytest.approx(4 * 8192 / 2e-3)
+
+
+def test_single_rank_group_is_a_no_op():
+    g = bench.RankGroup()
+    g.barrier()
+    assert g.max(3.25) == 3.25
+
+
+def _ranks(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        g = bench.RankGroup(dist, torch.device("cpu"))
+        g.barrier()
+        out[rank] = g.max(1.5 + rank)
+        g.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_agree_on_the_slowest_time():
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_ranks, args=(2, free_port(), out), nprocs=2, join=True,
+                       start_method="spawn")
+    assert dict(out) == {0: 2.5, 1: 2.5}
+
+
+def test_reference_arm_json_line():
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--steps", "1", "--warmup", "3"],
+                       capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = json_lines(r.stdout)
+    assert len(lines) == 1
+    d = lines[0]
+    assert d["impl"] == "reference" and d["unit"] == "tokens/s" and d["higher_is_better"]
+    assert d["metric"] == bench.METRIC and d["value"] > 0 and d["steps"] == 1
+    assert d["warmup"] >= 3 and d["n_gpus"] == 1
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+    assert d["config"]["seq_len"] == bench.T_PREFILL and "workload" in d["config"]
+
+
+def test_reference_arm_under_two_ranks_prints_once():
+    r = subprocess.run([sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+                        "--nproc-per-node", "2", "--master-addr", "127.0.0.1",
+                        "--master-port", str(free_port()),
+                        os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+                        "--steps", "1", "--warmup", "3"],
+                       capture_output=True, text=True, timeout=900, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = json_lines(r.stdout)
+    assert len(lines) == 1 and lines[0]["impl"] == "reference"
+    assert lines[0]["n_gpus"] == 2
