@@ -129,6 +129,19 @@ def _row_stride(t):
     return t.stride(0)
 
 
+def _expect(t, shape, name, dtype=None, contiguous=True):
+    """Shape (and dtype, contiguity) the C ABI assumes for a tensor argument;
+    checked before any pointer is taken, since the kernels write dense layouts."""
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if contiguous and not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
 def _stream(stream, device):
     if stream is None:
         stream = torch.cuda.current_stream(device)
@@ -148,6 +161,11 @@ def gdn_conv1d_silu(x, w, cu_seqlens, *, bias=None, conv_state_in=None,
     conv states [N, 3, C] (x's dtype). Returns y [T, C]."""
     T, C = x.shape
     N = cu_seqlens.numel() - 1
+    _expect(w, (C, 4), "w")
+    _expect(bias, (C,), "bias")
+    _expect(conv_state_in, (N, 3, C), "conv_state_in", x.dtype)
+    _expect(conv_state_out, (N, 3, C), "conv_state_out", x.dtype)
+    _expect(y, (T, C), "y", contiguous=False)
     if y is None:
         y = torch.empty((T, C), dtype=y_dtype or x.dtype, device=x.device)
     _check("gdn_conv1d_silu", load().gdn_conv1d_silu(
@@ -156,6 +174,16 @@ def gdn_conv1d_silu(x, w, cu_seqlens, *, bias=None, conv_state_in=None,
         _ptr(cu_seqlens), N, T, _ptr(conv_state_in), _ptr(conv_state_out),
         _ptr(y), _row_stride(y), _dtype_code(y.dtype), _stream(stream, x.device)))
     return y
+
+
+def _check_prefill_shapes(q, k, v, g, beta, state_in, state_out, o, T, H_k, H_v, N):
+    _expect(k, (T, H_k, HEAD_DIM), "k", contiguous=False)
+    _expect(v, (T, H_v, HEAD_DIM), "v", contiguous=False)
+    _expect(g, (T, H_v), "g")
+    _expect(beta, (T, H_v), "beta", g.dtype)
+    _expect(state_in, (N, H_v, HEAD_DIM, HEAD_DIM), "state_in", torch.float32)
+    _expect(state_out, (N, H_v, HEAD_DIM, HEAD_DIM), "state_out", torch.float32)
+    _expect(o, (T, H_v, HEAD_DIM), "o")
 
 
 def gdn_chunked_prefill_workspace(N, T_total, H_k=H_K, H_v=H_V) -> int:
@@ -171,6 +199,7 @@ def gdn_chunked_prefill(q, k, v, g, beta, cu_seqlens, *, state_in=None,
     T, H_k, _ = q.shape
     H_v = v.shape[1]
     N = cu_seqlens.numel() - 1
+    _check_prefill_shapes(q, k, v, g, beta, state_in, state_out, o, T, H_k, H_v, N)
     if o is None:
         o = torch.empty((T, H_v, HEAD_DIM), dtype=o_dtype or v.dtype, device=v.device)
     need = gdn_chunked_prefill_workspace(N, T, H_k, H_v)
@@ -195,6 +224,7 @@ def gdn_chunked_prefill_noalloc(q, k, v, g, beta, cu_seqlens, *, state_in=None,
     T, H_k, _ = q.shape
     H_v = v.shape[1]
     N = cu_seqlens.numel() - 1
+    _check_prefill_shapes(q, k, v, g, beta, state_in, state_out, o, T, H_k, H_v, N)
     if o is None:
         o = torch.empty((T, H_v, HEAD_DIM), dtype=o_dtype or v.dtype, device=v.device)
     _check("gdn_chunked_prefill_noalloc", load().gdn_chunked_prefill_noalloc(
@@ -212,6 +242,12 @@ def gdn_decode_step(q, k, v, g, beta, state, *, scale=1.0, o=None,
     Returns o [N, H_v, 128]."""
     N, H_k, _ = q.shape
     H_v = v.shape[1]
+    _expect(k, (N, H_k, HEAD_DIM), "k", contiguous=False)
+    _expect(v, (N, H_v, HEAD_DIM), "v", contiguous=False)
+    _expect(g, (N, H_v), "g")
+    _expect(beta, (N, H_v), "beta", g.dtype)
+    _expect(state, (N, H_v, HEAD_DIM, HEAD_DIM), "state", torch.float32)
+    _expect(o, (N, H_v, HEAD_DIM), "o")
     if o is None:
         o = torch.empty((N, H_v, HEAD_DIM), dtype=o_dtype or v.dtype, device=v.device)
     _check("gdn_decode_step", load().gdn_decode_step(
@@ -226,6 +262,9 @@ def gdn_gated_rmsnorm(x, z, w, *, eps=1e-6, y=None, y_dtype=None, stream=None):
     """y = x / sqrt(mean(x^2) + eps) * w * SiLU(z) over the last dim (128)."""
     dim = x.shape[-1]
     rows = x.numel() // dim if dim else 0
+    _expect(z, tuple(x.shape), "z")
+    _expect(w, (dim,), "w")
+    _expect(y, tuple(x.shape), "y")
     if y is None:
         y = torch.empty(x.shape, dtype=y_dtype or x.dtype, device=x.device)
     for t in (x, z, y):

@@ -164,3 +164,39 @@ def test_binding_refuses_cpu_tensors(lib):
         gdn.gdn_gated_rmsnorm(torch.zeros(2, 128), torch.zeros(2, 128),
                               torch.ones(128))
     del x
+
+
+def test_binding_checks_shapes_before_pointers(lib):
+    """The kernels write dense layouts, so the binding refuses a tensor of the
+    wrong shape, dtype or layout before any pointer reaches the library (the
+    tensors here are on the CPU: the check must come first to be seen)."""
+    import torch
+    T, N = 8, 1
+    q = torch.zeros(T, 16, 128, dtype=torch.bfloat16)
+    v = torch.zeros(T, 48, 128, dtype=torch.bfloat16)
+    g, b = torch.ones(T, 48), torch.ones(T, 48)
+    cu = torch.tensor([0, T], dtype=torch.int32)
+    pre = lambda **kw: gdn.gdn_chunked_prefill(q, q, v, g, b, cu, **kw)
+    with pytest.raises(ValueError, match="o: shape"):
+        pre(o=torch.empty(T, 47, 128))
+    with pytest.raises(ValueError, match="o must be contiguous"):
+        pre(o=torch.empty(T, 128, 48).transpose(1, 2))
+    with pytest.raises(ValueError, match="state_out: dtype"):
+        pre(state_out=torch.empty(N, 48, 128, 128, dtype=torch.float64))
+    with pytest.raises(ValueError, match="state_in: shape"):
+        pre(state_in=torch.empty(2, 48, 128, 128))
+    with pytest.raises(ValueError, match="beta: dtype"):
+        gdn.gdn_chunked_prefill(q, q, v, g, b.double(), cu)
+    with pytest.raises(ValueError, match="g: shape"):
+        gdn.gdn_chunked_prefill(q, q, v, g[:, :47], b, cu)
+    with pytest.raises(ValueError, match="k: shape"):
+        gdn.gdn_chunked_prefill(q, q[:, :8], v, g, b, cu)
+    with pytest.raises(ValueError, match="state: shape"):
+        gdn.gdn_decode_step(q[:1], q[:1], v[:1], g[:1], b[:1], torch.empty(2, 48, 128, 128))
+    with pytest.raises(ValueError, match="conv_state_out: dtype"):
+        gdn.gdn_conv1d_silu(torch.zeros(T, 256, dtype=torch.bfloat16), torch.ones(256, 4), cu,
+                            conv_state_out=torch.empty(N, 3, 256))
+    with pytest.raises(ValueError, match="w: shape"):
+        gdn.gdn_conv1d_silu(torch.zeros(T, 256, dtype=torch.bfloat16), torch.ones(256, 3), cu)
+    with pytest.raises(ValueError, match="z: shape"):
+        gdn.gdn_gated_rmsnorm(torch.zeros(T, 128), torch.zeros(T, 64), torch.ones(128))
