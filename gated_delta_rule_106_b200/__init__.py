@@ -161,8 +161,9 @@ def gdn_conv1d_silu(x, w, cu_seqlens, *, bias=None, conv_state_in=None,
     conv states [N, 3, C] (x's dtype). Returns y [T, C]."""
     T, C = x.shape
     N = cu_seqlens.numel() - 1
+    _expect(cu_seqlens, (N + 1,), "cu_seqlens", torch.int32)
     _expect(w, (C, 4), "w")
-    _expect(bias, (C,), "bias")
+    _expect(bias, (C,), "bias", w.dtype)
     _expect(conv_state_in, (N, 3, C), "conv_state_in", x.dtype)
     _expect(conv_state_out, (N, 3, C), "conv_state_out", x.dtype)
     _expect(y, (T, C), "y", contiguous=False)
@@ -176,9 +177,13 @@ def gdn_conv1d_silu(x, w, cu_seqlens, *, bias=None, conv_state_in=None,
     return y
 
 
-def _check_prefill_shapes(q, k, v, g, beta, state_in, state_out, o, T, H_k, H_v, N):
-    _expect(k, (T, H_k, HEAD_DIM), "k", contiguous=False)
-    _expect(v, (T, H_v, HEAD_DIM), "v", contiguous=False)
+def _check_prefill_shapes(q, k, v, g, beta, cu_seqlens, state_in, state_out, o, T,
+                          H_k, H_v, N):
+    # one qkv dtype crosses the C ABI (q's): k and v must share it
+    _expect(q, (T, H_k, HEAD_DIM), "q", contiguous=False)
+    _expect(k, (T, H_k, HEAD_DIM), "k", q.dtype, contiguous=False)
+    _expect(v, (T, H_v, HEAD_DIM), "v", q.dtype, contiguous=False)
+    _expect(cu_seqlens, (N + 1,), "cu_seqlens", torch.int32)
     _expect(g, (T, H_v), "g")
     _expect(beta, (T, H_v), "beta", g.dtype)
     _expect(state_in, (N, H_v, HEAD_DIM, HEAD_DIM), "state_in", torch.float32)
@@ -199,7 +204,8 @@ def gdn_chunked_prefill(q, k, v, g, beta, cu_seqlens, *, state_in=None,
     T, H_k, _ = q.shape
     H_v = v.shape[1]
     N = cu_seqlens.numel() - 1
-    _check_prefill_shapes(q, k, v, g, beta, state_in, state_out, o, T, H_k, H_v, N)
+    _check_prefill_shapes(q, k, v, g, beta, cu_seqlens, state_in, state_out, o, T,
+                          H_k, H_v, N)
     if o is None:
         o = torch.empty((T, H_v, HEAD_DIM), dtype=o_dtype or v.dtype, device=v.device)
     need = gdn_chunked_prefill_workspace(N, T, H_k, H_v)
@@ -224,7 +230,8 @@ def gdn_chunked_prefill_noalloc(q, k, v, g, beta, cu_seqlens, *, state_in=None,
     T, H_k, _ = q.shape
     H_v = v.shape[1]
     N = cu_seqlens.numel() - 1
-    _check_prefill_shapes(q, k, v, g, beta, state_in, state_out, o, T, H_k, H_v, N)
+    _check_prefill_shapes(q, k, v, g, beta, cu_seqlens, state_in, state_out, o, T,
+                          H_k, H_v, N)
     if o is None:
         o = torch.empty((T, H_v, HEAD_DIM), dtype=o_dtype or v.dtype, device=v.device)
     _check("gdn_chunked_prefill_noalloc", load().gdn_chunked_prefill_noalloc(
@@ -242,8 +249,9 @@ def gdn_decode_step(q, k, v, g, beta, state, *, scale=1.0, o=None,
     Returns o [N, H_v, 128]."""
     N, H_k, _ = q.shape
     H_v = v.shape[1]
-    _expect(k, (N, H_k, HEAD_DIM), "k", contiguous=False)
-    _expect(v, (N, H_v, HEAD_DIM), "v", contiguous=False)
+    _expect(q, (N, H_k, HEAD_DIM), "q", contiguous=False)
+    _expect(k, (N, H_k, HEAD_DIM), "k", q.dtype, contiguous=False)
+    _expect(v, (N, H_v, HEAD_DIM), "v", q.dtype, contiguous=False)
     _expect(g, (N, H_v), "g")
     _expect(beta, (N, H_v), "beta", g.dtype)
     _expect(state, (N, H_v, HEAD_DIM, HEAD_DIM), "state", torch.float32)

@@ -200,3 +200,38 @@ def test_binding_checks_shapes_before_pointers(lib):
         gdn.gdn_conv1d_silu(torch.zeros(T, 256, dtype=torch.bfloat16), torch.ones(256, 3), cu)
     with pytest.raises(ValueError, match="z: shape"):
         gdn.gdn_gated_rmsnorm(torch.zeros(T, 128), torch.zeros(T, 64), torch.ones(128))
+
+
+def test_binding_refuses_mixed_dtypes(lib):
+    """One qkv dtype crosses the C ABI (q's), and the conv bias is read in w's
+    dtype, cu_seqlens as int32: a k or v of another dtype than q, a bias of
+    another dtype than w, or int64 cu_seqlens would be read past their bytes
+    or misread, so the binding refuses them before any pointer is taken."""
+    import torch
+    T = 8
+    q32 = torch.zeros(T, 16, 128)
+    k16 = torch.zeros(T, 16, 128, dtype=torch.bfloat16)
+    v16 = torch.zeros(T, 48, 128, dtype=torch.bfloat16)
+    v32 = torch.zeros(T, 48, 128)
+    g, b = torch.ones(T, 48), torch.ones(T, 48)
+    cu = torch.tensor([0, T], dtype=torch.int32)
+    with pytest.raises(ValueError, match="k: dtype"):
+        gdn.gdn_chunked_prefill(q32, k16, v32, g, b, cu)
+    with pytest.raises(ValueError, match="v: dtype"):
+        gdn.gdn_chunked_prefill(q32, q32, v16, g, b, cu)
+    with pytest.raises(ValueError, match="k: dtype"):
+        gdn.gdn_chunked_prefill_noalloc(q32, k16, v32, g, b, cu)
+    with pytest.raises(ValueError, match="cu_seqlens: dtype"):
+        gdn.gdn_chunked_prefill(q32, q32, v32, g, b, cu.long())
+    with pytest.raises(ValueError, match="k: dtype"):
+        gdn.gdn_decode_step(q32[:1], k16[:1], v32[:1], g[:1], b[:1],
+                            torch.zeros(1, 48, 128, 128))
+    with pytest.raises(ValueError, match="v: dtype"):
+        gdn.gdn_decode_step(q32[:1], q32[:1], v16[:1], g[:1], b[:1],
+                            torch.zeros(1, 48, 128, 128))
+    x = torch.zeros(T, 256, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="bias: dtype"):
+        gdn.gdn_conv1d_silu(x, torch.ones(256, 4), cu,
+                            bias=torch.zeros(256, dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="cu_seqlens: dtype"):
+        gdn.gdn_conv1d_silu(x, torch.ones(256, 4), cu.long())
