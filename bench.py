@@ -5,18 +5,32 @@ One step = one pass of the layer's prefill hot path over one synthetic batch:
 causal conv k=4 + SiLU + q/k L2 (gdn_conv1d_silu) -> chunk-64 gated delta
 rule (gdn_chunked_prefill) -> gated RMS-norm (gdn_gated_rmsnorm), on the
 prefill workload B=1, T=8192, 16 key / 48 value heads, head dim 128, bf16
-activations, fp32 gates and state. The decode workload (256 sequences, one
-token per step: conv with in-place cache roll -> gdn_decode_step -> gated
-RMS-norm, fp32 state [256,48,128,128]) is timed in the same run and reported
-under "decode".
+activations, fp32 gates and state. That step gives the headline "value".
+The same run times, under their own keys:
+
+  prefill_l2_flushed  the same step with a 256 MB L2 flush between steps;
+  varlen              16 packed sequences of 512..16384 tokens (seeded), fp32
+                      initial states in and final states out, same chain;
+  decode              256 sequences, one token per step for 128 steps: conv
+                      with in-place cache roll -> gdn_decode_step -> gated
+                      RMS-norm, fp32 state [256,48,128,128];
+  long_context        T=262144 as 64 calls of 4096 tokens with the recurrent
+                      state and the conv history carried between calls (one
+                      step = all 64 calls), unflushed and L2-flushed.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                    [--shard replicas|heads]
+    python bench.py --profile-case NAME [--n N] [--t T] [--launches L]
 
-With N > 1 (launched by torch.distributed.run) every rank runs its own
-replica of the workload on its own synthetic data -- the layer shards by
-sequence with no exchange -- and the slowest rank's time is reported
-("scaling": "weak"). `--impl reference` times the fp64 CPU oracle on the
-host cores on a bounded sample of the same workload (rank 0 only).
+With N > 1 (launched by torch.distributed.run) each rank either runs its own
+replica of every workload on its own synthetic data ("replicas", the default:
+sequences are independent, weak scaling) or takes 16/N key heads and their
+3x value heads of the same workloads ("heads": the head split of a
+tensor-parallel layer, strong scaling). Neither needs a data-path collective;
+the slowest rank's device time is reported. `--impl reference` times the fp64
+CPU oracle on the host cores on a bounded sample of the prefill workload
+(rank 0 only). `--profile-case` runs a few fixed launches of one kernel for a
+profiler capture and exits.
 """
 from __future__ import annotations
 
@@ -40,11 +54,16 @@ import gdn_inputs as gi  # noqa: E402
 METRIC = "gated-delta-rule prefill tokens/s and decode tokens/s per layer; % of roofline"
 T_PREFILL = 8192
 N_DECODE = 256
+DECODE_STEPS = 128
+SEG, N_SEG = 4096, 64
+N_VARLEN = 16
 H_K, H_V, D, C = 16, 48, 128, 64
-# Algorithmic work per token, one layer, chunk C=64: 6d^2 (W S^T, Q S^T, U^T K)
+L2_FLUSH_BYTES = 256 << 20
+# Algorithmic work per token and value head, chunk C=64: 6d^2 (W S^T, Q S^T, U^T K)
 # + 6Cd (W, U, M U) + 4Cd/3 (K K^T, Q K^T shared by 3 value heads) + C^2/1.5
-# (triangular solve), for each of the 48 value heads.
-PREFILL_FLOP_PER_TOKEN = 48 * (6 * D * D + 6 * C * D + 4 * C * D / 3 + C * C / 1.5)
+# (triangular solve).
+FLOP_PER_TOKEN_HEAD = 6 * D * D + 6 * C * D + 4 * C * D / 3 + C * C / 1.5
+PREFILL_FLOP_PER_TOKEN = H_V * FLOP_PER_TOKEN_HEAD
 # bf16 q,k,v,o + fp32 g,beta per token
 PREFILL_BYTES_PER_TOKEN = 2 * (2 * H_K * D) + 2 * H_V * D + 2 * 4 * H_V + 2 * H_V * D
 # decode: fp32 state read + write, plus q,k (bf16), v, o (bf16), g, beta (bf16)
@@ -79,8 +98,8 @@ def kernel_traffic(kernel):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples taken while the timed loop
-    runs (50 ms period)."""
+    """nvidia-smi clock / throttle-reason samples (50 ms period) taken while
+    the timed legs run."""
 
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -89,6 +108,7 @@ class ClockSampler:
     def __init__(self, index):
         self.index = index
         self.proc = None
+        self.out = ""
 
     def __enter__(self):
         try:
@@ -101,7 +121,6 @@ class ClockSampler:
         return self
 
     def __exit__(self, *exc):
-        self.out = ""
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -127,81 +146,213 @@ class ClockSampler:
                           if v.lower() == "active"})
         return {"sm_mhz": statistics.median(r[0] for r in rows),
                 "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
-                "samples": len(rows)}
+                "samples": len(rows), "span": "every timed leg of this run"}
+
+
+def head_shard(rank, world, H_k=H_K, H_v=H_V):
+    """Key heads [kh0, kh1) and value heads [vh0, vh1) of one rank when the
+    layer's heads are split over `world` ranks (a tensor-parallel layer):
+    whole key-head groups, so local value head j reads local key head
+    j // (H_v / H_k) exactly as global value head vh0 + j reads global key
+    head (vh0 + j) // (H_v / H_k)."""
+    if H_k % world:
+        raise ValueError(f"{H_k} key heads do not split over {world} ranks")
+    per = H_k // world
+    grp = H_v // H_k
+    kh0 = rank * per
+    return kh0, kh0 + per, kh0 * grp, (kh0 + per) * grp
+
+
+def shard_channels(kh0, kh1, vh0, vh1, H_k=H_K):
+    """Indices of the conv channels (q | k | v of the full layer) that a head
+    shard owns, in the order q | k | v."""
+    q = np.arange(kh0 * D, kh1 * D)
+    k = H_k * D + np.arange(kh0 * D, kh1 * D)
+    v = 2 * H_k * D + np.arange(vh0 * D, vh1 * D)
+    return np.concatenate([q, k, v])
 
 
 # ---------------------------------------------------------------- GPU arm --
 
+def device_gates(gen, T, H_v, dev, dtype=torch.float32):
+    """beta = sigmoid(N(0,1)), g = exp(-softplus(N(0,1))) drawn on the device."""
+    nb = torch.randn((T, H_v), generator=gen, device=dev)
+    ng = torch.randn((T, H_v), generator=gen, device=dev)
+    return torch.exp(-torch.nn.functional.softplus(ng)).to(dtype), torch.sigmoid(nb).to(dtype)
+
+
+class Layer:
+    """One delta-rule layer (or a head shard of it): conv weights, the norm
+    weight, and the chain conv -> chunked prefill -> gated RMS-norm on
+    caller-given buffers. H_k / H_v are this rank's heads."""
+
+    def __init__(self, gdn, dev, conv_w, H_k, H_v):
+        self.gdn, self.dev = gdn, dev
+        self.H_k, self.H_v = H_k, H_v
+        self.qc, self.kc = H_k * D, 2 * H_k * D          # channel offsets of k and v
+        self.w = conv_w.to(dev)
+        self.nw = torch.ones(D, device=dev)
+
+    def views(self, y):
+        T = y.shape[0]
+        return (y[:, :self.qc].view(T, self.H_k, D), y[:, self.qc:self.kc].view(T, self.H_k, D),
+                y[:, self.kc:].view(T, self.H_v, D))
+
+    def chain(self, x, cu, gate, beta, z, y, o, out, ws, state_in=None, state_out=None,
+              conv_state=None, ev=None):
+        g = self.gdn
+        g.gdn_conv1d_silu(x, self.w, cu, conv_state_in=conv_state, conv_state_out=conv_state,
+                          l2norm_channels=self.kc, y=y)
+        if ev is not None:
+            ev[0].record()
+        q, k, v = self.views(y)
+        g.gdn_chunked_prefill(q, k, v, gate, beta, cu, state_in=state_in, state_out=state_out,
+                              o=o, workspace=ws)
+        if ev is not None:
+            ev[1].record()
+        g.gdn_gated_rmsnorm(o, z, self.nw, eps=1e-6, y=out)
+
+
 class PrefillWorkload:
-    """Device-resident buffers of the prefill workload and one step over it."""
+    """The T=8192 prefill workload, device-resident (host copies kept for the
+    end-to-end leg and the CPU oracle)."""
 
-    def __init__(self, gdn, dev, seed):
-        self.gdn = gdn
+    def __init__(self, gdn, dev, seed, shard):
+        kh0, kh1, vh0, vh1 = shard
         p = gi.prefill_inputs(T=T_PREFILL, seed=seed)
-        self.host = p
-        self.x = p["x_pre"].to(dev)
-        self.w = p["conv_w"].to(dev)
-        self.g = p["g"].to(dev)
-        self.b = p["beta"].to(dev)
-        self.z = p["z"].to(dev)
-        self.nw = p["norm_w"].to(dev)
+        ch = torch.from_numpy(shard_channels(kh0, kh1, vh0, vh1))
+        self.full = (kh1 - kh0) == H_K
+        self.host = {"x_pre": p["x_pre"] if self.full else p["x_pre"][:, ch].contiguous(),
+                     "g": p["g"][:, vh0:vh1].contiguous(), "beta": p["beta"][:, vh0:vh1].contiguous(),
+                     "z": p["z"][:, vh0:vh1].contiguous()}
+        self.layer = Layer(gdn, dev, p["conv_w"][ch], kh1 - kh0, vh1 - vh0)
+        self.x = self.host["x_pre"].to(dev)
+        self.g, self.b = self.host["g"].to(dev), self.host["beta"].to(dev)
+        self.z = self.host["z"].to(dev)
         self.cu = p["cu_seqlens"].to(dev)
+        Hv = vh1 - vh0
         self.y = torch.empty_like(self.x)
-        self.o = torch.empty((T_PREFILL, H_V, D), dtype=torch.bfloat16, device=dev)
+        self.o = torch.empty((T_PREFILL, Hv, D), dtype=torch.bfloat16, device=dev)
         self.out = torch.empty_like(self.o)
-        self.state = torch.empty((1, H_V, D, D), dtype=torch.float32, device=dev)
+        self.state = torch.empty((1, Hv, D, D), dtype=torch.float32, device=dev)
+        self.ws = torch.empty(max(1, gdn.gdn_chunked_prefill_workspace(1, T_PREFILL, kh1 - kh0, Hv)),
+                              dtype=torch.uint8, device=dev)
         self.launches_per_step = 3
+        self.tokens = T_PREFILL
+        self.flop = T_PREFILL * Hv * FLOP_PER_TOKEN_HEAD
 
-    def step(self, ev=None):
+    def step(self, i, ev=None):
         self.chain(self.x, self.g, self.b, self.z, self.out, ev)
 
     def chain(self, x, gate, beta, z, out, ev=None):
-        """conv -> chunked prefill -> gated RMSNorm on the given input and
-        output buffers (the intermediates are this workload's own)."""
-        g = self.gdn
-        g.gdn_conv1d_silu(x, self.w, self.cu, y=self.y)
-        if ev is not None:
-            ev[0].record()
-        y = self.y
-        g.gdn_chunked_prefill(y[:, :2048].view(-1, H_K, D), y[:, 2048:4096].view(-1, H_K, D),
-                              y[:, 4096:].view(-1, H_V, D), gate, beta, self.cu,
-                              state_out=self.state, o=self.o)
-        if ev is not None:
-            ev[1].record()
-        g.gdn_gated_rmsnorm(self.o, z, self.nw, eps=1e-6, y=out)
+        self.layer.chain(x, self.cu, gate, beta, z, self.y, self.o, out, self.ws,
+                         state_out=self.state, ev=ev)
+
+
+class VarlenWorkload:
+    """16 packed sequences, lengths uniform in [512, 16384] (seeded), fp32
+    initial states ~N(0, 0.02) in, final states out; inputs drawn on the
+    device with the prefill workload's distributions."""
+
+    def __init__(self, gdn, dev, seed, shard):
+        kh0, kh1, vh0, vh1 = shard
+        Hk, Hv = kh1 - kh0, vh1 - vh0
+        cu = gi.varlen_cu_seqlens(N_VARLEN, 512, 16384, seed=seed)
+        T = int(cu[-1])
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(1000 + seed)
+        ch = torch.from_numpy(shard_channels(kh0, kh1, vh0, vh1))
+        self.layer = Layer(gdn, dev, gi.conv_weight(seed)[ch], Hk, Hv)
+        self.cu = cu.to(dev)
+        self.x = torch.randn((T, len(ch)), generator=gen, device=dev).to(torch.bfloat16)
+        self.g, self.b = device_gates(gen, T, Hv, dev)
+        self.z = torch.randn((T, Hv, D), generator=gen, device=dev).to(torch.bfloat16)
+        self.s_in = torch.randn((N_VARLEN, Hv, D, D), generator=gen, device=dev) * gi.STATE_VAR ** 0.5
+        self.s_out = torch.empty_like(self.s_in)
+        self.y = torch.empty_like(self.x)
+        self.o = torch.empty((T, Hv, D), dtype=torch.bfloat16, device=dev)
+        self.out = torch.empty_like(self.o)
+        self.ws = torch.empty(max(1, gdn.gdn_chunked_prefill_workspace(N_VARLEN, T, Hk, Hv)),
+                              dtype=torch.uint8, device=dev)
+        self.tokens = T
+        self.flop = T * Hv * FLOP_PER_TOKEN_HEAD
+        self.launches_per_step = 3
+
+    def step(self, i, ev=None):
+        self.layer.chain(self.x, self.cu, self.g, self.b, self.z, self.y, self.o, self.out,
+                         self.ws, state_in=self.s_in, state_out=self.s_out, ev=ev)
+
+
+class LongContextWorkload:
+    """T=262144 as 64 calls of 4096 tokens; the recurrent state and the conv
+    history are carried from call to call. One step = all 64 calls."""
+
+    def __init__(self, gdn, dev, seed, shard):
+        kh0, kh1, vh0, vh1 = shard
+        Hk, Hv = kh1 - kh0, vh1 - vh0
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(2000 + seed)
+        ch = torch.from_numpy(shard_channels(kh0, kh1, vh0, vh1))
+        nch = len(ch)
+        self.layer = Layer(gdn, dev, gi.conv_weight(seed)[ch], Hk, Hv)
+        T = SEG * N_SEG
+        self.x = torch.randn((T, nch), generator=gen, device=dev).to(torch.bfloat16)
+        self.g, self.b = device_gates(gen, T, Hv, dev)
+        self.z = torch.randn((T, Hv, D), generator=gen, device=dev).to(torch.bfloat16)
+        self.cu = torch.tensor([0, SEG], dtype=torch.int32, device=dev)
+        self.state = torch.zeros((1, Hv, D, D), device=dev)
+        self.cache = torch.zeros((1, 3, nch), dtype=torch.bfloat16, device=dev)
+        self.y = torch.empty((SEG, nch), dtype=torch.bfloat16, device=dev)
+        self.o = torch.empty((SEG, Hv, D), dtype=torch.bfloat16, device=dev)
+        self.out = torch.empty((T, Hv, D), dtype=torch.bfloat16, device=dev)
+        self.ws = torch.empty(max(1, gdn.gdn_chunked_prefill_workspace(1, SEG, Hk, Hv)),
+                              dtype=torch.uint8, device=dev)
+        self.tokens = T
+        self.flop = T * Hv * FLOP_PER_TOKEN_HEAD
+        self.launches_per_step = N_SEG * 4     # conv, cache roll, prefill, norm
+
+    def segment(self, s, ev=None):
+        a, e = s * SEG, (s + 1) * SEG
+        self.layer.chain(self.x[a:e], self.cu, self.g[a:e], self.b[a:e], self.z[a:e], self.y,
+                         self.o, self.out[a:e], self.ws, state_in=self.state,
+                         state_out=self.state, conv_state=self.cache, ev=ev)
 
 
 class DecodeWorkload:
-    def __init__(self, gdn, dev, seed, steps):
+    def __init__(self, gdn, dev, seed, steps, shard):
+        kh0, kh1, vh0, vh1 = shard
+        Hk, Hv = kh1 - kh0, vh1 - vh0
+        ch = torch.from_numpy(shard_channels(kh0, kh1, vh0, vh1))
         self.gdn = gdn
         init = gi.decode_initial(N_DECODE, seed)
-        self.state = init["state"].to(dev)
-        self.cache = init["conv_state"].to(dev)
-        self.w = gi.conv_weight(seed).to(dev)
-        self.nw = torch.ones(D, device=dev)
+        self.state = init["state"][:, vh0:vh1].contiguous().to(dev)
+        self.cache = init["conv_state"][:, :, ch].contiguous().to(dev)
+        self.layer = Layer(gdn, dev, gi.conv_weight(seed)[ch], Hk, Hv)
         self.cu = torch.arange(N_DECODE + 1, dtype=torch.int32, device=dev)
         self.inputs = []
         for s in range(steps):
             st = gi.decode_step_inputs(s, N_DECODE, seed)
-            self.inputs.append({k: v.to(dev) for k, v in st.items()})
-        self.y = torch.empty((N_DECODE, gi.CONV_CHANNELS), dtype=torch.bfloat16, device=dev)
-        self.o = torch.empty((N_DECODE, H_V, D), dtype=torch.bfloat16, device=dev)
+            self.inputs.append({"x_pre": st["x_pre"][:, ch].contiguous().to(dev),
+                                "g": st["g"][:, vh0:vh1].contiguous().to(dev),
+                                "beta": st["beta"][:, vh0:vh1].contiguous().to(dev),
+                                "z": st["z"][:, vh0:vh1].contiguous().to(dev)})
+        self.y = torch.empty((N_DECODE, len(ch)), dtype=torch.bfloat16, device=dev)
+        self.o = torch.empty((N_DECODE, Hv, D), dtype=torch.bfloat16, device=dev)
         self.out = torch.empty_like(self.o)
         self.launches_per_step = 4
+        self.bytes = N_DECODE * (DECODE_BYTES_PER_TOKEN * Hv // H_V)
 
     def step(self, s, ev=None):
-        g, st = self.gdn, self.inputs[s % len(self.inputs)]
-        g.gdn_conv1d_silu(st["x_pre"], self.w, self.cu, conv_state_in=self.cache,
-                          conv_state_out=self.cache, y=self.y)
+        g, st, L = self.gdn, self.inputs[s % len(self.inputs)], self.layer
+        g.gdn_conv1d_silu(st["x_pre"], L.w, self.cu, conv_state_in=self.cache,
+                          conv_state_out=self.cache, l2norm_channels=L.kc, y=self.y)
         if ev is not None:
             ev[0].record()
-        y = self.y
-        g.gdn_decode_step(y[:, :2048].view(-1, H_K, D), y[:, 2048:4096].view(-1, H_K, D),
-                          y[:, 4096:].view(-1, H_V, D), st["g"], st["beta"], self.state,
-                          o=self.o)
+        q, k, v = L.views(self.y)
+        g.gdn_decode_step(q, k, v, st["g"], st["beta"], self.state, o=self.o)
         if ev is not None:
             ev[1].record()
-        g.gdn_gated_rmsnorm(self.o, st["z"], self.nw, eps=1e-6, y=self.out)
+        g.gdn_gated_rmsnorm(self.o, st["z"], L.nw, eps=1e-6, y=self.out)
 
 
 class RankGroup:
@@ -231,32 +382,51 @@ def throughput(units_per_rank, world, max_ms):
     return units_per_rank * world / (max_ms * 1e-3)
 
 
-def timed_loop(step_fn, steps, warmup, dist_barrier):
-    """Warm up, then time exactly `steps` back-to-back steps. Each step's
-    region and its dominant kernel are bracketed by CUDA events on the
-    current (launching) stream. No L2 flush: every workload's inputs exceed
-    the 126 MB L2, and back-to-back steps also pay for the previous step's
-    write-backs, as a steady stream of calls would. Returns (per-step ms
-    list, dominant-kernel ms list)."""
+class KernelEvents:
+    """CUDA-event pairs around a step's calls of its dominant kernel, on the
+    launching stream: ev[0].record() opens a pair, ev[1].record() closes it
+    (a step that calls the kernel several times records several pairs)."""
+
+    def __init__(self):
+        self.pairs = []
+
+    def __getitem__(self, j):
+        if j == 0:
+            self.pairs.append([torch.cuda.Event(enable_timing=True) for _ in range(2)])
+        return self.pairs[-1][j]
+
+    def ms(self):
+        return sum(a.elapsed_time(b) for a, b in self.pairs)
+
+
+def timed_loop(step_fn, steps, warmup, dist_barrier, flush=None):
+    """Warm up, then time exactly `steps` steps. Each step's region and its
+    dominant kernel are bracketed by CUDA events on the current (launching)
+    stream. Without `flush` the steps run back to back (every workload's
+    inputs exceed the 126 MB L2, and each step also pays the previous step's
+    write-backs); with it, `flush()` writes a buffer larger than L2 between
+    steps, outside the events. Returns (per-step ms, per-step kernel ms)."""
     for i in range(warmup):
         step_fn(i, None)
     torch.cuda.synchronize()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
     dist_barrier()
     torch.cuda.synchronize()
+    rec = []
     for i in range(steps):
-        e = evs[i]
-        e[0].record()
-        step_fn(i, (e[1], e[2]))
-        e[3].record()
+        if flush is not None:
+            flush()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        kev = KernelEvents()
+        a.record()
+        step_fn(i, kev)
+        b.record()
+        rec.append((a, b, kev))
     torch.cuda.synchronize()
     dist_barrier()
-    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
-    kern_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    return step_ms, kern_ms
+    return [a.elapsed_time(b) for a, b, _ in rec], [k.ms() for _, _, k in rec]
 
 
-def e2e_prefill(gdn, wl, dev, steps, warmup):
+def e2e_prefill(wl, dev, steps, warmup):
     """Same workload through the public API from pinned HOST buffers: every
     step's inputs are copied host->device and its output device->host inside
     the timed region. Steps are pipelined as a serving loop would run them:
@@ -314,6 +484,14 @@ def e2e_prefill(gdn, wl, dev, steps, warmup):
     return ms, h2d, d2h
 
 
+def tensor_roofline(name, flop, kms, peaks, peak_src, traffic):
+    ach = flop / (kms * 1e-3) / 1e12
+    return {"kernel": name, "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"],
+            "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"],
+            "peak_source": f"{peak_src} bf16 dense (burst)", "traffic": traffic,
+            "algorithmic_flop_per_launch": flop, "kernel_ms": kms}
+
+
 def gpu_arm(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -334,79 +512,129 @@ def gpu_arm(args):
     import gated_delta_rule_106_b200 as gdn
     gdn.load()
     peaks, peak_src = load_peaks()
+    heads = args.shard == "heads" and world > 1
+    shard = head_shard(rank, world) if heads else (0, H_K, 0, H_V)
+    seed = 0 if heads else rank     # head shards split one workload; replicas draw their own
+    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = lambda: flush_buf.fill_(1)
+    mean_max = lambda xs: max_over_ranks(statistics.mean(xs))
 
-    pre = PrefillWorkload(gdn, dev, seed=rank)
+    pre = PrefillWorkload(gdn, dev, seed, shard)
     with ClockSampler(local) as clk:
-        step_ms, kern_ms = timed_loop(lambda i, ev: pre.step(ev), args.steps,
-                                      args.warmup, barrier)
-    ms = max_over_ranks(statistics.mean(step_ms))
-    kms = max_over_ranks(statistics.mean(kern_ms))
-    e2e_ms, h2d, d2h = e2e_prefill(gdn, pre, dev, max(4, args.steps), 2)
+        step_ms, kern_ms = timed_loop(pre.step, args.steps, args.warmup, barrier)
+        ms, kms = mean_max(step_ms), mean_max(kern_ms)
+        f_step, f_kern = timed_loop(pre.step, args.steps, args.warmup, barrier, flush=flush)
+        f_ms, f_kms = mean_max(f_step), mean_max(f_kern)
+
+        var = VarlenWorkload(gdn, dev, seed, shard)
+        v_step, v_kern = timed_loop(var.step, args.steps, args.warmup, barrier)
+        v_ms, v_kms = mean_max(v_step), mean_max(v_kern)
+        v_tokens, v_flop = var.tokens, var.flop
+        del var
+
+        dwl = DecodeWorkload(gdn, dev, seed, DECODE_STEPS, shard)
+        d_step, d_kern = timed_loop(dwl.step, DECODE_STEPS, args.warmup, barrier)
+        d_ms, d_kms = mean_max(d_step), mean_max(d_kern)
+        d_bytes = dwl.bytes
+        del dwl
+
+        lc = LongContextWorkload(gdn, dev, seed, shard)
+        lsteps = max(1, min(args.steps, 5))
+        lc_fn = lambda i, ev: [lc.segment(s, ev) for s in range(N_SEG)]
+        l_step, l_kern = timed_loop(lc_fn, lsteps, 1, barrier)
+        l_ms, l_kms = mean_max(l_step), mean_max(l_kern)
+        # flushed: L2 written between the 64 calls (outside the events)
+        seg_ms, seg_kern = timed_loop(lambda i, ev: lc.segment(i % N_SEG, ev), N_SEG, 1,
+                                      barrier, flush=flush)
+        lf_ms, lf_kms = max_over_ranks(sum(seg_ms)), max_over_ranks(sum(seg_kern))
+        l_tokens, l_flop = lc.tokens, lc.flop
+        del lc
+    e2e_ms, h2d, d2h = e2e_prefill(pre, dev, max(4, args.steps), 2)
     e2e_ms = max_over_ranks(e2e_ms)
 
-    dec_steps = 128
-    dwl = DecodeWorkload(gdn, dev, seed=rank, steps=dec_steps)
-    d_step_ms, d_kern_ms = timed_loop(lambda i, ev: dwl.step(i, ev), dec_steps,
-                                      args.warmup, barrier)
-    d_ms = max_over_ranks(statistics.mean(d_step_ms))
-    d_kms = max_over_ranks(statistics.mean(d_kern_ms))
-
-    flops = PREFILL_FLOP_PER_TOKEN * T_PREFILL
-    pre_ach = flops / (kms * 1e-3) / 1e12
-    dec_bytes = DECODE_BYTES_PER_TOKEN * N_DECODE
-    dec_ach = dec_bytes / (d_kms * 1e-3) / 1e9
-    tr = kernel_traffic("prefill")
-    dtr = kernel_traffic("decode")
+    Hv = shard[3] - shard[2]
+    flops = pre.flop
+    dec_ach = d_bytes / (d_kms * 1e-3) / 1e9
+    units = 1 if heads else world       # head shards together make one workload
     line = {
         "metric": METRIC,
-        "value": throughput(T_PREFILL, world, ms),
+        "value": throughput(T_PREFILL, units, ms),
         "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms,
         "higher_is_better": True,
-        "scaling": "weak",
+        "scaling": "strong" if heads else "weak",
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded; shapes and distributions of the layer)",
         "config": {
             "workload": "prefill: one delta-rule layer, B=1, T=8192, 16 key / 48 value "
                         "heads, d=128; conv k=4+SiLU+L2 -> chunked C=64 -> gated RMSNorm",
-            "global_batch": world, "seq_len": T_PREFILL,
-            "parallelism": f"replicas{world}" if world > 1 else "single",
-            "l2": "no flush: inputs exceed L2 (x_pre 168 MB; decode state 768 MiB); "
-                  "steps run back to back",
+            "global_batch": units, "seq_len": T_PREFILL,
+            "parallelism": (f"heads{world} ({shard[1] - shard[0]} key / {Hv} value heads per rank)"
+                            if heads else (f"replicas{world}" if world > 1 else "single")),
+            "l2": "no flush: inputs exceed L2 (x_pre 168 MB; decode state 768 MiB); steps run "
+                  "back to back (flushed variant under prefill_l2_flushed)",
         },
-        "roofline": {
-            "kernel": "gdn_chunked_prefill",
-            "bound": "tensor", "achieved": pre_ach,
-            "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-            "frac": pre_ach / peaks["bf16_tflops"],
-            "peak_source": f"{peak_src} bf16 dense (burst)",
-            "traffic": tr,
-            "algorithmic_flop_per_launch": flops,
-            "kernel_ms": kms,
-        },
-        "e2e": {"value": throughput(T_PREFILL, world, e2e_ms), "unit": "tokens/s",
+        "roofline": tensor_roofline("gdn_chunked_prefill", flops, kms, peaks, peak_src,
+                                    kernel_traffic("prefill") if not heads else None),
+        "e2e": {"value": throughput(T_PREFILL, units, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms},
         "gpu_launches": pre.launches_per_step * args.steps,
         "clocks": clk.summary(),
+        "prefill_l2_flushed": {
+            "value": throughput(T_PREFILL, units, f_ms), "unit": "tokens/s", "ms_per_step": f_ms,
+            "l2": f"{L2_FLUSH_BYTES >> 20} MB written between steps (outside the events)",
+            "roofline": tensor_roofline("gdn_chunked_prefill", flops, f_kms, peaks, peak_src,
+                                        None)},
+        "varlen": {
+            "workload": f"{N_VARLEN} packed sequences, lengths uniform in [512, 16384] "
+                        f"({v_tokens} tokens), fp32 initial/final states; conv -> chunked "
+                        "prefill -> gated RMSNorm",
+            "value": throughput(v_tokens, units, v_ms), "unit": "tokens/s", "ms_per_step": v_ms,
+            "roofline": tensor_roofline("gdn_chunked_prefill", v_flop, v_kms, peaks, peak_src,
+                                        None),
+            "gpu_launches": 3 * args.steps},
         "decode": {
             "workload": "decode: 256 sequences x 128 steps, 1 token each, fp32 state "
                         "[256,48,128,128]; conv (cache roll) -> decode step -> gated RMSNorm",
-            "value": throughput(N_DECODE, world, d_ms), "unit": "tokens/s",
+            "value": throughput(N_DECODE, units, d_ms), "unit": "tokens/s",
             "ms_per_step": d_ms,
             "roofline": {"kernel": "gdn_decode_step", "bound": "hbm",
                          "achieved": dec_ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": dec_ach / peaks["hbm_gbs"],
                          "peak_source": f"{peak_src} HBM copy",
-                         "traffic": dtr, "algorithmic_bytes_per_launch": dec_bytes,
-                         "kernel_ms": d_kms},
-            "gpu_launches": dwl.launches_per_step * dec_steps,
+                         "traffic": kernel_traffic("decode") if not heads else None,
+                         "algorithmic_bytes_per_launch": d_bytes, "kernel_ms": d_kms},
+            "gpu_launches": 4 * DECODE_STEPS,
+        },
+        "long_context": {
+            "workload": f"T={SEG * N_SEG} as {N_SEG} calls of {SEG} tokens, recurrent state "
+                        "and conv history carried; one step = all calls",
+            "value": throughput(l_tokens, units, l_ms), "unit": "tokens/s", "ms_per_step": l_ms,
+            "steps": lsteps,
+            "roofline": tensor_roofline("gdn_chunked_prefill", l_flop, l_kms, peaks, peak_src,
+                                        None),
+            "l2_flushed": {"value": throughput(l_tokens, units, lf_ms), "unit": "tokens/s",
+                           "ms_per_step": lf_ms,
+                           "l2": f"{L2_FLUSH_BYTES >> 20} MB written between the calls",
+                           "roofline": tensor_roofline("gdn_chunked_prefill", l_flop, lf_kms,
+                                                       peaks, peak_src, None)},
+            "gpu_launches": 4 * N_SEG * lsteps,
         },
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(args.cpu_budget_s)
+        cb, ref_out, nheads = cpu_baseline(args.cpu_budget_s)
+        line["cpu_baseline"] = cb
+        got = pre.out[:, :nheads].double().cpu().numpy()
+        d = got - ref_out
+        line["chain_error"] = {
+            "what": "normed layer output of the timed step vs the fp64 oracle chain (conv -> "
+                    "recurrence -> gated RMSNorm) from the same x_pre, no GPU intermediate",
+            "value_heads": nheads,
+            "max_abs_over_rms": float(np.abs(d).max() / np.sqrt(np.mean(ref_out ** 2))),
+            "rel_frobenius": float(np.linalg.norm(d) / np.linalg.norm(ref_out))}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist is not None:
@@ -419,7 +647,8 @@ def gpu_arm(args):
 def oracle_sample(threads=0, heads=H_V, tokens=T_PREFILL, seed=0):
     """The oracle on (part of) the prefill workload: conv of every channel of
     `tokens` tokens, the recurrence for `heads` value heads (whole key-head
-    groups) and the gated RMS-norm of those heads. Returns (seconds, threads)."""
+    groups) and the gated RMS-norm of those heads. Returns (seconds, threads,
+    normed output [tokens, heads, 128])."""
     import oracle
     p = gi.prefill_inputs(T=tokens, seed=seed)
     x = gi.as_f64(p["x_pre"])
@@ -436,27 +665,29 @@ def oracle_sample(threads=0, heads=H_V, tokens=T_PREFILL, seed=0):
     o, _ = oracle.recurrence(q, k, v, gi.as_f64(p["g"])[:, :heads],
                              gi.as_f64(p["beta"])[:, :heads], None, cu,
                              threads=nthreads)
-    oracle.gated_rmsnorm(o, gi.as_f64(p["z"])[:, :heads], gi.as_f64(p["norm_w"]),
-                         1e-6, threads=nthreads)
-    return time.perf_counter() - t0, nthreads
+    out = oracle.gated_rmsnorm(o, gi.as_f64(p["z"])[:, :heads], gi.as_f64(p["norm_w"]),
+                               1e-6, threads=nthreads)
+    return time.perf_counter() - t0, nthreads, out
 
 
 def cpu_baseline(budget_s=20.0):
     """Oracle throughput on the host cores, scaled to tokens/s of the whole
-    layer: a short probe on 3 heads sizes a sample of ~budget_s seconds."""
-    probe_s, _ = oracle_sample(heads=3, tokens=1024)
+    layer: a short probe on 3 heads sizes a sample of ~budget_s seconds.
+    Returns (baseline dict, the oracle's normed output, its value heads)."""
+    probe_s, _, _ = oracle_sample(heads=3, tokens=1024)
     hw = os.cpu_count() or 1
     # conv dominates the probe's fixed part; size heads so the sample fits
     est_per_head = probe_s / 3 * (T_PREFILL / 1024)
     heads = int(max(3, min(H_V, (budget_s / max(est_per_head, 1e-9)) * min(hw, H_V))))
     heads -= heads % 3
-    sec, threads = oracle_sample(heads=heads)
+    sec, threads, out = oracle_sample(heads=heads)
     # the conv covers all heads already; scale the recurrence+norm share
     layer_s = sec * (H_V / heads) if heads < H_V else sec
-    return {"value": T_PREFILL / layer_s, "unit": "tokens/s", "cores": threads,
-            "kind": "oracle",
-            "sample": f"T={T_PREFILL}: full conv, recurrence + gated RMSNorm for "
-                      f"{heads}/{H_V} value heads ({sec:.1f} s), scaled to 48 heads"}
+    return ({"value": T_PREFILL / layer_s, "unit": "tokens/s", "cores": threads,
+             "kind": "oracle",
+             "sample": f"T={T_PREFILL}: full conv, recurrence + gated RMSNorm for "
+                       f"{heads}/{H_V} value heads ({sec:.1f} s), scaled to 48 heads"},
+            out, heads)
 
 
 def reference_arm(args):
@@ -470,7 +701,7 @@ def reference_arm(args):
     secs = []
     threads = 0
     for _ in range(args.steps):
-        s, threads = oracle_sample(heads=heads, tokens=1024)
+        s, threads, _ = oracle_sample(heads=heads, tokens=1024)
         secs.append(s)
     per_step = statistics.mean(secs)
     # tokens/s of the whole layer: 1024 tokens, 3 of 48 heads (conv: all)
@@ -495,18 +726,92 @@ def reference_arm(args):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------- profiler cases --
+
+def profile_case(args):
+    """A few fixed launches of one kernel, for a profiler capture. Inputs are
+    synthetic and seeded, larger than the 126 MB L2 at the defaults (so DRAM
+    counters mean something) and a few GB at most. Prints the mean CUDA-event
+    time per launch, for reference only."""
+    import gated_delta_rule_106_b200 as gdn
+    gdn.load()
+    dev = "cuda"
+    name, N, T = args.profile_case, args.n, args.t
+    if name == "decode":
+        st = gi.decode_step_inputs(0, N, seed=0)
+        state = gi.initial_states(0, N, tag="pstate").to(dev)
+        q = gi.to_bf16(gi.unit_heads(0, "pq", N, 16)).to(dev)
+        k = gi.to_bf16(gi.unit_heads(0, "pk", N, 16)).to(dev)
+        v = gi.to_bf16(gi.normal(0, "pv", (N, 48, 128))).to(dev)
+        g, b = st["g"].to(dev), st["beta"].to(dev)
+        o = torch.empty((N, 48, 128), dtype=torch.bfloat16, device=dev)
+        run = lambda: gdn.gdn_decode_step(q, k, v, g, b, state, o=o, scale=0.05)
+    elif name in ("prefill", "varlen"):
+        cu = (torch.tensor([0, T], dtype=torch.int32) if name == "prefill"
+              else gi.varlen_cu_seqlens(N_VARLEN, 512, 16384, seed=0))
+        T = int(cu[-1])
+        p = gi.prefill_inputs(T=T, seed=0, cu_seqlens=cu, with_state=name == "varlen")
+        y = gdn.gdn_conv1d_silu(p["x_pre"].to(dev), p["conv_w"].to(dev), cu.to(dev))
+        q, k, v = (y[:, :2048].view(T, 16, 128), y[:, 2048:4096].view(T, 16, 128),
+                   y[:, 4096:].view(T, 48, 128))
+        g, b, cud = p["g"].to(dev), p["beta"].to(dev), cu.to(dev)
+        si = p["state_in"].to(dev) if p["state_in"] is not None else None
+        o = torch.empty((T, 48, 128), dtype=torch.bfloat16, device=dev)
+        S = torch.empty((cu.numel() - 1, 48, 128, 128), device=dev)
+        run = lambda: gdn.gdn_chunked_prefill(q, k, v, g, b, cud, state_in=si, state_out=S, o=o)
+    elif name == "conv":
+        p = gi.prefill_inputs(T=T, seed=0)
+        x, w, cu = p["x_pre"].to(dev), p["conv_w"].to(dev), p["cu_seqlens"].to(dev)
+        y = torch.empty_like(x)
+        run = lambda: gdn.gdn_conv1d_silu(x, w, cu, y=y)
+    elif name == "norm":
+        x = gi.gate_z(1, T, tag="px").to(dev)
+        z = gi.gate_z(0, T).to(dev)
+        w = torch.ones(128, device=dev)
+        y = torch.empty_like(x)
+        run = lambda: gdn.gdn_gated_rmsnorm(x, z, w, eps=1e-6, y=y)
+    elif name == "dconv":
+        cache = gi.to_bf16(gi.normal(0, "dconv", (N, 3, gi.CONV_CHANNELS))).to(dev)
+        x = gi.decode_step_inputs(0, N, 0)["x_pre"].to(dev)
+        w = gi.conv_weight(0).to(dev)
+        cu = torch.arange(N + 1, dtype=torch.int32, device=dev)
+        y = torch.empty((N, gi.CONV_CHANNELS), dtype=torch.bfloat16, device=dev)
+        run = lambda: gdn.gdn_conv1d_silu(x, w, cu, conv_state_in=cache, conv_state_out=cache,
+                                          y=y)
+    else:
+        raise SystemExit(f"unknown profile case {name}")
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(args.launches):
+        run()
+    e.record()
+    torch.cuda.synchronize()
+    print(f"{name}: {s.elapsed_time(e) / args.launches:.4f} ms per launch")
+
+
+PROFILE_CASES = ("decode", "prefill", "varlen", "conv", "norm", "dconv")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="gdn", choices=["gdn", "reference"])
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=20.0)
+    ap.add_argument("--profile-case", choices=PROFILE_CASES)
+    ap.add_argument("--n", type=int, default=64)
+    ap.add_argument("--t", type=int, default=8192)
+    ap.add_argument("--launches", type=int, default=4)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    if args.impl == "reference":
+    if args.profile_case:
+        profile_case(args)
+    elif args.impl == "reference":
         reference_arm(args)
     else:
         gpu_arm(args)

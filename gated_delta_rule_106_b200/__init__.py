@@ -23,6 +23,7 @@ import torch
 __all__ = ["GDN_BF16", "GDN_F32", "GdnError", "library_path", "load",
            "gdn_conv1d_silu", "gdn_chunked_prefill",
            "gdn_chunked_prefill_workspace", "gdn_chunked_prefill_noalloc",
+           "gdn_stepwise_prefill",
            "gdn_decode_step",
            "gdn_gated_rmsnorm", "gdn_status_string", "gdn_version",
            "H_K", "H_V", "HEAD_DIM", "CHUNK"]
@@ -52,6 +53,9 @@ _SIGNATURES = {
                                    _int, _f32, _vp, _int, _vp, ctypes.c_size_t,
                                    _vp]),
     "gdn_chunked_prefill_workspace": (ctypes.c_size_t, [_int, _i64, _int, _int]),
+    "gdn_stepwise_prefill": (_int, [_vp, _vp, _vp, _int, _i64, _i64, _i64, _vp,
+                                    _vp, _int, _vp, _vp, _vp, _int, _i64, _int,
+                                    _int, _f32, _vp, _int, _vp]),
     "gdn_chunked_prefill_noalloc": (_int, [_vp, _vp, _vp, _int, _i64, _i64, _i64, _vp,
                                            _vp, _int, _vp, _vp, _vp, _int, _i64, _int,
                                            _int, _f32, _vp, _int, _vp]),
@@ -208,7 +212,8 @@ def gdn_chunked_prefill(q, k, v, g, beta, cu_seqlens, *, state_in=None,
                           H_k, H_v, N)
     if o is None:
         o = torch.empty((T, H_v, HEAD_DIM), dtype=o_dtype or v.dtype, device=v.device)
-    need = gdn_chunked_prefill_workspace(N, T, H_k, H_v)
+    # only the tensor-core path (bf16 inputs) works in a workspace
+    need = gdn_chunked_prefill_workspace(N, T, H_k, H_v) if q.dtype == torch.bfloat16 else 0
     if workspace is None and need:
         workspace = torch.empty(need, dtype=torch.uint8, device=v.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
@@ -218,6 +223,26 @@ def gdn_chunked_prefill(q, k, v, g, beta, cu_seqlens, *, state_in=None,
         _ptr(state_in), _ptr(state_out), _ptr(cu_seqlens), N, T, H_k, H_v,
         scale, _ptr(o), _dtype_code(o.dtype), _ptr(workspace), ws_bytes,
         _stream(stream, v.device)))
+    return o
+
+
+def gdn_stepwise_prefill(q, k, v, g, beta, cu_seqlens, *, state_in=None,
+                         state_out=None, scale=1.0, o=None, o_dtype=None,
+                         stream=None):
+    """The same recurrence as gdn_chunked_prefill advanced token by token (the
+    stepwise path), fp32 on the CUDA cores. Same arguments, no workspace."""
+    T, H_k, _ = q.shape
+    H_v = v.shape[1]
+    N = cu_seqlens.numel() - 1
+    _check_prefill_shapes(q, k, v, g, beta, cu_seqlens, state_in, state_out, o, T,
+                          H_k, H_v, N)
+    if o is None:
+        o = torch.empty((T, H_v, HEAD_DIM), dtype=o_dtype or v.dtype, device=v.device)
+    _check("gdn_stepwise_prefill", load().gdn_stepwise_prefill(
+        _ptr(q), _ptr(k), _ptr(v), _dtype_code(q.dtype), _row_stride(q),
+        _row_stride(k), _row_stride(v), _ptr(g), _ptr(beta), _dtype_code(g.dtype),
+        _ptr(state_in), _ptr(state_out), _ptr(cu_seqlens), N, T, H_k, H_v,
+        scale, _ptr(o), _dtype_code(o.dtype), _stream(stream, v.device)))
     return o
 
 

@@ -145,7 +145,33 @@ gdn_status gdn_chunked_prefill(const void* q, const void* k, const void* v,
                    T_total, H_k, H_v, scale, o, o_dtype, workspace,
                    workspace_bytes, stream};
   return from_cuda(qkv_dtype == GDN_BF16 ? gdn::launch_prefill_pc(a)
-                                         : gdn::launch_prefill_stepwise(a));
+                                         : gdn::launch_prefill_chunked_f32(a));
+}
+
+gdn_status gdn_stepwise_prefill(const void* q, const void* k, const void* v,
+                                gdn_dtype qkv_dtype, int64_t q_row_stride,
+                                int64_t k_row_stride, int64_t v_row_stride,
+                                const void* g, const void* beta,
+                                gdn_dtype gate_dtype, const float* state_in,
+                                float* state_out, const int32_t* cu_seqlens,
+                                int N, int64_t T_total, int H_k, int H_v,
+                                float scale, void* o, gdn_dtype o_dtype,
+                                cudaStream_t stream) {
+  if (N < 0 || T_total < 0) return GDN_ERR_INVALID_ARG;
+  gdn_status st = check_recurrence(q, k, v, qkv_dtype, q_row_stride, k_row_stride,
+                                   v_row_stride, g, beta, gate_dtype, H_k, H_v,
+                                   o, o_dtype, T_total > 0);
+  if (st != GDN_OK) return st;
+  if (N == 0) return T_total == 0 ? GDN_OK : GDN_ERR_INVALID_ARG;
+  if (!cu_seqlens) return GDN_ERR_INVALID_ARG;
+  if ((state_in && !aligned16(state_in)) || (state_out && !aligned16(state_out)))
+    return GDN_ERR_MISALIGNED;
+  const size_t st_bytes = (size_t)N * H_v * kHeadDim * kHeadDim * sizeof(float);
+  if (partial_overlap(state_in, st_bytes, state_out, st_bytes)) return GDN_ERR_INVALID_ARG;
+  gdn::RecurArgs a{q, k, v, qkv_dtype, q_row_stride, k_row_stride, v_row_stride,
+                   g, beta, gate_dtype, state_in, state_out, cu_seqlens, N,
+                   T_total, H_k, H_v, scale, o, o_dtype, nullptr, 0, stream};
+  return from_cuda(gdn::launch_prefill_stepwise(a));
 }
 
 gdn_status gdn_chunked_prefill_noalloc(const void* q, const void* k, const void* v,
@@ -175,7 +201,7 @@ gdn_status gdn_chunked_prefill_noalloc(const void* q, const void* k, const void*
                    g, beta, gate_dtype, state_in, state_out, cu_seqlens, N,
                    T_total, H_k, H_v, scale, o, o_dtype, nullptr, 0, stream};
   return from_cuda(qkv_dtype == GDN_BF16 ? gdn::launch_prefill_pc_noalloc(a)
-                                         : gdn::launch_prefill_stepwise(a));
+                                         : gdn::launch_prefill_chunked_f32(a));
 }
 
 size_t gdn_chunked_prefill_noalloc_scratch_bytes(void) {

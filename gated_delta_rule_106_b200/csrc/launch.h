@@ -43,6 +43,8 @@ cudaError_t launch_gated_rmsnorm(const NormArgs& a);
 cudaError_t launch_decode_step(const RecurArgs& a);
 // Stepwise fp32 recurrence on the CUDA cores (any input dtype).
 cudaError_t launch_prefill_stepwise(const RecurArgs& a);
+// Chunk-64 recurrence on the CUDA cores in fp32 (fp32 inputs; any input dtype).
+cudaError_t launch_prefill_chunked_f32(const RecurArgs& a);
 // Chunk-64 tensor-core prefill (bf16 inputs), persistent producer/consumer
 // kernel over all SMs; needs prefill_pc_workspace() bytes of workspace.
 cudaError_t launch_prefill_pc(const RecurArgs& a);

@@ -1158,7 +1158,7 @@ size_t prefill_pc_workspace(int N, int64_t T_total, int H_v) {
 
 cudaError_t launch_prefill_pc(const RecurArgs& a) {
   if (a.N == 0) return cudaSuccess;
-  if (a.T_total == 0) return launch_prefill_stepwise(a);   // only state copies
+  if (a.T_total == 0) return launch_prefill_chunked_f32(a);   // only state copies
   const int nsm = sm_count();
   if (nsm < 2) return cudaErrorInvalidDevice;
   const int NS = state_ctas((int64_t)a.N * a.H_v, a.H_v, nsm);

@@ -1,7 +1,6 @@
 // Stepwise gated delta rule over packed sequences on the CUDA cores, fp32.
 //
-// This serves gdn_chunked_prefill for fp32 inputs, where every product must
-// stay in fp32: the recurrence
+// This serves gdn_stepwise_prefill: the recurrence
 //   S_t = g_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T, o_t = scale S_t q_t
 // ("Agnes-3.0-Flash Preview" leaderboard commentary, section 二.1: the chunked
 // prefill and stepwise decode paths compute the same recurrence; the model

@@ -130,7 +130,9 @@ gdn_status gdn_conv1d_silu(const void* x, int64_t x_row_stride,
  * binary16 exactly when |x| lies in [2^-14, 65504]; smaller magnitudes keep
  * an absolute error below 2^-25); the state is carried in fp32. Inputs,
  * states and outputs must stay well inside the binary16 range (|x| < 6e4).
- * With qkv_dtype == GDN_F32 every product is fp32 on the CUDA cores.
+ * With qkv_dtype == GDN_F32 the same chunk-64 form runs on the CUDA cores
+ * with every product in fp32 (one CTA per sequence and value head); it needs
+ * no workspace.
  */
 gdn_status gdn_chunked_prefill(const void* q, const void* k, const void* v,
                                gdn_dtype qkv_dtype, int64_t q_row_stride,
@@ -145,6 +147,28 @@ gdn_status gdn_chunked_prefill(const void* q, const void* k, const void* v,
 
 /* Device scratch bytes gdn_chunked_prefill needs for these sizes (host). */
 size_t gdn_chunked_prefill_workspace(int N, int64_t T_total, int H_k, int H_v);
+
+/*
+ * gdn_stepwise_prefill -- the same packed-sequence recurrence advanced token by
+ * token (the stepwise path of [P2 二.1], which the modeling code uses for
+ * decode), for any prompt length: the recurrence written out, in fp32 on the
+ * CUDA cores. A warp owns 32 rows of one (sequence, value head) state and
+ * keeps them in registers for the whole sequence, so the state crosses HBM
+ * once per call; the time grows with the longest sequence (one dependent
+ * update per token). It is the reference-grade path next to the chunked one:
+ * both compute the same recurrence and must agree up to rounding.
+ * Arguments, layouts and errors are those of gdn_chunked_prefill without the
+ * workspace. Additional entry point (the pages name the path, not the call).
+ */
+gdn_status gdn_stepwise_prefill(const void* q, const void* k, const void* v,
+                                gdn_dtype qkv_dtype, int64_t q_row_stride,
+                                int64_t k_row_stride, int64_t v_row_stride,
+                                const void* g, const void* beta,
+                                gdn_dtype gate_dtype, const float* state_in,
+                                float* state_out, const int32_t* cu_seqlens,
+                                int N, int64_t T_total, int H_k, int H_v,
+                                float scale, void* o, gdn_dtype o_dtype,
+                                cudaStream_t stream);
 
 /*
  * gdn_chunked_prefill_noalloc -- gdn_chunked_prefill with no workspace

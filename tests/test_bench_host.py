@@ -88,3 +88,42 @@ def test_reference_arm_under_two_ranks_prints_once():
     lines = json_lines(r.stdout)
     assert len(lines) == 1 and lines[0]["impl"] == "reference"
     assert lines[0]["n_gpus"] == 2
+
+
+def _shards(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        mine = bench.head_shard(rank, world)
+        got = [None] * world
+        dist.all_gather_object(got, mine)
+        out[rank] = got
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_head_shards_tile_the_layer_on_gloo_ranks(world):
+    """bench.py --shard heads: every rank takes whole key-head groups; over the
+    ranks the key heads tile 0..15 and the value heads 0..47, and local value
+    head j of a rank reads local key head j // 3, i.e. global value head h reads
+    global key head h // 3 as in the unsharded layer."""
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_shards, args=(world, free_port(), out), nprocs=world, join=True,
+                       start_method="spawn")
+    views = [out[r] for r in range(world)]
+    assert all(v == views[0] for v in views)          # every rank sees the same plan
+    kh, vh = [], []
+    for r, (k0, k1, v0, v1) in enumerate(views[0]):
+        kh += list(range(k0, k1))
+        vh += list(range(v0, v1))
+        for j in range(v1 - v0):
+            assert k0 + j // 3 == (v0 + j) // 3
+        ch = bench.shard_channels(k0, k1, v0, v1)
+        assert len(ch) == 2 * (k1 - k0) * 128 + (v1 - v0) * 128
+        assert ch[0] == 128 * k0 and ch[(k1 - k0) * 128] == 2048 + 128 * k0
+        assert ch[2 * (k1 - k0) * 128] == 4096 + 128 * v0
+    assert kh == list(range(16)) and vh == list(range(48))
+    with pytest.raises(ValueError):
+        bench.head_shard(0, 3)

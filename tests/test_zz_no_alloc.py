@@ -5,9 +5,14 @@ operator inside a host framework whose allocator it cannot reach, a serving
 loop that must not allocate after start-up). For them the library offers a
 variant of the chunked prefill that works in its own static device array. This
 test calls it through the C ABI twice in a row on the same inputs and checks
-each result against the regular entry point (which is given a workspace), with
-the tolerances the other prefill tests use. The file is named so that pytest
-collects it last; it also passes when run alone in a fresh process.
+each result against the regular entry point (which is given a workspace). The
+two run the same kernel with the same launch shape, and its arithmetic does not
+depend on which CTA takes which work item, so the results must be identical
+bit for bit: a control word or ring slot left stale by the first call would show
+up on the second. The Python wrapper is called once as well. The file is named
+so that pytest collects it last; it also passes when run alone in a fresh
+process. (The size refusal, GDN_ERR_UNSUPPORTED, cannot be reached on a 148-SM
+B200: the array holds the rings of the most state CTAs the kernel uses there.)
 """
 import ctypes
 
@@ -17,7 +22,6 @@ import torch
 
 import gdn_inputs as gi
 import gated_delta_rule_106_b200 as gdn
-from _parity import O_TOL, S_TOL, o_err, state_err
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -51,5 +55,10 @@ def test_noalloc_matches_workspace_entry_point_twice():
             ctypes.c_float(1.0), o.data_ptr(), gdn.GDN_F32, stream)
         assert status == 0, gdn.gdn_status_string(status)
         torch.cuda.synchronize()
-        assert o_err(o, o_ref) <= O_TOL[torch.bfloat16], (call, o_err(o, o_ref))
-        assert state_err(S, S_ref) <= S_TOL[torch.bfloat16], (call, state_err(S, S_ref))
+        assert torch.equal(o, o_ref), (call, float((o - o_ref).abs().max()))
+        assert torch.equal(S, S_ref), (call, float((S - S_ref).abs().max()))
+    S = torch.full_like(S0, float("nan"))
+    o = gdn.gdn_chunked_prefill_noalloc(q, k, v, g, b, cu, state_in=S0, state_out=S,
+                                        o_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o_ref) and torch.equal(S, S_ref)
