@@ -66,8 +66,13 @@ FLOP_PER_TOKEN_HEAD = 6 * D * D + 6 * C * D + 4 * C * D / 3 + C * C / 1.5
 PREFILL_FLOP_PER_TOKEN = H_V * FLOP_PER_TOKEN_HEAD
 # bf16 q,k,v,o + fp32 g,beta per token
 PREFILL_BYTES_PER_TOKEN = 2 * (2 * H_K * D) + 2 * H_V * D + 2 * 4 * H_V + 2 * H_V * D
-# decode: fp32 state read + write, plus q,k (bf16), v, o (bf16), g, beta (bf16)
+# decode step kernel: fp32 state read + write, plus q,k (bf16), v, o (bf16), g, beta (bf16)
 DECODE_BYTES_PER_TOKEN = 2 * H_V * D * D * 4 + 2 * (2 * H_K * D) + 2 * 2 * H_V * D + 2 * 2 * H_V
+# fused decode layer step: fp32 state read + write, x (bf16, 10240 channels), the
+# 3-row conv cache read and written back rolled (bf16), z and y (bf16), g, beta (bf16)
+CONV_CH = 2 * H_K * D + H_V * D
+FUSED_DECODE_BYTES_PER_TOKEN = (2 * H_V * D * D * 4 + 2 * CONV_CH + 2 * 3 * 2 * CONV_CH
+                                + 2 * 2 * H_V * D + 2 * 2 * H_V)
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 
 
@@ -319,11 +324,17 @@ class LongContextWorkload:
 
 
 class DecodeWorkload:
-    def __init__(self, gdn, dev, seed, steps, shard):
+    """256 sequences, one token per step. fused: one gdn_decode_layer_step per
+    step on state and conv-cache pools indexed through a seeded permutation;
+    otherwise conv (in-place cache roll) -> gdn_decode_step -> gated RMS-norm."""
+
+    def __init__(self, gdn, dev, seed, steps, shard, fused):
         kh0, kh1, vh0, vh1 = shard
         Hk, Hv = kh1 - kh0, vh1 - vh0
         ch = torch.from_numpy(shard_channels(kh0, kh1, vh0, vh1))
-        self.gdn = gdn
+        self.gdn, self.fused = gdn, fused
+        self.idx = torch.from_numpy(
+            np.random.default_rng(seed).permutation(N_DECODE).astype(np.int32)).to(dev)
         init = gi.decode_initial(N_DECODE, seed)
         self.state = init["state"][:, vh0:vh1].contiguous().to(dev)
         self.cache = init["conv_state"][:, :, ch].contiguous().to(dev)
@@ -339,11 +350,22 @@ class DecodeWorkload:
         self.y = torch.empty((N_DECODE, len(ch)), dtype=torch.bfloat16, device=dev)
         self.o = torch.empty((N_DECODE, Hv, D), dtype=torch.bfloat16, device=dev)
         self.out = torch.empty_like(self.o)
-        self.launches_per_step = 4
-        self.bytes = N_DECODE * (DECODE_BYTES_PER_TOKEN * Hv // H_V)
+        self.launches_per_step = 2 if fused else 4
+        frac = Hv / H_V
+        self.bytes = int(N_DECODE * frac * (FUSED_DECODE_BYTES_PER_TOKEN if fused
+                                            else DECODE_BYTES_PER_TOKEN))
 
     def step(self, s, ev=None):
         g, st, L = self.gdn, self.inputs[s % len(self.inputs)], self.layer
+        if self.fused:
+            if ev is not None:
+                ev[0].record()
+            g.gdn_decode_layer_step(st["x_pre"], L.w, self.cache, st["g"], st["beta"],
+                                    self.state, self.idx, st["z"], L.nw, y=self.out,
+                                    H_k=L.H_k)
+            if ev is not None:
+                ev[1].record()
+            return
         g.gdn_conv1d_silu(st["x_pre"], L.w, self.cu, conv_state_in=self.cache,
                           conv_state_out=self.cache, l2norm_channels=L.kc, y=self.y)
         if ev is not None:
@@ -532,11 +554,16 @@ def gpu_arm(args):
         v_tokens, v_flop = var.tokens, var.flop
         del var
 
-        dwl = DecodeWorkload(gdn, dev, seed, DECODE_STEPS, shard)
+        dwl = DecodeWorkload(gdn, dev, seed, DECODE_STEPS, shard, fused=True)
         d_step, d_kern = timed_loop(dwl.step, DECODE_STEPS, args.warmup, barrier)
         d_ms, d_kms = mean_max(d_step), mean_max(d_kern)
         d_bytes = dwl.bytes
         del dwl
+        uwl = DecodeWorkload(gdn, dev, seed, DECODE_STEPS, shard, fused=False)
+        u_step, u_kern = timed_loop(uwl.step, DECODE_STEPS, args.warmup, barrier)
+        u_ms, u_kms = mean_max(u_step), mean_max(u_kern)
+        u_bytes = uwl.bytes
+        del uwl
 
         lc = LongContextWorkload(gdn, dev, seed, shard)
         lsteps = max(1, min(args.steps, 5))
@@ -555,6 +582,7 @@ def gpu_arm(args):
     Hv = shard[3] - shard[2]
     flops = pre.flop
     dec_ach = d_bytes / (d_kms * 1e-3) / 1e9
+    u_ach = u_bytes / (u_kms * 1e-3) / 1e9
     units = 1 if heads else world       # head shards together make one workload
     line = {
         "metric": METRIC,
@@ -597,16 +625,31 @@ def gpu_arm(args):
                                         None),
             "gpu_launches": 3 * args.steps},
         "decode": {
-            "workload": "decode: 256 sequences x 128 steps, 1 token each, fp32 state "
-                        "[256,48,128,128]; conv (cache roll) -> decode step -> gated RMSNorm",
+            "workload": "decode: 256 sequences x 128 steps, 1 token each, fp32 state pool "
+                        "[256,48,128,128] and conv-cache pool through a permuted state_idx; "
+                        "one fused launch per step (conv roll + SiLU + L2 -> recurrence -> "
+                        "gated RMSNorm)",
             "value": throughput(N_DECODE, units, d_ms), "unit": "tokens/s",
             "ms_per_step": d_ms,
-            "roofline": {"kernel": "gdn_decode_step", "bound": "hbm",
+            "roofline": {"kernel": "gdn_decode_layer_step", "bound": "hbm",
                          "achieved": dec_ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": dec_ach / peaks["hbm_gbs"],
                          "peak_source": f"{peak_src} HBM copy",
-                         "traffic": kernel_traffic("decode") if not heads else None,
+                         "traffic": kernel_traffic("decode_layer") if not heads else None,
                          "algorithmic_bytes_per_launch": d_bytes, "kernel_ms": d_kms},
+            "gpu_launches": 2 * DECODE_STEPS,
+        },
+        "decode_unfused": {
+            "workload": "the same decode workload as three calls per step: conv (cache roll) "
+                        "-> decode step -> gated RMSNorm",
+            "value": throughput(N_DECODE, units, u_ms), "unit": "tokens/s",
+            "ms_per_step": u_ms,
+            "roofline": {"kernel": "gdn_decode_step", "bound": "hbm",
+                         "achieved": u_ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": u_ach / peaks["hbm_gbs"],
+                         "peak_source": f"{peak_src} HBM copy",
+                         "traffic": kernel_traffic("decode") if not heads else None,
+                         "algorithmic_bytes_per_launch": u_bytes, "kernel_ms": u_kms},
             "gpu_launches": 4 * DECODE_STEPS,
         },
         "long_context": {

@@ -23,7 +23,7 @@ import torch
 __all__ = ["GDN_BF16", "GDN_F32", "GdnError", "library_path", "load",
            "gdn_conv1d_silu", "gdn_chunked_prefill",
            "gdn_chunked_prefill_workspace", "gdn_chunked_prefill_noalloc",
-           "gdn_stepwise_prefill",
+           "gdn_stepwise_prefill", "gdn_decode_layer_step",
            "gdn_decode_step",
            "gdn_gated_rmsnorm", "gdn_status_string", "gdn_version",
            "H_K", "H_V", "HEAD_DIM", "CHUNK"]
@@ -63,6 +63,9 @@ _SIGNATURES = {
     "gdn_decode_step": (_int, [_vp, _vp, _vp, _int, _i64, _i64, _i64, _vp, _vp,
                                _int, _vp, _int, _int, _int, _f32, _vp, _int,
                                _vp]),
+    "gdn_decode_layer_step": (_int, [_vp, _i64, _int, _vp, _int, _vp, _vp, _vp, _vp, _int,
+                                      _vp, _vp, _int, _int, _int, _int, _f32, _f32, _vp,
+                                      _vp, _f32, _vp, _int, _vp]),
     "gdn_gated_rmsnorm": (_int, [_vp, _int, _vp, _int, _vp, _int, _i64, _int,
                                  _f32, _vp, _int, _vp]),
 }
@@ -289,6 +292,40 @@ def gdn_decode_step(q, k, v, g, beta, state, *, scale=1.0, o=None,
         _ptr(state), N, H_k, H_v, scale, _ptr(o), _dtype_code(o.dtype),
         _stream(stream, v.device)))
     return o
+
+
+def gdn_decode_layer_step(x, conv_w, conv_state, g, beta, state, state_idx, z, norm_w, *,
+                          conv_bias=None, scale=1.0, l2_eps=1e-6, norm_eps=1e-6, y=None,
+                          y_dtype=None, H_k=H_K, stream=None):
+    """One decode token of the whole layer for N sequences (conv roll + SiLU +
+    q/k L2, the recurrence, gated RMS-norm) on pooled states: x [N, C] (C =
+    2*H_k*128 + H_v*128); conv_w [C, 4]; conv_state [P, 3, C] (x's dtype) and
+    state fp32 [P, H_v, 128, 128], both updated in place at the slots
+    state_idx int32 [N] (a slot outside [0, P) marks padding); g, beta [N, H_v];
+    z [N, H_v, 128] (x's dtype); norm_w [128] (conv_w's dtype). Returns the
+    normed output y [N, H_v, 128]."""
+    N, C = x.shape
+    P, H_v = state.shape[0], state.shape[1]
+    if C != (2 * H_k + H_v) * HEAD_DIM:
+        raise ValueError(f"x: {C} channels, expected {(2 * H_k + H_v) * HEAD_DIM}")
+    _expect(conv_w, (C, 4), "conv_w")
+    _expect(conv_bias, (C,), "conv_bias", conv_w.dtype)
+    _expect(conv_state, (P, 3, C), "conv_state", x.dtype)
+    _expect(g, (N, H_v), "g")
+    _expect(beta, (N, H_v), "beta", g.dtype)
+    _expect(state, (P, H_v, HEAD_DIM, HEAD_DIM), "state", torch.float32)
+    _expect(state_idx, (N,), "state_idx", torch.int32)
+    _expect(z, (N, H_v, HEAD_DIM), "z", x.dtype)
+    _expect(norm_w, (HEAD_DIM,), "norm_w", conv_w.dtype)
+    _expect(y, (N, H_v, HEAD_DIM), "y")
+    if y is None:
+        y = torch.empty((N, H_v, HEAD_DIM), dtype=y_dtype or x.dtype, device=x.device)
+    _check("gdn_decode_layer_step", load().gdn_decode_layer_step(
+        _ptr(x), _row_stride(x), _dtype_code(x.dtype), _ptr(conv_w), _dtype_code(conv_w.dtype),
+        _ptr(conv_bias), _ptr(conv_state), _ptr(g), _ptr(beta), _dtype_code(g.dtype),
+        _ptr(state), _ptr(state_idx), N, P, H_k, H_v, scale, l2_eps, _ptr(z), _ptr(norm_w),
+        norm_eps, _ptr(y), _dtype_code(y.dtype), _stream(stream, x.device)))
+    return y
 
 
 def gdn_gated_rmsnorm(x, z, w, *, eps=1e-6, y=None, y_dtype=None, stream=None):

@@ -229,6 +229,40 @@ gdn_status gdn_decode_step(const void* q, const void* k, const void* v,
   return from_cuda(gdn::launch_decode_step(a));
 }
 
+gdn_status gdn_decode_layer_step(const void* x, int64_t x_row_stride, gdn_dtype x_dtype,
+                                 const void* conv_w, gdn_dtype w_dtype,
+                                 const void* conv_bias, void* conv_state,
+                                 const void* g, const void* beta, gdn_dtype gate_dtype,
+                                 float* state, const int32_t* state_idx, int N, int P,
+                                 int H_k, int H_v, float scale, float l2_eps,
+                                 const void* z, const void* norm_w, float norm_eps,
+                                 void* y, gdn_dtype y_dtype, cudaStream_t stream) {
+  if (!valid_dtype(x_dtype) || !valid_dtype(w_dtype) || !valid_dtype(gate_dtype) ||
+      !valid_dtype(y_dtype))
+    return GDN_ERR_INVALID_ARG;
+  if (N < 0 || P < 0 || H_k <= 0 || H_v <= 0 || H_v % H_k != 0 || !(l2_eps >= 0.f) ||
+      !(norm_eps >= 0.f))
+    return GDN_ERR_INVALID_ARG;
+  if (H_v / H_k > 8) return GDN_ERR_UNSUPPORTED;
+  const int64_t C = 2 * (int64_t)H_k * kHeadDim + (int64_t)H_v * kHeadDim;
+  if (x_row_stride < C) return GDN_ERR_INVALID_ARG;
+  if (N == 0) return GDN_OK;
+  if (P == 0 || !x || !conv_w || !conv_state || !g || !beta || !state || !state_idx || !z ||
+      !norm_w || !y)
+    return GDN_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(conv_w) || (conv_bias && !aligned16(conv_bias)) ||
+      !aligned16(conv_state) || !aligned16(state) || !aligned16(z) || !aligned16(norm_w) ||
+      !aligned16(y) || !aligned_to(state_idx, 4))
+    return GDN_ERR_MISALIGNED;
+  if (!stride_ok(x_row_stride, x_dtype)) return GDN_ERR_MISALIGNED;
+  const int gb = gdn::elem_bytes(gate_dtype);
+  if (!aligned_to(g, gb) || !aligned_to(beta, gb)) return GDN_ERR_MISALIGNED;
+  gdn::DecodeLayerArgs a{x, x_row_stride, x_dtype, conv_w, w_dtype, conv_bias, conv_state,
+                         g, beta, gate_dtype, state, state_idx, N, P, H_k, H_v, scale,
+                         l2_eps, z, norm_w, norm_eps, y, y_dtype, stream};
+  return from_cuda(gdn::launch_decode_layer(a));
+}
+
 gdn_status gdn_gated_rmsnorm(const void* x, gdn_dtype x_dtype, const void* z,
                              gdn_dtype z_dtype, const void* w,
                              gdn_dtype w_dtype, int64_t rows, int dim,

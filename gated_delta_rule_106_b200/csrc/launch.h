@@ -32,6 +32,22 @@ struct RecurArgs {
   cudaStream_t stream;
 };
 
+// Fused decode step of the layer (conv roll + SiLU + q/k L2, recurrence on a
+// pooled state, gated RMS-norm). x, the conv cache and z share x_dtype; the
+// conv weights, bias and norm weight share w_dtype.
+struct DecodeLayerArgs {
+  const void* x; int64_t x_row_stride; gdn_dtype x_dtype;
+  const void* conv_w; gdn_dtype w_dtype; const void* conv_bias;
+  void* conv_state;                  // [P, 3, C] pool
+  const void* g; const void* beta; gdn_dtype gate_dtype;
+  float* state;                      // [P, H_v, 128, 128] pool
+  const int32_t* state_idx;          // [N] slots (device)
+  int N; int P; int H_k; int H_v; float scale; float l2_eps;
+  const void* z; const void* norm_w; float norm_eps;
+  void* y; gdn_dtype y_dtype;
+  cudaStream_t stream;
+};
+
 struct NormArgs {
   const void* x; gdn_dtype x_dtype; const void* z; gdn_dtype z_dtype;
   const void* w; gdn_dtype w_dtype; int64_t rows; int dim; float eps;
@@ -41,6 +57,7 @@ struct NormArgs {
 cudaError_t launch_conv1d_silu(const ConvArgs& a);
 cudaError_t launch_gated_rmsnorm(const NormArgs& a);
 cudaError_t launch_decode_step(const RecurArgs& a);
+cudaError_t launch_decode_layer(const DecodeLayerArgs& a);
 // Stepwise fp32 recurrence on the CUDA cores (any input dtype).
 cudaError_t launch_prefill_stepwise(const RecurArgs& a);
 // Chunk-64 recurrence on the CUDA cores in fp32 (fp32 inputs; any input dtype).

@@ -229,6 +229,52 @@ gdn_status gdn_decode_step(const void* q, const void* k, const void* v,
                            cudaStream_t stream);
 
 /*
+ * gdn_decode_layer_step -- one decode token of the whole delta-rule layer for
+ * N sequences in one launch: the causal conv (kernel 4) over the conv cache
+ * with the cache rolled in place, SiLU and the per-head L2 norm of q and k, the
+ * stepwise gated delta rule on the sequence's fp32 state, and the gated
+ * RMS-norm of the output (the stepwise decode path of [P2 二.1]; conv k=4,
+ * gated RMS-norm and fp32 state: [P3 架构]). The result equals
+ * gdn_conv1d_silu -> gdn_decode_step -> gdn_gated_rmsnorm except that q, k, v
+ * stay in fp32 between the stages (they are not stored in x_dtype).
+ * Additional entry point (fused form of the three calls, for serving).
+ *
+ * States and conv caches live in pools indexed by a slot per sequence, as a
+ * server keeps them:
+ *   x           [N, C] x_dtype, row stride x_row_stride: the new token's
+ *               pre-conv channels q | k | v, C = 2*H_k*128 + H_v*128.
+ *   conv_w      [C, 4] w_dtype (tap 3 = current token); conv_bias [C] w_dtype
+ *               or NULL.
+ *   conv_state  [P, 3, C] x_dtype pool, oldest row first; slot state_idx[n]
+ *               is read and rolled in place (its rows become h1, h2, x_n).
+ *   g, beta     [N, H_v] gate_dtype.
+ *   state       [P, H_v, 128, 128] fp32 pool; slot state_idx[n] is updated in
+ *               place.
+ *   state_idx   [N] int32 (device): the pool slot of sequence n, the same in
+ *               both pools. Slots of different sequences must differ. A slot
+ *               outside [0, P) marks padding: nothing of it is read or
+ *               written except its output rows, which are set to 0.
+ *   scale       multiplies o (1.0 for the plain rule); l2_eps: the q/k norm's
+ *               epsilon, y / sqrt(sum y^2 + l2_eps).
+ *   z           [N, H_v, 128] x_dtype, the output gate; norm_w [128] w_dtype;
+ *               norm_eps: out = o / sqrt(mean(o^2) + norm_eps) * norm_w * SiLU(z).
+ *   y           [N, H_v, 128] contiguous, y_dtype: the normed output.
+ * Two launches on `stream`: the layer kernel (one CTA per sequence and value
+ * head; each computes q and k of its key head itself and rolls its own v
+ * cache rows) and a small kernel that then rolls the q/k cache rows, which
+ * every value head of a key head reads. H_v / H_k must be at most 8, else
+ * GDN_ERR_UNSUPPORTED. N == 0 is valid.
+ */
+gdn_status gdn_decode_layer_step(const void* x, int64_t x_row_stride, gdn_dtype x_dtype,
+                                 const void* conv_w, gdn_dtype w_dtype,
+                                 const void* conv_bias, void* conv_state,
+                                 const void* g, const void* beta, gdn_dtype gate_dtype,
+                                 float* state, const int32_t* state_idx, int N, int P,
+                                 int H_k, int H_v, float scale, float l2_eps,
+                                 const void* z, const void* norm_w, float norm_eps,
+                                 void* y, gdn_dtype y_dtype, cudaStream_t stream);
+
+/*
  * gdn_gated_rmsnorm -- gated RMS-norm on the layer output ([P3 架构]):
  *   y = x / sqrt(mean(x^2) + eps) * w * SiLU(z)
  * over rows of `dim` channels (one row per token and value head).

@@ -235,3 +235,54 @@ def test_binding_refuses_mixed_dtypes(lib):
                             bias=torch.zeros(256, dtype=torch.bfloat16))
     with pytest.raises(ValueError, match="cu_seqlens: dtype"):
         gdn.gdn_conv1d_silu(x, torch.ones(256, 4), cu.long())
+
+
+def decode_layer(lib, **kw):
+    a = dict(x=A, xs=10240, xdt=BF16, w=A, wdt=F32, bias=None, cache=A, g=A, beta=A,
+             gdt=F32, state=A, idx=A, N=4, P=8, H_k=16, H_v=48, scale=1.0, l2_eps=1e-6,
+             z=A, nw=A, norm_eps=1e-6, y=A, ydt=BF16, s=None)
+    a.update(kw)
+    return lib.gdn_decode_layer_step(*a.values())
+
+
+def test_decode_layer_validation(lib):
+    assert decode_layer(lib, N=-1) == INVALID
+    assert decode_layer(lib, H_v=47) == INVALID            # H_v % H_k
+    assert decode_layer(lib, H_k=4, H_v=48, xs=7168) == UNSUPPORTED  # 12 per key head
+    assert decode_layer(lib, xs=10239) == INVALID           # stride below C = 10240
+    assert decode_layer(lib, P=0) == INVALID
+    assert decode_layer(lib, idx=None) == INVALID
+    assert decode_layer(lib, z=None) == INVALID
+    assert decode_layer(lib, x=A + 2) == MISALIGNED
+    assert decode_layer(lib, state=A + 8) == MISALIGNED
+    assert decode_layer(lib, idx=A + 2) == MISALIGNED
+    assert decode_layer(lib, xs=10244) == MISALIGNED        # 20488 bytes, not 16-aligned
+    assert decode_layer(lib, l2_eps=-1.0) == INVALID
+    assert decode_layer(lib, xdt=7) == INVALID
+    assert decode_layer(lib, N=0) == OK
+
+
+def test_decode_layer_binding_checks(lib):
+    import torch
+    N, P = 2, 3
+    x = torch.zeros(N, 10240, dtype=torch.bfloat16)
+    w = torch.zeros(10240, 4)
+    cache = torch.zeros(P, 3, 10240, dtype=torch.bfloat16)
+    g = torch.ones(N, 48)
+    S = torch.zeros(P, 48, 128, 128)
+    idx = torch.zeros(N, dtype=torch.int32)
+    z = torch.zeros(N, 48, 128, dtype=torch.bfloat16)
+    nw = torch.ones(128)
+    call = lambda **kw: gdn.gdn_decode_layer_step(
+        kw.get("x", x), w, kw.get("cache", cache), g, g, S, kw.get("idx", idx),
+        kw.get("z", z), kw.get("nw", nw))
+    with pytest.raises(ValueError, match="channels"):
+        call(x=torch.zeros(N, 10112, dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="conv_state: dtype"):
+        call(cache=cache.float())
+    with pytest.raises(ValueError, match="state_idx: dtype"):
+        call(idx=idx.long())
+    with pytest.raises(ValueError, match="z: dtype"):
+        call(z=z.float())
+    with pytest.raises(ValueError, match="norm_w: dtype"):
+        call(nw=nw.bfloat16())
