@@ -10,16 +10,17 @@
 //                M_ts = e^{G_t-G_s} q_t.k_s (s<=t)
 //   state chain: Delta = U - W S0^T
 //                O     = scale (diag(e^G) Q S0^T + M Delta)
-//                S_L   = e^{G_L} S0 + Delta^T diag(e^{G_L-G}) K
+//                S_L   = e^{G_L} S0 + (diag(e^{G_L-G}) Delta)^T K
 //
 // One cooperative launch, one CTA per SM, two roles:
 //  * state CTAs (about a third of the SMs) each own a list of (sequence,
 //    value head) items and run their chunks in order. Per chunk: D1 = S0
 //    [-W ; Q~]^T (N = 128: the S0 part of Delta and S0 q~ per token together,
-//    Q~ = diag(e^G) Q), the Delta readout, then P = Delta_hi^T K~ (the state
-//    update, K~ = diag(e^{G_L-G}) K) and the M Delta products, which accumulate
-//    onto S0 q~ in TMEM; the fp32 state stays in registers (four threads per
-//    row). Few wide MMAs matter because each tcgen05.mma instruction costs
+//    Q~ = diag(e^G) Q), the Delta readout, then P = Delta'^T K (the state
+//    update with Delta' = diag(e^{G_L-G}) Delta as binary16 high and low parts
+//    against the exact binary16 image of the bf16 keys) and the M Delta
+//    products, which accumulate onto S0 q~ in TMEM; the fp32 state stays in
+//    registers (four threads per row). Few wide MMAs matter because each tcgen05.mma instruction costs
 //    about the same time whether N is 64 or 128. A chunk's outputs are read
 //    during the next chunk and leave as one TMA tensor store.
 //  * prep CTAs run two independent 256-thread pipelines each; a pipeline claims
@@ -28,8 +29,8 @@
 //    tensor cores (bf16, exact products: K K^T for A, Q K^T for M); decays; the
 //    UT solve in fp32; W and U as bf16 hi/lo MMAs (~17 significant bits, unit
 //    diagonal included); it writes binary16 images of [-W ; Q~] and
-//    [K~ | M hi | M lo] and U in fp32 straight into a ring slot in the caller's
-//    workspace (6 slots per state CTA, ~97 KB each, L2-resident) and releases
+//    [K | M hi | M lo], U in fp32 and the chunk's decays straight into a ring
+//    slot in the caller's workspace (6 slots per state CTA, ~97 KB each, L2-resident) and releases
 //    its flag; the state CTA acquires it, bulk-copies the operand images into
 //    shared memory and releases the slot once read.
 // Deadlock freedom: all CTAs are co-resident (cooperative launch); a prep CTA
@@ -59,17 +60,19 @@ constexpr uint64_t kLimitNs = 2000000000ull;
 // B operand of S0 [-W ; Q~]^T: K-major, [2 d_k blocks][128 rows][64], rows 0-63 = -W
 // (token t), rows 64-127 = Q~ = diag(e^G) Q (token t), binary16.
 constexpr uint32_t SL_WQ = 0;
-// Four 8 KB blocks: K~ = diag(e^{G_L-G}) K, MN-major [64 tokens s][64 d_k] (d_k 0-63,
-// 64-127; the B operand of P = Delta^T K~), then the lower triangle of M
+// Four 8 KB blocks: K, MN-major [64 tokens s][64 d_k] (d_k 0-63, 64-127; the B
+// operand of P = Delta'^T K; bf16 keys are exact in binary16), then the lower triangle of M
 // (M[t][s] = M_ts for s <= t) as binary16 high and low parts, K-major [64 t][64 s]
 // (the B operands of the M Delta products).
 constexpr uint32_t SL_BKM = 32768;
-constexpr uint32_t SL_VEC = 65536;     // gL (the chunk's total decay)
-constexpr uint32_t SL_IMG = 66560;     // bytes of the shared-memory image above
+constexpr uint32_t SL_OPS = 65536;     // bytes of the operand images above
+// fp32 [0] = e^{G_L} (the chunk's total decay), [1 + t] = e^{G_L - G_t}
+constexpr uint32_t SL_VEC = 65536;
+constexpr uint32_t SL_VEC_BYTES = 272;  // 65 floats, rounded up to 16 bytes
 constexpr uint32_t SL_UT = 66560;      // U fp32 [64 t][128 i] (copied to shared memory separately)
 constexpr uint32_t SLOT_BYTES = 99328;
 // state CTA use of a slot image buffer once its MMAs are done: the [-W ; Q~] area
-// stages that step's outputs (o's dtype), the K~/M area receives the next step's U
+// stages that step's outputs (o's dtype), the K/M area receives the next step's U
 constexpr uint32_t S_STG_OFF = SL_WQ, S_UT_OFF = SL_BKM;
 
 constexpr uint32_t CTRL_BYTES = 16384; // counter, abort word, per-state-CTA flags
@@ -89,13 +92,17 @@ constexpr uint32_t PP_TF = 66560;      // fp32 T [64][kLd]
 constexpr uint32_t PP_T2 = 83968;      // bf16 T'' hi | lo [64][64] each
 constexpr uint32_t P_SMALL = 2 * PIPE_BYTES;
 // ---- state CTA shared memory --------------------------------------------
-constexpr uint32_t S_BUF = 0;          // 2 x slot image
-constexpr uint32_t S_S0 = 133120;      // binary16 state, K-major [2 blocks][128 rows]
-constexpr uint32_t S_DTH = 165888;     // Delta^T high, K-major A [128 d_v][64 t]
-constexpr uint32_t S_DTL = 182272;     // Delta^T low
-constexpr uint32_t S_SMALL = 215040;
+constexpr uint32_t S_BUF = 0;          // 2 x slot operand images (SL_OPS each)
+constexpr uint32_t S_VEC = 131072;     // 2 x slot decay vectors (512 bytes each)
+constexpr uint32_t S_S0 = 132096;      // binary16 state, K-major [2 blocks][128 rows]
+constexpr uint32_t S_DTH = 164864;     // Delta^T high, K-major A [128 d_v][64 t]
+constexpr uint32_t S_DTL = 181248;     // Delta^T low
+constexpr uint32_t S_DPH = 197632;     // Delta'^T high, Delta' = diag(e^{G_L-G}) Delta
+constexpr uint32_t S_DPL = 214016;     // Delta'^T low
+constexpr uint32_t S_SMALL = 230400;
 constexpr uint32_t PC_SMEM_BYTES = S_SMALL + 1024;   // the state role needs the most
-constexpr uint32_t PC_SMEM_ALLOC = PC_SMEM_BYTES + 1024;
+constexpr uint32_t PC_SMEM_ALLOC = PC_SMEM_BYTES + 1024;   // 227 KB: the sm_100 limit
+static_assert(PC_SMEM_ALLOC <= 232448, "over the shared memory of a CTA");
 
 // TMEM columns
 // prep, per pipeline (256 columns each): Gram [128 x 64] at 0, then W^T as
@@ -103,7 +110,7 @@ constexpr uint32_t PC_SMEM_ALLOC = PC_SMEM_BYTES + 1024;
 constexpr uint32_t PT_GR = 0, PT_W = 0, PT_U = 128, PT_PIPE = 256, PT_COLS = 512;
 // state: D1 = S0 [-W ; Q~]^T -> [Delta^T - U^T | OA = S0 Q~^T], in one of two column
 //        sets by step parity (a step's outputs outlive the next step's D1), and
-//        Delta_lo^T M_hi^T accumulated onto OA;  P = Delta_hi^T K~;
+//        Delta_lo^T M_hi^T accumulated onto OA;  P = Delta'^T K (hi and lo parts);
 //        OB = Delta_hi^T [M hi ; M lo]^T -> [OB_hh | OB_hl] (M with its diagonal).
 //        o^T = scale (OA + OB_hh + OB_hl)
 constexpr uint32_t ST_D1A = 0, ST_P = 128, ST_D1B = 256, ST_OB = 384, ST_COLS = 512;
@@ -489,15 +496,15 @@ __device__ void prep_role(const PcParams& p, const CUtensorMap* tm_q, const CUte
       }
       mma_commit(&ss.bar_mma);
     }
-    // meanwhile: binary16 images of K~ = diag(tail) K and Q~ = diag(gamma) Q, straight
-    // to the slot
+    // meanwhile: binary16 images of K (exact: bf16 values) and Q~ = diag(gamma) Q,
+    // straight to the slot
 #pragma unroll 2
     for (int idx = ptid; idx < 2048; idx += kPipeThreads) {
       const int which = idx >> 10, b = (idx >> 9) & 1, x = idx & 511;
       const uint8_t* src = kq + b * 16384 + which * 8192 + x * 16;
       float f[8];
       load8(reinterpret_cast<const __nv_bfloat16*>(src), f);
-      const float sc = which == 0 ? ss.tail[x >> 3] : ss.gamma[x >> 3];
+      const float sc = which == 0 ? 1.f : ss.gamma[x >> 3];
 #pragma unroll
       for (int u = 0; u < 8; ++u) f[u] *= sc;
       uint8_t* dst = which == 0 ? slot + SL_BKM + b * 8192 + x * 16
@@ -663,6 +670,7 @@ __device__ void prep_role(const PcParams& p, const CUtensorMap* tm_q, const CUte
       }
       float* vec = reinterpret_cast<float*>(slot + SL_VEC);
       if (ptid == 0) vec[0] = ss.gL;
+      if (ptid < kChunk) vec[1 + ptid] = ss.tail[ptid];
     }
     fence_proxy_async_all();   // the state CTA reads the slot with a bulk copy
     tc_fence_before();
@@ -720,6 +728,7 @@ __device__ void state_role(const PcParams& p, const CUtensorMap* tm_o, uint8_t* 
   const int total = steps_of(p, p.cu, s);
   const uint32_t a_s0 = smem_u32(sm + S_S0), a_dth = smem_u32(sm + S_DTH);
   const uint32_t a_dtl = smem_u32(sm + S_DTL);
+  const uint32_t a_dph = smem_u32(sm + S_DPH), a_dpl = smem_u32(sm + S_DPL);
   const uint32_t id_d1 = idesc_f16(128, 128, false, false);
   const uint32_t id_p = idesc_f16(128, 128, false, true);
   const uint32_t id_ob = idesc_f16(128, 128, false, false);
@@ -738,16 +747,18 @@ __device__ void state_role(const PcParams& p, const CUtensorMap* tm_o, uint8_t* 
     fence_proxy_async_all();
     bulk_wait_read_all();   // an output store of this thread may still read the buffer
     uint64_t* bar = &ss.bar_slot[step & 1];
-    mbar_arrive_expect_tx(bar, SL_IMG);
-    bulk_g2s(sm + S_BUF + (step & 1) * SL_IMG, slot_of(p.ws, s, step), SL_IMG, bar);
+    uint8_t* src = slot_of(p.ws, s, step);
+    mbar_arrive_expect_tx(bar, SL_OPS + SL_VEC_BYTES);
+    bulk_g2s(sm + S_BUF + (step & 1) * SL_OPS, src, SL_OPS, bar);
+    bulk_g2s(sm + S_VEC + (step & 1) * 512, src + SL_VEC, SL_VEC_BYTES, bar);
     return true;
   };
-  // U^T of `step` goes to the other buffer's K~/M area, free once step-1's output
+  // U^T of `step` goes to the other buffer's K/M area, free once step-1's output
   // MMAs are done (the caller has acquired the slot and fenced the async proxy)
   auto issue_ut = [&](int step) {
     const int ub = (step + 1) & 1;
     mbar_arrive_expect_tx(&ss.bar_ut[ub], 32768);
-    bulk_g2s(sm + S_BUF + ub * SL_IMG + S_UT_OFF, slot_of(p.ws, s, step) + SL_UT, 32768,
+    bulk_g2s(sm + S_BUF + ub * SL_OPS + S_UT_OFF, slot_of(p.ws, s, step) + SL_UT, 32768,
              &ss.bar_ut[ub]);
   };
   // staged outputs of an earlier step (o's dtype, [64 t][128 rows] over a buffer's
@@ -827,7 +838,7 @@ __device__ void state_role(const PcParams& p, const CUtensorMap* tm_o, uint8_t* 
 
     for (int c = 0; c < nch; ++c, ++r) {
       const int b = r & 1;
-      uint8_t* buf = sm + S_BUF + b * SL_IMG;
+      uint8_t* buf = sm + S_BUF + b * SL_OPS;
       const uint32_t a_buf = smem_u32(buf);
       const int64_t t0 = s0 + (int64_t)c * kChunk;
       const int L = (int)((s1 - t0) < kChunk ? (s1 - t0) : kChunk);
@@ -844,7 +855,7 @@ __device__ void state_role(const PcParams& p, const CUtensorMap* tm_o, uint8_t* 
       }
       __syncthreads();
       if (!ss.ok) { ok = false; break; }
-      uint8_t* ubuf = sm + S_BUF + ((r + 1) & 1) * SL_IMG;   // U^T of step r
+      uint8_t* ubuf = sm + S_BUF + ((r + 1) & 1) * SL_OPS;   // U^T of step r
       const uint32_t d1 = (r & 1) ? ST_D1B : ST_D1A;
       const uint32_t ut_par = (uint32_t)((r >> 1) & 1);        // step r is its r>>1-th use
       if (!mbar_wait_bounded(&ss.bar_slot[b], (uint32_t)((r >> 1) & 1), kLimitNs)) ok = false;
@@ -882,8 +893,9 @@ __device__ void state_role(const PcParams& p, const CUtensorMap* tm_o, uint8_t* 
       if (!mbar_wait_bounded(&ss.bar_dt, par_dt, kLimitNs)) ok = false;
       par_dt ^= 1;
       tc_fence_after();
-      // ---- Delta = U - W S0^T as binary16 high and low parts ----
-      const float* vec = reinterpret_cast<const float*>(buf + SL_VEC);
+      // ---- Delta = U - W S0^T (for the outputs) and Delta' = diag(e^{G_L-G})
+      //      Delta (for the state update), each as binary16 high and low parts ----
+      const float* vec = reinterpret_cast<const float*>(sm + S_VEC + b * 512);
       {
         float v[16], d[16];
         tmem_ld16(tmem + lane_base + d1 + 16 * cg, v);
@@ -897,20 +909,34 @@ __device__ void state_role(const PcParams& p, const CUtensorMap* tm_o, uint8_t* 
           *reinterpret_cast<uint4*>(sm + S_DTH + swz(row, 2 * cg + q)) = hi;
           *reinterpret_cast<uint4*>(sm + S_DTL + swz(row, 2 * cg + q)) = lo;
         }
+#pragma unroll
+        for (int j = 0; j < 16; ++j) d[j] *= vec[1 + 16 * cg + j];
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          uint4 hi, lo;
+          split_half8(d + 8 * q, hi, lo);
+          *reinterpret_cast<uint4*>(sm + S_DPH + swz(row, 2 * cg + q)) = hi;
+          *reinterpret_cast<uint4*>(sm + S_DPL + swz(row, 2 * cg + q)) = lo;
+        }
       }
       // stage step r-1's outputs over this step's [-W ; Q~] image (D1 is done)
       if (pend) stage_out(buf, ov);
       fence_proxy_async_smem();
       tc_fence_before();
       if (__syncthreads_or(!ok)) { ok = false; break; }
-      // ---- P = Delta_hi^T K~ (critical path), then Delta_hi^T [M hi ; M lo]^T and
-      //      Delta_lo^T M_hi^T (onto OA) for the output, read during the next step ----
+      // ---- P = Delta'_hi^T K + Delta'_lo^T K (critical path), then Delta_hi^T
+      //      [M hi ; M lo]^T and Delta_lo^T M_hi^T (onto OA) for the output, read
+      //      during the next step ----
       if (tid == 0) {
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
-          mma_f16(tmem + ST_P, sw128_desc(a_dth + ks * 32, 16, 1024),
+          mma_f16(tmem + ST_P, sw128_desc(a_dph + ks * 32, 16, 1024),
                   sw128_desc(a_buf + SL_BKM + ks * 2048, 8192, 1024), id_p, ks > 0);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          mma_f16(tmem + ST_P, sw128_desc(a_dpl + ks * 32, 16, 1024),
+                  sw128_desc(a_buf + SL_BKM + ks * 2048, 8192, 1024), id_p, 1);
         mma_commit(&ss.bar_p);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
@@ -949,7 +975,7 @@ __device__ void state_role(const PcParams& p, const CUtensorMap* tm_o, uint8_t* 
       if (!mbar_wait_bounded(&ss.bar_o, par_o, kLimitNs)) ok = false;
       par_o ^= 1;
       tc_fence_after();
-      // step r+1's U^T into this buffer's K~/M area, which the output MMAs have
+      // step r+1's U^T into this buffer's K/M area, which the output MMAs have
       // finished reading
       if (tid == 32 && issued == r + 2 && ut_issued == r + 1) {
         issue_ut(r + 1);
@@ -975,7 +1001,7 @@ __device__ void state_role(const PcParams& p, const CUtensorMap* tm_o, uint8_t* 
     float ov[16];
     tc_fence_after();
     load_out(((r - 1) & 1) ? ST_D1B : ST_D1A, ov);
-    uint8_t* lbuf = sm + S_BUF + ((r - 1) & 1) * SL_IMG;
+    uint8_t* lbuf = sm + S_BUF + ((r - 1) & 1) * SL_OPS;
     stage_out(lbuf, ov);
     fence_proxy_async_smem();
     __syncthreads();
