@@ -24,12 +24,14 @@ __all__ = ["GDN_BF16", "GDN_F32", "GdnError", "library_path", "load",
            "gdn_conv1d_silu", "gdn_chunked_prefill",
            "gdn_chunked_prefill_workspace", "gdn_chunked_prefill_noalloc",
            "gdn_stepwise_prefill", "gdn_decode_layer_step",
+           "gdn_chunked_prefill_status", "gdn_set_wait_limit_ns", "GDN_ERR_TIMEOUT",
            "gdn_decode_step",
            "gdn_gated_rmsnorm", "gdn_status_string", "gdn_version",
            "H_K", "H_V", "HEAD_DIM", "CHUNK"]
 
 GDN_BF16 = 0
 GDN_F32 = 1
+GDN_ERR_TIMEOUT = -5
 H_K, H_V, HEAD_DIM, CHUNK = 16, 48, 128, 64
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -53,6 +55,8 @@ _SIGNATURES = {
                                    _int, _f32, _vp, _int, _vp, ctypes.c_size_t,
                                    _vp]),
     "gdn_chunked_prefill_workspace": (ctypes.c_size_t, [_int, _i64, _int, _int]),
+    "gdn_chunked_prefill_status": (_int, [_vp, _vp]),
+    "gdn_set_wait_limit_ns": (None, [ctypes.c_uint64]),
     "gdn_stepwise_prefill": (_int, [_vp, _vp, _vp, _int, _i64, _i64, _i64, _vp,
                                     _vp, _int, _vp, _vp, _vp, _int, _i64, _int,
                                     _int, _f32, _vp, _int, _vp]),
@@ -227,6 +231,21 @@ def gdn_chunked_prefill(q, k, v, g, beta, cu_seqlens, *, state_in=None,
         scale, _ptr(o), _dtype_code(o.dtype), _ptr(workspace), ws_bytes,
         _stream(stream, v.device)))
     return o
+
+
+def gdn_chunked_prefill_status(workspace=None, stream=None) -> int:
+    """Waits for `stream`, then returns 0 if the last gdn_chunked_prefill that
+    worked in `workspace` (None: the no-alloc call's own array) completed, or
+    GDN_ERR_TIMEOUT if a bounded wait inside it gave up (its unfinished outputs
+    are NaN). Not for the hot path: it synchronises."""
+    dev = workspace.device if workspace is not None else torch.device("cuda")
+    return int(load().gdn_chunked_prefill_status(_ptr(workspace), _stream(stream, dev)))
+
+
+def gdn_set_wait_limit_ns(ns: int) -> None:
+    """Bound (ns) on each wait of the chunked prefill kernel for another CTA's
+    flag; 0 restores the default (2 s). Process-wide."""
+    load().gdn_set_wait_limit_ns(int(ns))
 
 
 def gdn_stepwise_prefill(q, k, v, g, beta, cu_seqlens, *, state_in=None,

@@ -64,6 +64,7 @@ const char* gdn_status_string(gdn_status s) {
     case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED: unsupported shape or option";
     case GDN_ERR_MISALIGNED: return "GDN_ERR_MISALIGNED: pointer or stride not 16-byte aligned";
     case GDN_ERR_CUDA: return "GDN_ERR_CUDA: CUDA launch failed";
+    case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT: a bounded wait in a kernel gave up";
   }
   return "unknown gdn_status";
 }
@@ -147,6 +148,15 @@ gdn_status gdn_chunked_prefill(const void* q, const void* k, const void* v,
   return from_cuda(qkv_dtype == GDN_BF16 ? gdn::launch_prefill_pc(a)
                                          : gdn::launch_prefill_chunked_f32(a));
 }
+
+gdn_status gdn_chunked_prefill_status(const void* workspace, cudaStream_t stream) {
+  if (workspace && !aligned16(workspace)) return GDN_ERR_MISALIGNED;
+  int word = 0;
+  if (gdn::prefill_abort_word(workspace, stream, &word) != cudaSuccess) return GDN_ERR_CUDA;
+  return word ? GDN_ERR_TIMEOUT : GDN_OK;
+}
+
+void gdn_set_wait_limit_ns(uint64_t ns) { gdn::set_wait_limit_ns(ns); }
 
 gdn_status gdn_stepwise_prefill(const void* q, const void* k, const void* v,
                                 gdn_dtype qkv_dtype, int64_t q_row_stride,

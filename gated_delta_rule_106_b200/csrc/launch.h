@@ -69,5 +69,11 @@ size_t prefill_pc_workspace(int N, int64_t T_total, int H_v);
 // The same kernel on the library-owned static scratch (no workspace argument).
 cudaError_t launch_prefill_pc_noalloc(const RecurArgs& a);
 size_t prefill_noalloc_scratch_bytes();
+// Limit of the chunk kernel's waits on another CTA's flag (0 restores 2 s).
+void set_wait_limit_ns(uint64_t ns);
+uint64_t wait_limit_ns();
+// Synchronises `stream`, then reads the abort word of the workspace (NULL: the
+// library-owned scratch) that the last chunk-kernel call on it left.
+cudaError_t prefill_abort_word(const void* workspace, cudaStream_t stream, int* word);
 
 }  // namespace gdn

@@ -36,11 +36,17 @@
 // Deadlock freedom: all CTAs are co-resident (cooperative launch); a prep CTA
 // works on claims in increasing order and a claim only waits on the
 // consumption of an earlier step of the same state CTA. Every wait is
-// bounded (2 s); on a timeout the CTA raises a global abort word, every CTA
-// leaves its loops, and the outputs of unfinished items are left NaN-marked.
+// bounded: waits on another CTA's flag by a settable limit (2 s unless
+// gdn_set_wait_limit_ns changed it), waits on this CTA's own copies and MMAs
+// by 2 s. On a timeout the CTA raises the abort word in the workspace, every
+// CTA leaves its loops, waits for its own copies in flight and frees its
+// tensor memory; a state CTA then writes NaN to the outputs (o and state_out)
+// of every (sequence, head) it did not finish. gdn_chunked_prefill_status
+// reads the abort word.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "gdn_common.cuh"
@@ -54,7 +60,7 @@ using namespace sm100;
 
 constexpr int kPcThreads = 512;
 constexpr int kRing = 6;            // slots per state CTA: how far prep may run ahead
-constexpr uint64_t kLimitNs = 2000000000ull;
+constexpr uint64_t kLimitNs = 2000000000ull;   // own copies and MMAs; default for flags
 
 // ---- ring slot (global), 1024-aligned sections ---------------------------
 // B operand of S0 [-W ; Q~]^T: K-major, [2 d_k blocks][128 rows][64], rows 0-63 = -W
@@ -122,6 +128,7 @@ struct PcParams {
   void* o;
   uint8_t* ws;          // workspace base
   int NS;               // state CTAs
+  uint64_t wait_ns;     // limit of a wait on another CTA's flag
 };
 
 constexpr int kCuCache = 513;   // sequences whose boundaries the prep CTAs keep on chip
@@ -427,7 +434,7 @@ __device__ void prep_role(const PcParams& p, const CUtensorMap* tm_q, const CUte
 
     // the slot is written directly: wait until step r - kRing has been consumed
     if (ptid == 0)
-      ss.ok = wait_flag_ge(flags_of(p.ws, s) + kRing, r + 1 - kRing, &ctrl[1], kLimitNs);
+      ss.ok = wait_flag_ge(flags_of(p.ws, s) + kRing, r + 1 - kRing, &ctrl[1], p.wait_ns);
     if (warp == 1) {   // gates: cumulative log-decay and derived vectors
       const Tg* g = static_cast<const Tg*>(p.g);
       const Tg* bt = static_cast<const Tg*>(p.beta);
@@ -743,7 +750,7 @@ __device__ void state_role(const PcParams& p, const CUtensorMap* tm_o, uint8_t* 
   // wait (bounded) for the producer's release of that slot.
   auto issue_copy = [&](int step, bool acquired) -> bool {
     int* full = flags + (step % kRing);
-    if (!acquired && !wait_flag_ge(full, step + 1, &ctrl[1], kLimitNs)) return false;
+    if (!acquired && !wait_flag_ge(full, step + 1, &ctrl[1], p.wait_ns)) return false;
     fence_proxy_async_all();
     bulk_wait_read_all();   // an output store of this thread may still read the buffer
     uint64_t* bar = &ss.bar_slot[step & 1];
@@ -814,6 +821,7 @@ __device__ void state_role(const PcParams& p, const CUtensorMap* tm_o, uint8_t* 
   bool pend = false;              // a step's outputs wait in TMEM
   int64_t pend_t0 = 0;
   int pend_L = 0, pend_h = 0;
+  int fail_item = -1;             // the item being worked on when a wait gave up
 
   for (int i = s; i < p.N * p.H_v && ok; i += p.NS) {
     const int n = i / p.H_v, h = i % p.H_v;
@@ -988,13 +996,15 @@ __device__ void state_role(const PcParams& p, const CUtensorMap* tm_o, uint8_t* 
       pend_L = L;
       pend_h = h;
     }
+    if (!ok) {
+      fail_item = i;
+      break;
+    }
     if (p.state_out) {
       float* dst = p.state_out + (nh * kHeadDim + row) * kHeadDim + cg * 32;
-      const float qnan = __int_as_float(0x7fc00000);
 #pragma unroll
       for (int j = 0; j < 32; j += 4)
-        *reinterpret_cast<float4*>(dst + j) =
-            ok ? make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]) : make_float4(qnan, qnan, qnan, qnan);
+        *reinterpret_cast<float4*>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
     }
   }
   if (ok && pend) {   // the last step's outputs
@@ -1015,9 +1025,23 @@ __device__ void state_role(const PcParams& p, const CUtensorMap* tm_o, uint8_t* 
     for (int st = r; st < ut_issued; ++st)
       mbar_wait_bounded(&ss.bar_ut[(st + 1) & 1], (uint32_t)((st >> 1) & 1), kLimitNs);
     bulk_wait_all();   // output stores complete
+    fence_proxy_async_all();
   }
   tc_fence_before();
   __syncthreads();
+  if (fail_item >= 0) {   // every unfinished (sequence, head): outputs and state NaN
+    const float qnan = __int_as_float(0x7fc00000);
+    for (int i = fail_item; i < p.N * p.H_v; i += p.NS) {
+      const int n = i / p.H_v, h = i % p.H_v;
+      int64_t s0, s1;
+      seq_chunks(p.cu, p.T, n, &s0, &s1);
+      for (int64_t e = tid; e < (s1 - s0) * kHeadDim; e += kPcThreads)
+        o[((s0 + e / kHeadDim) * p.H_v + h) * kHeadDim + e % kHeadDim] = from_f32<To>(qnan);
+      if (p.state_out)
+        for (int e = tid; e < kHeadDim * kHeadDim; e += kPcThreads)
+          p.state_out[((int64_t)n * p.H_v + h) * kHeadDim * kHeadDim + e] = qnan;
+    }
+  }
   if (warp == 0) tmem_dealloc(tmem, ST_COLS);
 }
 
@@ -1100,7 +1124,8 @@ cudaError_t launch_typed(const RecurArgs& a, int nsm, int NS) {
   e = cudaMemsetAsync(a.workspace, 0, CTRL_BYTES, a.stream);
   if (e != cudaSuccess) return e;
   PcParams p{a.g, a.beta, a.state_in, a.state_out, a.cu_seqlens, a.T_total, a.N,
-             a.H_k, a.H_v, a.scale, a.o, static_cast<uint8_t*>(a.workspace), NS};
+             a.H_k, a.H_v, a.scale, a.o, static_cast<uint8_t*>(a.workspace), NS,
+             wait_limit_ns()};
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)nsm);
   cfg.blockDim = dim3(kPcThreads);
@@ -1133,6 +1158,8 @@ int state_ctas(int64_t items, int H_v, int nsm) {
   return base;
 }
 
+std::atomic<uint64_t> g_wait_ns{kLimitNs};
+
 // ---- library-owned scratch for callers that cannot allocate --------------
 // Room for the rings of 49 state CTAs (a third of a 148-SM B200). Every GPU
 // that loads the library holds this array until the process exits.
@@ -1162,6 +1189,22 @@ cudaError_t noalloc_scratch(void** out) {
 }
 
 }  // namespace
+
+void set_wait_limit_ns(uint64_t ns) { g_wait_ns.store(ns ? ns : kLimitNs); }
+uint64_t wait_limit_ns() { return g_wait_ns.load(); }
+
+cudaError_t prefill_abort_word(const void* workspace, cudaStream_t stream, int* word) {
+  const void* ws = workspace;
+  if (!ws) {
+    void* scratch = nullptr;
+    cudaError_t e = noalloc_scratch(&scratch);
+    if (e != cudaSuccess) return e;
+    ws = scratch;
+  }
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return e;
+  return cudaMemcpy(word, static_cast<const int*>(ws) + 1, sizeof(int), cudaMemcpyDeviceToHost);
+}
 
 size_t prefill_noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
 

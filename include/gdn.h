@@ -58,7 +58,8 @@ typedef enum {
   GDN_ERR_INVALID_ARG = -1, /* null pointer, negative size, bad dtype ...  */
   GDN_ERR_UNSUPPORTED = -2, /* valid but not implemented (head dim != 128) */
   GDN_ERR_MISALIGNED = -3,  /* pointer or stride not 16-byte aligned        */
-  GDN_ERR_CUDA = -4         /* a CUDA launch or query failed               */
+  GDN_ERR_CUDA = -4,        /* a CUDA launch or query failed               */
+  GDN_ERR_TIMEOUT = -5      /* a bounded wait inside a kernel gave up      */
 } gdn_status;
 
 typedef enum { GDN_BF16 = 0, GDN_F32 = 1 } gdn_dtype;
@@ -147,6 +148,30 @@ gdn_status gdn_chunked_prefill(const void* q, const void* k, const void* v,
 
 /* Device scratch bytes gdn_chunked_prefill needs for these sizes (host). */
 size_t gdn_chunked_prefill_workspace(int N, int64_t T_total, int H_k, int H_v);
+
+/*
+ * gdn_chunked_prefill_status -- did the last gdn_chunked_prefill (bf16 inputs)
+ * that worked in `workspace` complete? Its CTAs hand chunks to one another
+ * through flags in the workspace, and every wait on such a flag is bounded
+ * (gdn_set_wait_limit_ns); a wait that runs out makes the whole call give up:
+ * each CTA leaves, the outputs o and state_out of every (sequence, head) not
+ * finished are written as NaN, and the workspace's abort word is set. This
+ * call waits for `stream` (it synchronises: it is not meant for the hot path),
+ * reads that word and returns GDN_OK or GDN_ERR_TIMEOUT (GDN_ERR_CUDA if the
+ * synchronisation or the 4-byte read fails). workspace == NULL reads the
+ * library-owned array of gdn_chunked_prefill_noalloc instead. The word is
+ * cleared by the next call that uses the workspace. Additional entry point.
+ */
+gdn_status gdn_chunked_prefill_status(const void* workspace, cudaStream_t stream);
+
+/*
+ * gdn_set_wait_limit_ns -- the bound, in nanoseconds, on each wait of the
+ * chunked prefill kernel for a flag that another CTA sets (0 restores the
+ * default, 2 s). A lower bound makes a stuck call give up sooner; the waits of
+ * a CTA on its own copies and tensor-core products keep their 2 s bound.
+ * Process-wide; read at each launch. Additional entry point.
+ */
+void gdn_set_wait_limit_ns(uint64_t ns);
 
 /*
  * gdn_stepwise_prefill -- the same packed-sequence recurrence advanced token by
