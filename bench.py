@@ -253,6 +253,17 @@ class PrefillWorkload:
         self.layer.chain(x, self.cu, gate, beta, z, self.y, self.o, out, self.ws,
                          state_out=self.state, ev=ev)
 
+    def step_fused(self, i, ev=None):
+        """The same pass as one gdn_prefill_layer launch (conv in the load stage,
+        norm before the outputs leave)."""
+        L = self.layer
+        if ev is not None:
+            ev[0].record()
+        L.gdn.gdn_prefill_layer(self.x, L.w, self.g, self.b, self.cu, self.z, L.nw,
+                                state_out=self.state, y=self.out, H_k=L.H_k, workspace=self.ws)
+        if ev is not None:
+            ev[1].record()
+
 
 class VarlenWorkload:
     """16 packed sequences, lengths uniform in [512, 16384] (seeded), fp32
@@ -547,6 +558,8 @@ def gpu_arm(args):
         ms, kms = mean_max(step_ms), mean_max(kern_ms)
         f_step, f_kern = timed_loop(pre.step, args.steps, args.warmup, barrier, flush=flush)
         f_ms, f_kms = mean_max(f_step), mean_max(f_kern)
+        u_step, _ = timed_loop(pre.step_fused, args.steps, args.warmup, barrier)
+        fu_ms = mean_max(u_step)
 
         var = VarlenWorkload(gdn, dev, seed, shard)
         v_step, v_kern = timed_loop(var.step, args.steps, args.warmup, barrier)
@@ -611,6 +624,13 @@ def gpu_arm(args):
                 "ms_per_step": e2e_ms},
         "gpu_launches": pre.launches_per_step * args.steps,
         "clocks": clk.summary(),
+        "prefill_layer_fused": {
+            "workload": "the same prefill step as one gdn_prefill_layer launch: conv + SiLU + "
+                        "L2 in the chunk kernel's load stage, gated RMSNorm before the outputs "
+                        "leave",
+            "value": throughput(T_PREFILL, units, fu_ms), "unit": "tokens/s",
+            "ms_per_step": fu_ms, "gpu_launches": args.steps,
+            "roofline": tensor_roofline("gdn_prefill_layer", flops, fu_ms, peaks, peak_src, None)},
         "prefill_l2_flushed": {
             "value": throughput(T_PREFILL, units, f_ms), "unit": "tokens/s", "ms_per_step": f_ms,
             "l2": f"{L2_FLUSH_BYTES >> 20} MB written between steps (outside the events)",
@@ -802,6 +822,24 @@ def profile_case(args):
         o = torch.empty((T, 48, 128), dtype=torch.bfloat16, device=dev)
         S = torch.empty((cu.numel() - 1, 48, 128, 128), device=dev)
         run = lambda: gdn.gdn_chunked_prefill(q, k, v, g, b, cud, state_in=si, state_out=S, o=o)
+    elif name == "dlayer":
+        # the fused decode layer step on pools of N slots (identity slots)
+        st = gi.decode_step_inputs(0, N, seed=0)
+        state = gi.initial_states(0, N, tag="pstate").to(dev)
+        cache = gi.to_bf16(gi.normal(0, "dconv", (N, 3, gi.CONV_CHANNELS))).to(dev)
+        x, g, b, z = (st[k].to(dev) for k in ("x_pre", "g", "beta", "z"))
+        w = gi.conv_weight(0).to(dev)
+        nw = torch.ones(128, device=dev)
+        idx = torch.arange(N, dtype=torch.int32, device=dev)
+        yo = torch.empty((N, 48, 128), dtype=torch.bfloat16, device=dev)
+        run = lambda: gdn.gdn_decode_layer_step(x, w, cache, g, b, state, idx, z, nw, y=yo)
+    elif name == "layer":
+        p = gi.prefill_inputs(T=T, seed=0)
+        x, w, g, b, z, nw, cu = (p[k].to(dev) for k in ("x_pre", "conv_w", "g", "beta", "z",
+                                                         "norm_w", "cu_seqlens"))
+        S = torch.empty((1, 48, 128, 128), device=dev)
+        yo = torch.empty((T, 48, 128), dtype=torch.bfloat16, device=dev)
+        run = lambda: gdn.gdn_prefill_layer(x, w, g, b, cu, z, nw, state_out=S, y=yo)
     elif name == "conv":
         p = gi.prefill_inputs(T=T, seed=0)
         x, w, cu = p["x_pre"].to(dev), p["conv_w"].to(dev), p["cu_seqlens"].to(dev)
@@ -833,7 +871,7 @@ def profile_case(args):
     print(f"{name}: {s.elapsed_time(e) / args.launches:.4f} ms per launch")
 
 
-PROFILE_CASES = ("decode", "prefill", "varlen", "conv", "norm", "dconv")
+PROFILE_CASES = ("decode", "dlayer", "prefill", "layer", "varlen", "conv", "norm", "dconv")
 
 
 def main():

@@ -23,7 +23,7 @@ import torch
 __all__ = ["GDN_BF16", "GDN_F32", "GdnError", "library_path", "load",
            "gdn_conv1d_silu", "gdn_chunked_prefill",
            "gdn_chunked_prefill_workspace", "gdn_chunked_prefill_noalloc",
-           "gdn_stepwise_prefill", "gdn_decode_layer_step",
+           "gdn_stepwise_prefill", "gdn_decode_layer_step", "gdn_prefill_layer",
            "gdn_chunked_prefill_status", "gdn_set_wait_limit_ns", "GDN_ERR_TIMEOUT",
            "gdn_decode_step",
            "gdn_gated_rmsnorm", "gdn_status_string", "gdn_version",
@@ -56,6 +56,9 @@ _SIGNATURES = {
                                    _vp]),
     "gdn_chunked_prefill_workspace": (ctypes.c_size_t, [_int, _i64, _int, _int]),
     "gdn_chunked_prefill_status": (_int, [_vp, _vp]),
+    "gdn_prefill_layer": (_int, [_vp, _i64, _vp, _int, _vp, _vp, _vp, _vp, _vp, _int, _vp,
+                                 _vp, _vp, _int, _i64, _int, _int, _f32, _f32, _vp, _vp,
+                                 _f32, _vp, _int, _vp, ctypes.c_size_t, _vp]),
     "gdn_set_wait_limit_ns": (None, [ctypes.c_uint64]),
     "gdn_stepwise_prefill": (_int, [_vp, _vp, _vp, _int, _i64, _i64, _i64, _vp,
                                     _vp, _int, _vp, _vp, _vp, _int, _i64, _int,
@@ -231,6 +234,48 @@ def gdn_chunked_prefill(q, k, v, g, beta, cu_seqlens, *, state_in=None,
         scale, _ptr(o), _dtype_code(o.dtype), _ptr(workspace), ws_bytes,
         _stream(stream, v.device)))
     return o
+
+
+def gdn_prefill_layer(x, conv_w, g, beta, cu_seqlens, z, norm_w, *, conv_bias=None,
+                      conv_state_in=None, conv_state_out=None, state_in=None,
+                      state_out=None, scale=1.0, l2_eps=1e-6, norm_eps=1e-6, y=None,
+                      y_dtype=None, H_k=H_K, workspace=None, stream=None):
+    """The whole prefill of the layer in one kernel: conv + SiLU + q/k L2 from the
+    pre-conv x [T, C] (bf16, C = 2*H_k*128 + H_v*128), the chunked gated delta
+    rule, and the gated RMS-norm with gate z [T, H_v, 128] (bf16) and weight
+    norm_w [128] (conv_w's dtype). Returns the normed output y [T, H_v, 128]."""
+    T, C = x.shape
+    H_v = g.shape[1]
+    N = cu_seqlens.numel() - 1
+    if x.dtype != torch.bfloat16:
+        raise ValueError("x must be bf16")
+    if C != (2 * H_k + H_v) * HEAD_DIM:
+        raise ValueError(f"x: {C} channels, expected {(2 * H_k + H_v) * HEAD_DIM}")
+    _expect(conv_w, (C, 4), "conv_w")
+    _expect(conv_bias, (C,), "conv_bias", conv_w.dtype)
+    _expect(conv_state_in, (N, 3, C), "conv_state_in", torch.bfloat16)
+    _expect(conv_state_out, (N, 3, C), "conv_state_out", torch.bfloat16)
+    _expect(cu_seqlens, (N + 1,), "cu_seqlens", torch.int32)
+    _expect(g, (T, H_v), "g")
+    _expect(beta, (T, H_v), "beta", g.dtype)
+    _expect(state_in, (N, H_v, HEAD_DIM, HEAD_DIM), "state_in", torch.float32)
+    _expect(state_out, (N, H_v, HEAD_DIM, HEAD_DIM), "state_out", torch.float32)
+    _expect(z, (T, H_v, HEAD_DIM), "z", torch.bfloat16)
+    _expect(norm_w, (HEAD_DIM,), "norm_w", conv_w.dtype)
+    _expect(y, (T, H_v, HEAD_DIM), "y")
+    if y is None:
+        y = torch.empty((T, H_v, HEAD_DIM), dtype=y_dtype or torch.bfloat16, device=x.device)
+    need = gdn_chunked_prefill_workspace(N, T, H_k, H_v)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("gdn_prefill_layer", load().gdn_prefill_layer(
+        _ptr(x), _row_stride(x), _ptr(conv_w), _dtype_code(conv_w.dtype), _ptr(conv_bias),
+        _ptr(conv_state_in), _ptr(conv_state_out), _ptr(g), _ptr(beta), _dtype_code(g.dtype),
+        _ptr(state_in), _ptr(state_out), _ptr(cu_seqlens), N, T, H_k, H_v, scale, l2_eps,
+        _ptr(z), _ptr(norm_w), norm_eps, _ptr(y), _dtype_code(y.dtype), _ptr(workspace),
+        ws_bytes, _stream(stream, x.device)))
+    return y
 
 
 def gdn_chunked_prefill_status(workspace=None, stream=None) -> int:

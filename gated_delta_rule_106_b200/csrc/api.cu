@@ -149,6 +149,51 @@ gdn_status gdn_chunked_prefill(const void* q, const void* k, const void* v,
                                          : gdn::launch_prefill_chunked_f32(a));
 }
 
+gdn_status gdn_prefill_layer(const void* x, int64_t x_row_stride, const void* conv_w,
+                             gdn_dtype w_dtype, const void* conv_bias,
+                             const void* conv_state_in, void* conv_state_out,
+                             const void* g, const void* beta, gdn_dtype gate_dtype,
+                             const float* state_in, float* state_out,
+                             const int32_t* cu_seqlens, int N, int64_t T_total, int H_k,
+                             int H_v, float scale, float l2_eps, const void* z,
+                             const void* norm_w, float norm_eps, void* y, gdn_dtype y_dtype,
+                             void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (!valid_dtype(w_dtype) || !valid_dtype(gate_dtype) || !valid_dtype(y_dtype))
+    return GDN_ERR_INVALID_ARG;
+  if (N < 0 || T_total < 0 || H_k <= 0 || H_v <= 0 || H_v % H_k != 0 || !(l2_eps >= 0.f) ||
+      !(norm_eps >= 0.f))
+    return GDN_ERR_INVALID_ARG;
+  const int64_t C = 2 * (int64_t)H_k * kHeadDim + (int64_t)H_v * kHeadDim;
+  if (x_row_stride < C) return GDN_ERR_INVALID_ARG;
+  if (N == 0) return T_total == 0 ? GDN_OK : GDN_ERR_INVALID_ARG;
+  if (!cu_seqlens || !conv_w || !norm_w) return GDN_ERR_INVALID_ARG;
+  if (T_total > 0 && (!x || !g || !beta || !z || !y)) return GDN_ERR_INVALID_ARG;
+  if ((x && !aligned16(x)) || !aligned16(conv_w) || (conv_bias && !aligned16(conv_bias)) ||
+      (conv_state_in && !aligned16(conv_state_in)) ||
+      (conv_state_out && !aligned16(conv_state_out)) || (z && !aligned16(z)) ||
+      !aligned16(norm_w) || (y && !aligned16(y)) || (state_in && !aligned16(state_in)) ||
+      (state_out && !aligned16(state_out)))
+    return GDN_ERR_MISALIGNED;
+  if (!stride_ok(x_row_stride, GDN_BF16)) return GDN_ERR_MISALIGNED;
+  const int gb = gdn::elem_bytes(gate_dtype);
+  if ((g && !aligned_to(g, gb)) || (beta && !aligned_to(beta, gb))) return GDN_ERR_MISALIGNED;
+  const size_t st_bytes = (size_t)N * H_v * kHeadDim * kHeadDim * sizeof(float);
+  if (partial_overlap(state_in, st_bytes, state_out, st_bytes)) return GDN_ERR_INVALID_ARG;
+  const size_t cs_bytes = (size_t)N * 3 * C * 2;
+  if (partial_overlap(conv_state_in, cs_bytes, conv_state_out, cs_bytes))
+    return GDN_ERR_INVALID_ARG;
+  if (T_total > 0) {
+    if (workspace_bytes < gdn_chunked_prefill_workspace(N, T_total, H_k, H_v) || !workspace)
+      return GDN_ERR_INVALID_ARG;
+    if (!aligned16(workspace)) return GDN_ERR_MISALIGNED;
+  }
+  gdn::LayerPrefillArgs a{x, x_row_stride, conv_w, w_dtype, conv_bias, conv_state_in,
+                          conv_state_out, g, beta, gate_dtype, state_in, state_out,
+                          cu_seqlens, N, T_total, H_k, H_v, scale, l2_eps, z, norm_w,
+                          norm_eps, y, y_dtype, workspace, workspace_bytes, stream};
+  return from_cuda(gdn::launch_prefill_layer(a));
+}
+
 gdn_status gdn_chunked_prefill_status(const void* workspace, cudaStream_t stream) {
   if (workspace && !aligned16(workspace)) return GDN_ERR_MISALIGNED;
   int word = 0;

@@ -341,6 +341,19 @@ cudaError_t launch_w(const ConvArgs& a) {
 
 }  // namespace
 
+cudaError_t launch_conv_state_roll(const void* x, int64_t x_row_stride, gdn_dtype x_dtype,
+                                   int channels, const int32_t* cu, int N, int64_t T,
+                                   const void* cs_in, void* cs_out, cudaStream_t stream) {
+  const int eb = elem_bytes(x_dtype);
+  const int row_bytes = channels * eb;
+  const int64_t threads = (int64_t)N * (row_bytes / 16);
+  if (threads == 0) return cudaSuccess;
+  conv_state_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, stream>>>(
+      static_cast<const char*>(x), x_row_stride * eb, row_bytes, cu, N, T,
+      static_cast<const char*>(cs_in), static_cast<char*>(cs_out), 0);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_conv1d_silu(const ConvArgs& a) {
   return a.x_dtype == GDN_F32 ? launch_w<float>(a) : launch_w<__nv_bfloat16>(a);
 }

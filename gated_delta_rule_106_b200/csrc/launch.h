@@ -48,6 +48,23 @@ struct DecodeLayerArgs {
   cudaStream_t stream;
 };
 
+// The whole prefill layer in the chunk kernel: conv + SiLU + q/k L2 from the
+// pre-conv x (bf16) in the load stage, gated RMS-norm of the outputs before
+// they leave. Conv weights, bias and the norm weight share w_dtype; z is bf16.
+struct LayerPrefillArgs {
+  const void* x; int64_t x_row_stride;
+  const void* conv_w; gdn_dtype w_dtype; const void* conv_bias;
+  const void* conv_state_in; void* conv_state_out;
+  const void* g; const void* beta; gdn_dtype gate_dtype;
+  const float* state_in; float* state_out;
+  const int32_t* cu_seqlens; int N; int64_t T_total; int H_k; int H_v;
+  float scale; float l2_eps;
+  const void* z; const void* norm_w; float norm_eps;
+  void* y; gdn_dtype y_dtype;
+  void* workspace; size_t workspace_bytes;
+  cudaStream_t stream;
+};
+
 struct NormArgs {
   const void* x; gdn_dtype x_dtype; const void* z; gdn_dtype z_dtype;
   const void* w; gdn_dtype w_dtype; int64_t rows; int dim; float eps;
@@ -55,6 +72,12 @@ struct NormArgs {
 };
 
 cudaError_t launch_conv1d_silu(const ConvArgs& a);
+// conv_state_out[n] = the last three pre-conv rows of sequence n (shifted in
+// from conv_state_in when shorter); conv_state_out may alias conv_state_in.
+cudaError_t launch_conv_state_roll(const void* x, int64_t x_row_stride, gdn_dtype x_dtype,
+                                   int channels, const int32_t* cu, int N, int64_t T,
+                                   const void* cs_in, void* cs_out, cudaStream_t stream);
+cudaError_t launch_prefill_layer(const LayerPrefillArgs& a);
 cudaError_t launch_gated_rmsnorm(const NormArgs& a);
 cudaError_t launch_decode_step(const RecurArgs& a);
 cudaError_t launch_decode_layer(const DecodeLayerArgs& a);

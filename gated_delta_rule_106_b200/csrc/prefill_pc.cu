@@ -129,6 +129,13 @@ struct PcParams {
   uint8_t* ws;          // workspace base
   int NS;               // state CTAs
   uint64_t wait_ns;     // limit of a wait on another CTA's flag
+  // the whole layer (gdn_prefill_layer): pre-conv x [T, C] bf16 with row stride xs,
+  // conv taps cw [C, 4] and bias cb (conv weight dtype), carried conv history
+  // cs_in [N, 3, C] (bf16, may be null), q/k L2 epsilon; gated RMS-norm gate z
+  // [T, H_v, 128] bf16, weight nw [128] (conv weight dtype), epsilon
+  const void* x; int64_t xs; const void* cw; const void* cb; const void* cs_in; int C;
+  float l2_eps;
+  const void* z; const void* nw; float norm_eps;
 };
 
 constexpr int kCuCache = 513;   // sequences whose boundaries the prep CTAs keep on chip
@@ -320,8 +327,99 @@ __device__ __forceinline__ void merge_level(const float* Af, float* Tf, float* X
   bar_sync_n(bar, kPipeThreads);
 }
 
+// The layer's prologue inside a prep pipeline: the K, Q (key head kh) and V
+// (value head h) tiles of the chunk at t0 (L tokens of sequence n, which starts
+// at s0) from the pre-conv input: causal conv k=4 (+ bias) over rows t0-3 ..
+// t0+63, SiLU, and the per-token L2 norm of the q and k heads, rounded to bf16
+// into the 128-byte-swizzled [64 tokens][64 channels] blocks that the tensor
+// cores read (the layout the tensor-map loads of the plain path produce). Rows
+// before the sequence start come from the carried conv history (zeros if none);
+// tokens at or past L are written as zeros. Warps 0-5: warp = 2 * part + half,
+// part 0/1/2 = q/k/v, half = tokens 0-31 / 32-63; lane = 4 channels. The
+// arithmetic (and its order) is the conv kernel's, so the tiles hold exactly
+// the values that kernel would store.
+template <class Tw>
+__device__ __forceinline__ void conv_fill(const PcParams& p, uint8_t* kq, uint8_t* vv, int n,
+                                          int kh, int h, int64_t s0, int64_t t0, int L,
+                                          int warp, int lane) {
+  const int part = warp >> 1, half = warp & 1;
+  const int c = (part == 0 ? kh * kHeadDim
+                           : part == 1 ? (p.H_k + kh) * kHeadDim : (2 * p.H_k + h) * kHeadDim) +
+                lane * 4;
+  const Tw* w = static_cast<const Tw*>(p.cw);
+  const Tw* bias = static_cast<const Tw*>(p.cb);
+  float wt[4][4], b[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    b[e] = bias ? to_f32(bias[c + e]) : 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) wt[e][j] = to_f32(w[(c + e) * 4 + j]);
+  }
+  const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(p.x);
+  const __nv_bfloat16* cs = static_cast<const __nv_bfloat16*>(p.cs_in);
+  // the pre-conv row of chunk token tt (tt may be -3..-1), as loaded (4 bf16)
+  auto load_row = [&](int tt) -> uint2 {
+    const int64_t tg = t0 + tt;
+    if (tg >= s0 && tg < p.T) return __ldg(reinterpret_cast<const uint2*>(x + tg * p.xs + c));
+    if (tg < s0 && cs)
+      return __ldg(reinterpret_cast<const uint2*>(cs + ((int64_t)n * 3 + 3 + (tg - s0)) * p.C + c));
+    return make_uint2(0u, 0u);
+  };
+  auto unpack = [](uint2 u, float (&f)[4]) {
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+    const float2 bb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+    f[0] = a.x; f[1] = a.y; f[2] = bb.x; f[3] = bb.y;
+  };
+  uint8_t* tile = (part == 0 ? kq + 8192 : part == 1 ? kq : vv) +
+                  (lane >> 4) * (part == 2 ? 8192 : 16384);
+  const int chunk = (lane & 15) >> 1, sub = (lane & 1) * 8;
+  float h0[4], h1[4], h2[4];
+#pragma unroll 1
+  for (int bt = 0; bt < 2; ++bt) {   // two batches of 16 tokens, every load issued first
+    const int tb = half * 32 + bt * 16;
+    uint2 raw[19];
+#pragma unroll
+    for (int i = 0; i < 19; ++i) raw[i] = (bt == 0 || i >= 3) ? load_row(tb - 3 + i) : make_uint2(0u, 0u);
+    if (bt == 0) {
+      unpack(raw[0], h0);
+      unpack(raw[1], h1);
+      unpack(raw[2], h2);
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int tt = tb + i;
+      float h3[4], out[4], ss = 0.f;
+      unpack(raw[3 + i], h3);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float a = fmaf(wt[e][3], h3[e], fmaf(wt[e][2], h2[e], fmaf(wt[e][1], h1[e], fmaf(wt[e][0], h0[e], b[e]))));
+        out[e] = silu(a);
+        ss = fmaf(out[e], out[e], ss);
+      }
+      if (part < 2) {   // warp-uniform: the warp is one 128-channel q or k head
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+        const float inv = rsqrtf(ss + p.l2_eps);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) out[e] *= inv;
+      }
+      const bool live = tt < L;
+      const __nv_bfloat162 lo = __floats2bfloat162_rn(live ? out[0] : 0.f, live ? out[1] : 0.f);
+      const __nv_bfloat162 hi = __floats2bfloat162_rn(live ? out[2] : 0.f, live ? out[3] : 0.f);
+      *reinterpret_cast<uint2*>(tile + swz(tt, chunk) + sub) =
+          make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        h0[e] = h1[e];
+        h1[e] = h2[e];
+        h2[e] = h3[e];
+      }
+    }
+  }
+}
+
 // ===================================================================== prep ==
-template <class Tg>
+template <class Tg, bool Fused, class Tw>
 __device__ void prep_role(const PcParams& p, const CUtensorMap* tm_q, const CUtensorMap* tm_k,
                           const CUtensorMap* tm_v, uint8_t* sm) {
   PrepSmall& sh = *reinterpret_cast<PrepSmall*>(sm + P_SMALL);
@@ -407,7 +505,7 @@ __device__ void prep_role(const PcParams& p, const CUtensorMap* tm_q, const CUte
   if (ptid == kIssuer) {
     const int x = claim();
     ss.claim = x;
-    if (x < E) {
+    if (!Fused && x < E) {
       issue_tiles(x);
       pend = true;
     }
@@ -433,9 +531,13 @@ __device__ void prep_role(const PcParams& p, const CUtensorMap* tm_q, const CUte
     bool ok = true;
 
     // the slot is written directly: wait until step r - kRing has been consumed
-    if (ptid == 0)
+    // (the layer's form waits in warp 6, which has no share of the conv)
+    if (ptid == (Fused ? 192 : 0))
       ss.ok = wait_flag_ge(flags_of(p.ws, s) + kRing, r + 1 - kRing, &ctrl[1], p.wait_ns);
-    if (warp == 1) {   // gates: cumulative log-decay and derived vectors
+    if constexpr (Fused) {   // the chunk's q, k, v tiles from the pre-conv input
+      if (warp < 6) conv_fill<Tw>(p, kq, vv, n, h / (p.H_v / p.H_k), h, s0, t0, L, warp, lane);
+    }
+    if (warp == (Fused ? 7 : 1)) {   // gates: cumulative log-decay and derived vectors
       const Tg* g = static_cast<const Tg*>(p.g);
       const Tg* bt = static_cast<const Tg*>(p.beta);
       float lg[2], be[2];
@@ -471,16 +573,20 @@ __device__ void prep_role(const PcParams& p, const CUtensorMap* tm_q, const CUte
       }
       if (lane == 0) ss.gL = __expf(Gl);
     }
-    ok = mbar_wait_bounded(&ss.bar_tma, tma_par, kLimitNs);
-    if (ok) {   // a phase seen complete by this thread
-      tma_par ^= 1;
-      if (ptid == kIssuer) pend = false;
+    if constexpr (Fused) {
+      fence_proxy_async_smem();   // the tensor cores read what the threads wrote
+    } else {
+      ok = mbar_wait_bounded(&ss.bar_tma, tma_par, kLimitNs);
+      if (ok) {   // a phase seen complete by this thread
+        tma_par ^= 1;
+        if (ptid == kIssuer) pend = false;
+      }
     }
     bar_sync_n(bar, kPipeThreads);
     ok = ok && ss.ok;
     if (bar_or_n(bar, kPipeThreads, !ok)) goto fail;
 
-    if (L < kChunk) {   // rows past the sequence end hold other data: zero them
+    if (!Fused && L < kChunk) {   // rows past the sequence end hold other data: zero them
       for (int idx = ptid; idx < 3072; idx += kPipeThreads) {
         const int rr = (idx & 511) >> 3;
         if (rr >= L) {
@@ -647,7 +753,7 @@ __device__ void prep_role(const PcParams& p, const CUtensorMap* tm_q, const CUte
     mma_par ^= 1;
     tc_fence_after();
     // the tiles are free: start the next item's loads
-    if (ptid == kIssuer && ok && next < E) {
+    if (!Fused && ptid == kIssuer && ok && next < E) {
       issue_tiles(next);
       pend = true;
     }
@@ -702,7 +808,7 @@ __device__ void prep_role(const PcParams& p, const CUtensorMap* tm_q, const CUte
 }
 
 // ==================================================================== state ==
-template <class To>
+template <class To, bool Fused, class Tw>
 __device__ void state_role(const PcParams& p, const CUtensorMap* tm_o, uint8_t* sm, int s) {
   StateSmall& ss = *reinterpret_cast<StateSmall*>(sm + S_SMALL);
   int* ctrl = reinterpret_cast<int*>(p.ws);
@@ -818,6 +924,43 @@ __device__ void state_role(const PcParams& p, const CUtensorMap* tm_o, uint8_t* 
       for (int j = 0; j < 16; ++j) stg[(16 * cg + j) * kHeadDim + row] = ov[j];
     }
   };
+  // the layer's epilogue: gated RMS-norm of a staged [64 t][128 i] output tile in
+  // place, y = o / sqrt(mean(o^2) + eps) * w * SiLU(z) per token (8 threads per
+  // token, 16 channels each); the staged o is already in o's dtype, as the plain
+  // path would store it
+  auto norm_stage = [&](uint8_t* stage, int64_t ot0, int oL, int oh) {
+    const int t = tid >> 3, c0 = (tid & 7) * 16;
+    To* sv = reinterpret_cast<To*>(stage) + t * kHeadDim + c0;
+    float ssum = 0.f;
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      float v[8];
+      load8(sv + 8 * q, v);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) ssum = fmaf(v[j], v[j], ssum);
+    }
+    ssum += __shfl_xor_sync(0xffffffffu, ssum, 1);
+    ssum += __shfl_xor_sync(0xffffffffu, ssum, 2);
+    ssum += __shfl_xor_sync(0xffffffffu, ssum, 4);
+    if (t < oL) {
+      const float inv = rsqrtf(ssum * (1.0f / kHeadDim) + p.norm_eps);
+      const __nv_bfloat16* zr =
+          static_cast<const __nv_bfloat16*>(p.z) + ((ot0 + t) * p.H_v + oh) * kHeadDim + c0;
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        float v[8], zz[8], wv[8];
+        load8(sv + 8 * q, v);
+        load8(zr + 8 * q, zz);
+        load8(static_cast<const Tw*>(p.nw) + c0 + 8 * q, wv);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = v[j] * inv * wv[j] * silu(zz[j]);
+        store8(sv + 8 * q, v);
+      }
+    }
+  };
+  bool staged = false;            // (fused) a normed tile waits in the stage of buffer r & 1
+  int64_t stg_t0 = 0;
+  int stg_L = 0, stg_h = 0;
   bool pend = false;              // a step's outputs wait in TMEM
   int64_t pend_t0 = 0;
   int pend_L = 0, pend_h = 0;
@@ -960,9 +1103,19 @@ __device__ void state_role(const PcParams& p, const CUtensorMap* tm_o, uint8_t* 
         issue_copy(r + 1, true);
         issued = r + 2;
       }
-      // and step r-1's outputs leave from the stage
+      // and step r-1's outputs leave from the stage (the layer's form first normalises
+      // them there and leaves them after the step's last barrier)
       if (pend) {
-        emit_out(buf + S_STG_OFF, pend_t0, pend_L, pend_h);
+        if constexpr (Fused) {
+          norm_stage(buf + S_STG_OFF, pend_t0, pend_L, pend_h);
+          fence_proxy_async_smem();
+          staged = true;
+          stg_t0 = pend_t0;
+          stg_L = pend_L;
+          stg_h = pend_h;
+        } else {
+          emit_out(buf + S_STG_OFF, pend_t0, pend_L, pend_h);
+        }
         pend = false;
       }
       if (!mbar_wait_bounded(&ss.bar_p, par_p, kLimitNs)) ok = false;
@@ -991,6 +1144,10 @@ __device__ void state_role(const PcParams& p, const CUtensorMap* tm_o, uint8_t* 
       }
       tc_fence_before();
       if (__syncthreads_or(!ok)) { ok = false; break; }
+      if (Fused && staged) {   // the normed tile of step r-1, staged in this step's buffer
+        emit_out(buf + S_STG_OFF, stg_t0, stg_L, stg_h);
+        staged = false;
+      }
       pend = true;
       pend_t0 = t0;
       pend_L = L;
@@ -1015,6 +1172,11 @@ __device__ void state_role(const PcParams& p, const CUtensorMap* tm_o, uint8_t* 
     stage_out(lbuf, ov);
     fence_proxy_async_smem();
     __syncthreads();
+    if constexpr (Fused) {
+      norm_stage(lbuf + S_STG_OFF, pend_t0, pend_L, pend_h);
+      fence_proxy_async_smem();
+      __syncthreads();
+    }
     emit_out(lbuf + S_STG_OFF, pend_t0, pend_L, pend_h);
   }
   if (!ok && tid == 0) atomicExch(&ctrl[1], 1);
@@ -1045,7 +1207,7 @@ __device__ void state_role(const PcParams& p, const CUtensorMap* tm_o, uint8_t* 
   if (warp == 0) tmem_dealloc(tmem, ST_COLS);
 }
 
-template <class Tg, class To>
+template <class Tg, class To, bool Fused, class Tw>
 __global__ void __launch_bounds__(kPcThreads, 1)
 prefill_pc_kernel(const __grid_constant__ CUtensorMap tm_q,
                   const __grid_constant__ CUtensorMap tm_k,
@@ -1054,8 +1216,8 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap tm_q,
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  if ((int)blockIdx.x < p.NS) state_role<To>(p, &tm_o, sm, blockIdx.x);
-  else prep_role<Tg>(p, &tm_q, &tm_k, &tm_v, sm);
+  if ((int)blockIdx.x < p.NS) state_role<To, Fused, Tw>(p, &tm_o, sm, blockIdx.x);
+  else prep_role<Tg, Fused, Tw>(p, &tm_q, &tm_k, &tm_v, sm);
 }
 
 // ------------------------------------------------------------------ host --
@@ -1105,6 +1267,11 @@ int sm_count() {
   return n;
 }
 
+template <class Tg, class To, bool Fused, class Tw>
+cudaError_t launch_kernel(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                          const CUtensorMap& mo, const PcParams& p, int nsm, void* workspace,
+                          cudaStream_t stream);
+
 template <class Tg, class To>
 cudaError_t launch_typed(const RecurArgs& a, int nsm, int NS) {
   CUtensorMap mq, mk, mv, mo;
@@ -1117,20 +1284,28 @@ cudaError_t launch_typed(const RecurArgs& a, int nsm, int NS) {
   } else {
     mo = mv;   // unused: fp32 outputs are stored by the threads
   }
-  auto kern = prefill_pc_kernel<Tg, To>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)PC_SMEM_ALLOC);
-  if (e != cudaSuccess) return e;
-  e = cudaMemsetAsync(a.workspace, 0, CTRL_BYTES, a.stream);
-  if (e != cudaSuccess) return e;
   PcParams p{a.g, a.beta, a.state_in, a.state_out, a.cu_seqlens, a.T_total, a.N,
              a.H_k, a.H_v, a.scale, a.o, static_cast<uint8_t*>(a.workspace), NS,
              wait_limit_ns()};
+  return launch_kernel<Tg, To, false, float>(mq, mk, mv, mo, p, nsm, a.workspace, a.stream);
+}
+
+// one cooperative launch of the kernel, one CTA per SM
+template <class Tg, class To, bool Fused, class Tw>
+cudaError_t launch_kernel(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                          const CUtensorMap& mo, const PcParams& p, int nsm, void* workspace,
+                          cudaStream_t stream) {
+  auto kern = prefill_pc_kernel<Tg, To, Fused, Tw>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)PC_SMEM_ALLOC);
+  if (e != cudaSuccess) return e;
+  e = cudaMemsetAsync(workspace, 0, CTRL_BYTES, stream);
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)nsm);
   cfg.blockDim = dim3(kPcThreads);
   cfg.dynamicSmemBytes = PC_SMEM_ALLOC;
-  cfg.stream = a.stream;
+  cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
@@ -1234,6 +1409,64 @@ cudaError_t launch_prefill_pc(const RecurArgs& a) {
   if (a.workspace_bytes < CTRL_BYTES + (size_t)NS * kRing * SLOT_BYTES || !a.workspace)
     return cudaErrorInvalidValue;
   return a.gate_dtype == GDN_F32 ? pick_o<float>(a, nsm, NS) : pick_o<__nv_bfloat16>(a, nsm, NS);
+}
+
+namespace {
+
+template <class Tg, class To, class Tw>
+cudaError_t launch_layer_typed(const LayerPrefillArgs& a, int nsm, int NS) {
+  const int64_t C = 2 * (int64_t)a.H_k * kHeadDim + (int64_t)a.H_v * kHeadDim;
+  CUtensorMap mx, mo;
+  // the q/k/v tensor maps of the plain path are not read in the layer's form;
+  // a valid map over x stands in their place
+  if (!make_map(&mx, a.x, C, a.T_total, a.x_row_stride)) return cudaErrorInvalidValue;
+  if (sizeof(To) == 2) {
+    if (!make_out_map(&mo, a.y, (int64_t)a.H_v * kHeadDim, a.T_total)) return cudaErrorInvalidValue;
+  } else {
+    mo = mx;
+  }
+  PcParams p{a.g, a.beta, a.state_in, a.state_out, a.cu_seqlens, a.T_total, a.N, a.H_k, a.H_v,
+             a.scale, a.y, static_cast<uint8_t*>(a.workspace), NS, wait_limit_ns(),
+             a.x, a.x_row_stride, a.conv_w, a.conv_bias, a.conv_state_in, (int)C, a.l2_eps,
+             a.z, a.norm_w, a.norm_eps};
+  return launch_kernel<Tg, To, true, Tw>(mx, mx, mx, mo, p, nsm, a.workspace, a.stream);
+}
+template <class Tg, class To>
+cudaError_t layer_pick_w(const LayerPrefillArgs& a, int nsm, int NS) {
+  return a.w_dtype == GDN_F32 ? launch_layer_typed<Tg, To, float>(a, nsm, NS)
+                              : launch_layer_typed<Tg, To, __nv_bfloat16>(a, nsm, NS);
+}
+template <class Tg>
+cudaError_t layer_pick_o(const LayerPrefillArgs& a, int nsm, int NS) {
+  return a.y_dtype == GDN_F32 ? layer_pick_w<Tg, float>(a, nsm, NS)
+                              : layer_pick_w<Tg, __nv_bfloat16>(a, nsm, NS);
+}
+
+}  // namespace
+
+cudaError_t launch_prefill_layer(const LayerPrefillArgs& a) {
+  if (a.N == 0) return cudaSuccess;
+  cudaError_t e = cudaSuccess;
+  if (a.T_total > 0) {
+    const int nsm = sm_count();
+    if (nsm < 2) return cudaErrorInvalidDevice;
+    const int NS = state_ctas((int64_t)a.N * a.H_v, a.H_v, nsm);
+    if (a.workspace_bytes < CTRL_BYTES + (size_t)NS * kRing * SLOT_BYTES || !a.workspace)
+      return cudaErrorInvalidValue;
+    e = a.gate_dtype == GDN_F32 ? layer_pick_o<float>(a, nsm, NS)
+                                : layer_pick_o<__nv_bfloat16>(a, nsm, NS);
+  } else {   // no tokens: the states pass through
+    RecurArgs r{a.x, a.x, a.x, GDN_BF16, a.x_row_stride, a.x_row_stride, a.x_row_stride,
+                a.g, a.beta, a.gate_dtype, a.state_in, a.state_out, a.cu_seqlens, a.N, 0,
+                a.H_k, a.H_v, a.scale, a.y, a.y_dtype, nullptr, 0, a.stream};
+    e = launch_prefill_chunked_f32(r);
+  }
+  if (e != cudaSuccess || !a.conv_state_out) return e;
+  // the carried conv history for the next call: each sequence's last three
+  // pre-conv rows (after the kernel, which read conv_state_in: they may alias)
+  return launch_conv_state_roll(a.x, a.x_row_stride, GDN_BF16,
+                                2 * a.H_k * kHeadDim + a.H_v * kHeadDim, a.cu_seqlens, a.N,
+                                a.T_total, a.conv_state_in, a.conv_state_out, a.stream);
 }
 
 }  // namespace gdn

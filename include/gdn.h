@@ -150,6 +150,42 @@ gdn_status gdn_chunked_prefill(const void* q, const void* k, const void* v,
 size_t gdn_chunked_prefill_workspace(int N, int64_t T_total, int H_k, int H_v);
 
 /*
+ * gdn_prefill_layer -- the whole prefill of the delta-rule layer in one launch
+ * of the tensor-core chunk kernel: the causal conv (kernel 4) + SiLU + per-head
+ * L2 norm of q and k ([P2 二.1], [P3 架构]) is computed in the kernel's load
+ * stage from the pre-conv input, the chunked (chunk = 64) gated delta rule
+ * ([P2 二.1]) as in gdn_chunked_prefill, and the gated RMS-norm ([P3 架构]) is
+ * applied to each output tile before it leaves. The result equals
+ * gdn_conv1d_silu -> gdn_chunked_prefill (o in y_dtype) -> gdn_gated_rmsnorm:
+ * the conv values enter the chunk products rounded to bf16 exactly as the conv
+ * kernel stores them, and the norm reads the outputs in y_dtype. Neither the
+ * conv output nor the un-normed output is written to memory. Additional entry
+ * point (fused form of the three calls).
+ *
+ *   x            [T_total, C] bf16, row stride x_row_stride: pre-conv q | k | v,
+ *                C = 2*H_k*128 + H_v*128.
+ *   conv_w       [C, 4] w_dtype (tap 3 = current token); conv_bias [C] w_dtype or NULL.
+ *   conv_state_in   [N, 3, C] bf16 history before each sequence, or NULL (zeros).
+ *   conv_state_out  [N, 3, C] bf16 or NULL: each sequence's last three pre-conv
+ *                rows (may alias conv_state_in; written after the kernel has read it).
+ *   g, beta, state_in, state_out, cu_seqlens, N, T_total, H_k, H_v, scale,
+ *                workspace: as gdn_chunked_prefill (gdn_chunked_prefill_workspace).
+ *   l2_eps       q/k L2 epsilon: y / sqrt(sum y^2 + l2_eps).
+ *   z            [T_total, H_v, 128] bf16 gate; norm_w [128] w_dtype; norm_eps.
+ *   y            [T_total, H_v, 128] contiguous, y_dtype: the normed output.
+ * A bounded wait that gives up is reported by gdn_chunked_prefill_status.
+ */
+gdn_status gdn_prefill_layer(const void* x, int64_t x_row_stride, const void* conv_w,
+                             gdn_dtype w_dtype, const void* conv_bias,
+                             const void* conv_state_in, void* conv_state_out,
+                             const void* g, const void* beta, gdn_dtype gate_dtype,
+                             const float* state_in, float* state_out,
+                             const int32_t* cu_seqlens, int N, int64_t T_total, int H_k,
+                             int H_v, float scale, float l2_eps, const void* z,
+                             const void* norm_w, float norm_eps, void* y, gdn_dtype y_dtype,
+                             void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * gdn_chunked_prefill_status -- did the last gdn_chunked_prefill (bf16 inputs)
  * that worked in `workspace` complete? Its CTAs hand chunks to one another
  * through flags in the workspace, and every wait on such a flag is bounded
