@@ -14,6 +14,9 @@ section 二.1, and the Agnes-3.0-Flash Preview model card, section 架构):
 * :func:`recurrence` -- the stepwise gated delta rule
   ``S_t = g_t S_{t-1}(I - b_t k_t k_t^T) + b_t v_t k_t^T``, ``o_t = scale S_t q_t``.
 * :func:`gated_rmsnorm` -- ``x / sqrt(mean x^2 + eps) * w * SiLU(z)``.
+* :func:`attention` -- the hybrid decoder's global-attention layer (model card,
+  架构 table; commentary section 二.1): q/k RMS-norm, rotary on the first 64
+  dims, causal GQA softmax attention, sigmoid output gate.
 * :mod:`oracle.chunked` -- the chunk-64 (WY / UT-transform) form of the same
   recurrence in numpy fp64, with optional operand-rounding emulation; a
   test-only cross-check, not the oracle of record.
@@ -75,6 +78,13 @@ def _load():
         lib.oracle_recurrence.argtypes = [
             _dp, _dp, _dp, _dp, _dp, _dp, _ip, ctypes.c_int, ctypes.c_int,
             ctypes.c_int, ctypes.c_int, ctypes.c_double, _dp, _dp, ctypes.c_int]
+        lib.oracle_attention.restype = None
+        lib.oracle_attention.argtypes = [
+            _dp, _dp, _dp, _dp, _ip, ctypes.POINTER(ctypes.c_int64),
+            ctypes.POINTER(ctypes.c_int64), ctypes.c_int,
+            ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, _dp, _dp,
+            ctypes.c_double, ctypes.c_int, ctypes.c_double, ctypes.c_double, _dp, _dp, _dp,
+            ctypes.c_int]
         lib.oracle_gated_rmsnorm.restype = None
         lib.oracle_gated_rmsnorm.argtypes = [
             _dp, _dp, _dp, ctypes.c_int64, ctypes.c_int, ctypes.c_double, _dp,
@@ -175,3 +185,49 @@ def gated_rmsnorm(x, z, w, eps=1e-6, threads=0):
     _load().oracle_gated_rmsnorm(_ptr(x2), _ptr(z2), _ptr(w), x2.shape[0], dim,
                                  float(eps), _ptr(y), int(threads))
     return y.reshape(shape)
+
+
+def attention(q, k, v, gate, wq, wk, cu_seqlens=None, pos0=None, positions=None,
+              eps=1e-6, rope_dims=64, rope_base=1e7, scale=None, threads=0):
+    """Global-attention layer (fp64): per token and head, q and k RMS-normed
+    over the head dim with weights wq / wk, rotary (rotate-half pairs
+    (i, i + R/2), theta = p * base^(-2i/R)) on the first ``rope_dims`` dims,
+    causal softmax attention with query head h reading kv head h // (Hq/Hkv),
+    output times sigmoid(gate).
+
+    Pair i turns by the token's position on axis i % 3 (text, height, width):
+    ``positions`` [3, T] gives them; without it every axis carries the token's
+    index within its sequence plus ``pos0[n]`` (0 without pos0).
+
+    q, gate [T, Hq, D]; k, v [T, Hkv, D]; wq, wk [D]; pos0 [N] or None.
+    Returns (out [T, Hq, D], q_rot [T, Hq, D], k_rot [T, Hkv, D]); scale
+    defaults to D**-0.5."""
+    q, k, v, gate, wq, wk = (_f64(a) for a in (q, k, v, gate, wq, wk))
+    T, Hq, D = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (T, Hkv, D) or v.shape != (T, Hkv, D) or gate.shape != q.shape \
+            or Hq % Hkv or wq.shape != (D,) or wk.shape != (D,) or rope_dims % 2 \
+            or rope_dims > D:
+        raise ValueError("inconsistent shapes")
+    cu = _cu(cu_seqlens, T)
+    N = len(cu) - 1
+    p0 = None
+    if pos0 is not None:
+        p0 = np.ascontiguousarray(np.asarray(pos0, dtype=np.int64))
+    p3 = None
+    if positions is not None:
+        p3 = np.ascontiguousarray(np.asarray(positions, dtype=np.int64))
+        if p3.shape != (3, T):
+            raise ValueError("positions must be [3, T]")
+    out = np.zeros_like(q)
+    qr = np.zeros_like(q)
+    kr = np.zeros_like(k)
+    i64 = ctypes.POINTER(ctypes.c_int64)
+    _load().oracle_attention(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(gate), cu.ctypes.data_as(_ip),
+        None if p0 is None else p0.ctypes.data_as(i64),
+        None if p3 is None else p3.ctypes.data_as(i64), N, T, Hq,
+        Hkv, D, _ptr(wq), _ptr(wk), float(eps), int(rope_dims), float(rope_base),
+        float(D ** -0.5 if scale is None else scale), _ptr(out), _ptr(qr), _ptr(kr),
+        int(threads))
+    return out, qr, kr

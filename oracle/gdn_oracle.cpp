@@ -23,6 +23,16 @@
 //  sequence's start is the carried conv state (zeros when absent); the gated
 //  RMS-norm normalises first and then multiplies by w and SiLU(z).
 //
+//  The hybrid decoder's other layer type, global attention (model card,
+//  section 架构, rows 全局注意力 and 位置编码; commentary section 二.1): 24
+//  query / 4 key-value heads (GQA 6 : 1), head dim 256, RMS-norm on q and k,
+//  a sigmoid gate on the output, and three-axis rotary (text / height /
+//  width, interleaved 11 : 11 : 10, base 1e7) on the first 64 dims of each
+//  head. Read plainly: the norms are per head over the head dim with a weight
+//  vector; rotary pair i couples dims i and i + 32 (rotate-half); the gate is
+//  elementwise on each head's output; softmax scale is D^-1/2; attention is
+//  causal within each packed sequence.
+//
 // Every function is the plain definition written out in fp64, with no
 // blocking, fusion or reordering beyond it. Work is split over independent
 // (sequence, value head) pairs with std::thread only.
@@ -208,6 +218,96 @@ void oracle_gated_rmsnorm(const double* x, const double* z, const double* w,
     double inv = 1.0 / std::sqrt(ss / dim + eps);
     for (int c = 0; c < dim; ++c)
       y[r * dim + c] = xr[c] * inv * w[c] * silu(zr[c]);
+  });
+}
+
+// Global-attention layer of the same hybrid decoder (the fourth layer of each
+// four: "Agnes-3.0-Flash Preview" model card, 架构 table; leaderboard
+// commentary, section 二.1): 24 query / 4 key-value heads (each kv head shared
+// by 6 query heads), head dim 256, RMS-norm on q and on k, rotary position
+// encoding on the first 64 dims (base 1e7; the three-axis interleaved form of
+// the pages gives every frequency the same angle when the text, height and
+// width positions coincide, as they do for text tokens), causal softmax
+// attention, and a sigmoid gate on the output. Per sequence n (tokens
+// cu[n] .. cu[n+1]-1, position p = t - cu[n] + pos0[n]) and token t:
+//   qn[h] = q[t,h] / sqrt(mean(q[t,h]^2) + eps) * wq          (per head, D dims)
+//   kn[g] = k[t,g] / sqrt(mean(k[t,g]^2) + eps) * wk
+//   rotary on dims [0, R): for i < R/2, theta = p * base^(-2i/R),
+//     (x_i, x_{i+R/2}) <- (x_i cos theta - x_{i+R/2} sin theta,
+//                          x_{i+R/2} cos theta + x_i sin theta)
+//   for query head h (kv head g = h / (Hq/Hkv)):
+//     s_j = scale * qr[t,h] . kr[j,g] for the sequence's tokens j <= t
+//     o[t,h] = sum_j softmax(s)_j v[j,g]
+//   out[t,h] = o[t,h] * sigmoid(gate[t,h])                      (elementwise)
+// q_rot / k_rot (nullable) receive qr and kr.
+// Layouts: q, gate, out, q_rot [T, Hq, D]; k, v, k_rot [T, Hkv, D]; wq, wk [D];
+// pos0 [N] (nullable: 0).
+void oracle_attention(const double* q, const double* k, const double* v,
+                      const double* gate, const int32_t* cu_seqlens, const int64_t* pos0,
+                      const int64_t* pos3, int N, int64_t T, int Hq, int Hkv, int D,
+                      const double* wq, const double* wk, double eps, int R, double base,
+                      double scale, double* out, double* q_rot, double* k_rot, int threads) {
+  // Per-head RMS-norm with weight w, then rotary on dims [0, R): pair i couples
+  // dims i and i + R/2 and turns by theta_i = p * base^(-2i/R), where p is the
+  // token's position on axis i mod 3 (text, height, width interleaved, which
+  // gives the 11 : 11 : 10 split of the 32 pairs at R = 64). Without explicit
+  // per-axis positions all three axes carry the index within the sequence.
+  std::vector<double> qr((size_t)T * Hq * D), kr((size_t)T * Hkv * D);
+  auto prep = [&](const double* x, const double* w, double* y, const int64_t* p) {
+    double ss = 0.0;
+    for (int d = 0; d < D; ++d) ss += x[d] * x[d];
+    const double inv = 1.0 / std::sqrt(ss / D + eps);
+    for (int d = 0; d < D; ++d) y[d] = x[d] * inv * w[d];
+    for (int i = 0; i < R / 2; ++i) {
+      const double theta = (double)p[i % 3] * std::pow(base, -2.0 * i / R);
+      const double c = std::cos(theta), s = std::sin(theta);
+      const double a = y[i], b = y[i + R / 2];
+      y[i] = a * c - b * s;
+      y[i + R / 2] = b * c + a * s;
+    }
+  };
+  int nt = resolve_threads(threads, N);
+  parallel_for(N, nt, [&](int64_t n) {
+    for (int64_t t = cu_seqlens[n]; t < cu_seqlens[n + 1]; ++t) {
+      int64_t p[3];
+      for (int ax = 0; ax < 3; ++ax)
+        p[ax] = pos3 ? pos3[ax * T + t] : t - cu_seqlens[n] + (pos0 ? pos0[n] : 0);
+      for (int h = 0; h < Hq; ++h) prep(q + (t * Hq + h) * D, wq, qr.data() + (t * Hq + h) * D, p);
+      for (int g = 0; g < Hkv; ++g) prep(k + (t * Hkv + g) * D, wk, kr.data() + (t * Hkv + g) * D, p);
+    }
+  });
+  if (q_rot) std::memcpy(q_rot, qr.data(), sizeof(double) * qr.size());
+  if (k_rot) std::memcpy(k_rot, kr.data(), sizeof(double) * kr.size());
+  // causal softmax attention per (sequence, query head)
+  const int group = Hq / Hkv;
+  const int64_t pairs = (int64_t)N * Hq;
+  nt = resolve_threads(threads, pairs);
+  parallel_for(pairs, nt, [&](int64_t idx) {
+    const int n = (int)(idx / Hq), h = (int)(idx % Hq), g = h / group;
+    const int64_t s0 = cu_seqlens[n], s1 = cu_seqlens[n + 1];
+    std::vector<double> sc((size_t)(s1 - s0)), o(D);
+    for (int64_t t = s0; t < s1; ++t) {
+      const double* qt = qr.data() + (t * Hq + h) * D;
+      double m = -INFINITY;
+      for (int64_t j = s0; j <= t; ++j) {
+        const double* kj = kr.data() + (j * Hkv + g) * D;
+        double acc = 0.0;
+        for (int d = 0; d < D; ++d) acc += qt[d] * kj[d];
+        sc[j - s0] = scale * acc;
+        if (sc[j - s0] > m) m = sc[j - s0];
+      }
+      double l = 0.0;
+      for (int64_t j = s0; j <= t; ++j) l += std::exp(sc[j - s0] - m);
+      for (int d = 0; d < D; ++d) o[d] = 0.0;
+      for (int64_t j = s0; j <= t; ++j) {
+        const double pj = std::exp(sc[j - s0] - m) / l;
+        const double* vj = v + (j * Hkv + g) * D;
+        for (int d = 0; d < D; ++d) o[d] += pj * vj[d];
+      }
+      const double* gt = gate + (t * Hq + h) * D;
+      double* ot = out + (t * Hq + h) * D;
+      for (int d = 0; d < D; ++d) ot[d] = o[d] / (1.0 + std::exp(-gt[d]));
+    }
   });
 }
 

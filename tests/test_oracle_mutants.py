@@ -31,10 +31,20 @@ MUTANTS = {
     "rms_sum_not_mean": ("std::sqrt(ss / dim + eps);", "std::sqrt(ss + eps);"),
     "gate_without_silu": ("* w[c] * silu(zr[c]);", "* w[c] * zr[c];"),
     "bias_dropped": ("double acc = bias ? bias[c] : 0.0;", "double acc = 0.0;"),
+    "rope_turns_backwards": ("y[i + R / 2] = b * c + a * s;", "y[i + R / 2] = b * c - a * s;"),
+    "rope_half_frequency": ("std::pow(base, -2.0 * i / R);", "std::pow(base, -1.0 * i / R);"),
+    "rope_one_axis": ("(double)p[i % 3] * std::pow", "(double)p[0] * std::pow"),
+    "qk_norm_sum_not_mean": ("1.0 / std::sqrt(ss / D + eps);", "1.0 / std::sqrt(ss + eps);"),
+    "qk_norm_weight_dropped": ("y[d] = x[d] * inv * w[d];", "y[d] = x[d] * inv;"),
+    "attention_interleaved_gqa": ("g = h / group;", "g = h % Hkv;"),
+    "softmax_unshifted_sum": ("l += std::exp(sc[j - s0] - m);", "l += std::exp(sc[j - s0]);"),
+    "gate_sign": ("o[d] / (1.0 + std::exp(-gt[d]));", "o[d] / (1.0 + std::exp(gt[d]));"),
+    "mask_drops_diagonal": ("const double pj = std::exp(sc[j - s0] - m) / l;",
+                            "const double pj = j == t && t > s0 ? 0.0 : std::exp(sc[j - s0] - m) / l;"),
 }
 
 PIN_FILES = ["tests/test_oracle_recurrence.py", "tests/test_oracle_conv_norm.py",
-             "tests/test_oracle_chunked.py"]
+             "tests/test_oracle_chunked.py", "tests/test_oracle_attention.py"]
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
