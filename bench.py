@@ -16,7 +16,12 @@ The same run times, under their own keys:
                       RMS-norm, fp32 state [256,48,128,128];
   long_context        T=262144 as 64 calls of 4096 tokens with the recurrent
                       state and the conv history carried between calls (one
-                      step = all 64 calls), unflushed and L2-flushed.
+                      step = all 64 calls), unflushed and L2-flushed;
+  attention_prefill   the decoder's global-attention layer (24 query / 4
+                      key-value heads, head dim 256, q/k RMS-norm, rotary,
+                      sigmoid gate) over the same B=1, T=8192 prompt;
+  attention_decode    that layer's decode step for 256 sequences holding 4096
+                      cached tokens each, one token per sequence per step.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
                     [--shard replicas|heads]
@@ -74,6 +79,24 @@ CONV_CH = 2 * H_K * D + H_V * D
 FUSED_DECODE_BYTES_PER_TOKEN = (2 * H_V * D * D * 4 + 2 * CONV_CH + 2 * 3 * 2 * CONV_CH
                                 + 2 * 2 * H_V * D + 2 * 2 * H_V)
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+# Global-attention layer: S = Q K^T and O = P V over the causal triangle,
+# 2 * 2 * d flops per (query, key) pair and query head.
+A_HQ, A_HKV, A_D = 24, 4, 256
+A_CTX = 4096                 # cached tokens per sequence at the first decode step
+A_LMAX = A_CTX + 256         # cache rows per slot (room for warm-up + timed steps)
+
+
+def attn_prefill_flop(T, H_q=A_HQ):
+    return 4 * A_D * H_q * T * (T + 1) / 2
+
+
+def attn_decode_bytes(N, L, H_q=A_HQ, H_kv=A_HKV):
+    """Algorithmic bytes of one decode step with L cached tokens per sequence:
+    read the L + 1 fp16 key and value rows (the new one included), write the
+    new row, read q, k, v, gate (bf16), write o (bf16)."""
+    row = H_kv * A_D * 2                       # one token's fp16 keys (or values)
+    inputs = 2 * A_D * (2 * H_q + 2 * H_kv)    # q, gate, k, v in bf16
+    return N * (2 * (L + 1) * row + 2 * row + inputs + 2 * A_D * H_q)
 
 
 def load_peaks():
@@ -388,6 +411,89 @@ class DecodeWorkload:
         g.gdn_gated_rmsnorm(self.o, st["z"], L.nw, eps=1e-6, y=self.out)
 
 
+class AttentionPrefillWorkload:
+    """The global-attention layer over the B=1, T=8192 prompt: q, k, v, gate
+    bf16 N(0, 1), norm weights 1 + N(0, 0.01); one gdn_attention_prefill call
+    (q/k norm + rotary launch, attention launch) per step."""
+
+    def __init__(self, gdn, dev, seed, kv=(0, A_HKV)):
+        self.gdn = gdn
+        G = A_HQ // A_HKV
+        self.H_kv = kv[1] - kv[0]
+        self.H_q = self.H_kv * G
+        p = gi.attention_inputs(T_PREFILL, seed=seed)
+        qh = slice(kv[0] * G, kv[1] * G)
+        self.q = p["q"][:, qh].contiguous().to(dev)
+        self.gate = p["gate"][:, qh].contiguous().to(dev)
+        self.k = p["k"][:, kv[0]:kv[1]].contiguous().to(dev)
+        self.v = p["v"][:, kv[0]:kv[1]].contiguous().to(dev)
+        self.wq, self.wk = p["q_norm_w"].to(dev), p["k_norm_w"].to(dev)
+        self.cu = torch.tensor([0, T_PREFILL], dtype=torch.int32, device=dev)
+        self.o = torch.empty_like(self.q)
+        self.k_rot = torch.empty(self.k.shape, dtype=torch.float16, device=dev)
+        self.v_h = torch.empty_like(self.k_rot)
+        self.ws = torch.empty(gdn.load().gdn_attention_prefill_workspace(T_PREFILL, self.H_q, A_D),
+                              dtype=torch.uint8, device=dev)
+        self.flop = attn_prefill_flop(T_PREFILL, self.H_q)
+
+    def step(self, i, ev=None):
+        if ev is not None:
+            ev[0].record()
+        self.gdn.gdn_attention_prefill(self.q, self.k, self.v, self.gate, self.wq, self.wk,
+                                       self.cu, o=self.o, k_rot=self.k_rot, v_h=self.v_h,
+                                       workspace=self.ws)
+        if ev is not None:
+            ev[1].record()
+
+
+class AttentionDecodeWorkload:
+    """256 sequences in permuted pool slots, A_CTX cached tokens each (fp16
+    keys and values drawn N(0, 1) on the device, seeded); each step decodes
+    one new token per sequence (q, k, v, gate bf16 N(0, 1)), which appends to
+    the caches and advances cache_len."""
+
+    def __init__(self, gdn, dev, seed, steps, kv=(0, A_HKV)):
+        self.gdn = gdn
+        G = A_HQ // A_HKV
+        self.H_kv = kv[1] - kv[0]
+        self.H_q = self.H_kv * G
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(1000 + seed)
+        shape = (N_DECODE, A_LMAX, self.H_kv, A_D)
+        self.kc = torch.randn(shape, generator=gen, device=dev, dtype=torch.float16)
+        self.vc = torch.randn(shape, generator=gen, device=dev, dtype=torch.float16)
+        self.idx = torch.from_numpy(
+            np.random.default_rng(seed).permutation(N_DECODE).astype(np.int32)).to(dev)
+        self.len = torch.full((N_DECODE,), A_CTX, dtype=torch.int32, device=dev)
+        self.inputs = []
+        for s in range(min(steps, 16)):
+            a = gi.attention_inputs(N_DECODE, seed=seed, tag=("attn_decode", s))
+            self.inputs.append({k: (v[:, kv[0] * G:kv[1] * G] if k in ("q", "gate") else
+                                    v[:, kv[0]:kv[1]] if k in ("k", "v") else v)
+                                .contiguous().to(dev) for k, v in a.items()})
+        self.o = torch.empty((N_DECODE, self.H_q, A_D), dtype=torch.bfloat16, device=dev)
+        self.ws = torch.empty(gdn.load().gdn_attention_decode_workspace(N_DECODE, self.H_q,
+                                                                        A_LMAX, A_D),
+                              dtype=torch.uint8, device=dev)
+
+    def reset(self):
+        self.len.fill_(A_CTX)
+
+    def bytes_for(self, first_len, steps):
+        return sum(attn_decode_bytes(N_DECODE, first_len + s, self.H_q, self.H_kv)
+                   for s in range(steps))
+
+    def step(self, s, ev=None):
+        st = self.inputs[s % len(self.inputs)]
+        if ev is not None:
+            ev[0].record()
+        self.gdn.gdn_attention_decode(st["q"], st["k"], st["v"], st["gate"], st["q_norm_w"],
+                                      st["k_norm_w"], self.kc, self.vc, self.len,
+                                      cache_idx=self.idx, o=self.o, workspace=self.ws)
+        if ev is not None:
+            ev[1].record()
+
+
 class RankGroup:
     """Barrier and max-over-ranks around the timed regions; no-ops at one rank.
     `dist` is torch.distributed with an initialised process group (NCCL on the
@@ -589,6 +695,22 @@ def gpu_arm(args):
         lf_ms, lf_kms = max_over_ranks(sum(seg_ms)), max_over_ranks(sum(seg_kern))
         l_tokens, l_flop = lc.tokens, lc.flop
         del lc
+
+        # global-attention layer; head shards split its 4 key-value heads
+        akv = (0, A_HKV)
+        if heads and A_HKV % world == 0:
+            akv = (rank * A_HKV // world, (rank + 1) * A_HKV // world)
+        apre = AttentionPrefillWorkload(gdn, dev, seed, akv)
+        a_step, a_kern = timed_loop(apre.step, args.steps, args.warmup, barrier)
+        a_ms, a_kms = mean_max(a_step), mean_max(a_kern)
+        a_flop = apre.flop
+        del apre
+        adec = AttentionDecodeWorkload(gdn, dev, seed, DECODE_STEPS, akv)
+        adec.reset()
+        ad_step, ad_kern = timed_loop(adec.step, DECODE_STEPS, args.warmup, barrier)
+        ad_ms, ad_kms = mean_max(ad_step), mean_max(ad_kern)
+        ad_bytes = adec.bytes_for(A_CTX + args.warmup, DECODE_STEPS) / DECODE_STEPS
+        del adec
     e2e_ms, h2d, d2h = e2e_prefill(pre, dev, max(4, args.steps), 2)
     e2e_ms = max_over_ranks(e2e_ms)
 
@@ -687,6 +809,29 @@ def gpu_arm(args):
             "gpu_launches": 4 * N_SEG * lsteps,
         },
     }
+    a_units = 1 if (heads and A_HKV % world == 0) else world
+    ad_ach = ad_bytes / (ad_kms * 1e-3) / 1e9
+    line["attention_prefill"] = {
+        "workload": "global-attention layer (24 query / 4 key-value heads, head dim 256, q/k "
+                    "RMS-norm, rotary on 64 dims, causal, sigmoid gate), B=1, T=8192; one "
+                    "gdn_attention_prefill call (norm+rotary launch, attention launch)",
+        "value": throughput(T_PREFILL, a_units, a_ms), "unit": "tokens/s", "ms_per_step": a_ms,
+        "roofline": dict(tensor_roofline("gdn_attention_prefill", a_flop, a_kms, peaks, peak_src,
+                                         kernel_traffic("attention") if not heads else None),
+                         dtype="fp16 operands (same dense rate as bf16)",
+                         kernel_ms_includes="the q/k norm + rotary launch"),
+        "gpu_launches": 2 * args.steps}
+    line["attention_decode"] = {
+        "workload": f"global-attention decode: {N_DECODE} sequences in permuted pool slots, "
+                    f"{A_CTX} cached tokens each at the first step (+1 per step), fp16 KV "
+                    "cache, one token per sequence per step",
+        "value": throughput(N_DECODE, a_units, ad_ms), "unit": "tokens/s", "ms_per_step": ad_ms,
+        "roofline": {"kernel": "gdn_attention_decode", "bound": "hbm", "achieved": ad_ach,
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": ad_ach / peaks["hbm_gbs"],
+                     "peak_source": f"{peak_src} HBM copy",
+                     "traffic": kernel_traffic("attention_decode") if not heads else None,
+                     "algorithmic_bytes_per_launch": ad_bytes, "kernel_ms": ad_kms},
+        "gpu_launches": 3 * DECODE_STEPS}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cb, ref_out, nheads = cpu_baseline(args.cpu_budget_s)
         line["cpu_baseline"] = cb
@@ -859,6 +1004,14 @@ def profile_case(args):
         y = torch.empty((N, gi.CONV_CHANNELS), dtype=torch.bfloat16, device=dev)
         run = lambda: gdn.gdn_conv1d_silu(x, w, cu, conv_state_in=cache, conv_state_out=cache,
                                           y=y)
+    elif name == "attn":
+        wl = AttentionPrefillWorkload(gdn, dev, 0) if T == T_PREFILL else None
+        if wl is None:
+            raise SystemExit("attn case runs the T=8192 workload (--t 8192)")
+        run = lambda: wl.step(0)
+    elif name == "adec":
+        wl = AttentionDecodeWorkload(gdn, dev, 0, 1)
+        run = lambda: (wl.reset(), wl.step(0))
     else:
         raise SystemExit(f"unknown profile case {name}")
     torch.cuda.synchronize()
@@ -871,7 +1024,8 @@ def profile_case(args):
     print(f"{name}: {s.elapsed_time(e) / args.launches:.4f} ms per launch")
 
 
-PROFILE_CASES = ("decode", "dlayer", "prefill", "layer", "varlen", "conv", "norm", "dconv")
+PROFILE_CASES = ("decode", "dlayer", "prefill", "layer", "varlen", "conv", "norm", "dconv",
+                 "attn", "adec")
 
 
 def main():

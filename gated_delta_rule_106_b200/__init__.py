@@ -27,6 +27,8 @@ __all__ = ["GDN_BF16", "GDN_F32", "GdnError", "library_path", "load",
            "gdn_chunked_prefill_status", "gdn_set_wait_limit_ns", "GDN_ERR_TIMEOUT",
            "gdn_decode_step",
            "gdn_gated_rmsnorm", "gdn_status_string", "gdn_version",
+           "gdn_attention_prefill", "gdn_attention_decode", "gdn_attention_status",
+           "ATTN_H_Q", "ATTN_H_KV", "ATTN_HEAD_DIM",
            "H_K", "H_V", "HEAD_DIM", "CHUNK"]
 
 GDN_BF16 = 0
@@ -46,6 +48,15 @@ _f32 = ctypes.c_float
 
 # name -> (restype, argtypes)
 _SIGNATURES = {
+    "gdn_attention_prefill_workspace": (ctypes.c_size_t, [_i64, _int, _int]),
+    "gdn_attention_prefill": (_int, [_vp, _i64, _vp, _i64, _vp, _i64, _vp, _i64, _vp, _vp, _int,
+                                     _vp, _vp, _vp, _int, _i64, _int, _int, _int, _f32, _int,
+                                     _f32, _f32, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
+    "gdn_attention_decode_workspace": (ctypes.c_size_t, [_int, _int, _int, _int]),
+    "gdn_attention_decode": (_int, [_vp, _i64, _vp, _i64, _vp, _i64, _vp, _i64, _vp, _vp, _int,
+                                    _vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _int,
+                                    _f32, _int, _f32, _f32, _vp, _vp, ctypes.c_size_t, _vp]),
+    "gdn_attention_status": (_int, [_vp, _vp]),
     "gdn_status_string": (ctypes.c_char_p, [_int]),
     "gdn_version": (ctypes.c_char_p, []),
     "gdn_conv1d_silu": (_int, [_vp, _i64, _int, _vp, _int, _vp, _int, _int, _f32,
@@ -409,3 +420,100 @@ def gdn_gated_rmsnorm(x, z, w, *, eps=1e-6, y=None, y_dtype=None, stream=None):
         _dtype_code(w.dtype), rows, dim, eps, _ptr(y), _dtype_code(y.dtype),
         _stream(stream, x.device)))
     return y
+
+
+# ------------------------------------------------------------ global attention
+ATTN_H_Q, ATTN_H_KV, ATTN_HEAD_DIM = 24, 4, 256
+
+
+def _head_rows(t, n, H, name):
+    """[n, H, 256] bf16 with dense heads and any row stride: returns the stride."""
+    _expect(t, (n, H, ATTN_HEAD_DIM), name, torch.bfloat16, contiguous=False)
+    return _row_stride(t)
+
+
+def gdn_attention_prefill(q, k, v, gate, q_norm_w, k_norm_w, cu_seqlens, *, positions=None,
+                          pos0=None, eps=1e-6, rope_dims=64, rope_base=1e7, scale=None,
+                          o=None, k_rot=None, v_h=None, workspace=None, stream=None):
+    """Global-attention layer over packed prompts: q/k RMS-norm, rotary, causal
+    GQA attention, sigmoid output gate. q, gate [T, H_q, 256]; k, v [T, H_kv,
+    256] (bf16, any token stride); norm weights [256] (bf16 or fp32, one
+    dtype); positions [3, T] int32 or pos0 [N] int32. Returns (o, k_rot, v_h):
+    o bf16; k_rot, v_h the cache rows in fp16 (normed rotated keys, values)."""
+    T, H_q, _ = q.shape
+    H_kv = k.shape[1]
+    N = cu_seqlens.numel() - 1
+    qs = _head_rows(q, T, H_q, "q")
+    ks = _head_rows(k, T, H_kv, "k")
+    vs = _head_rows(v, T, H_kv, "v")
+    gs = _head_rows(gate, T, H_q, "gate")
+    _expect(q_norm_w, (ATTN_HEAD_DIM,), "q_norm_w")
+    _expect(k_norm_w, (ATTN_HEAD_DIM,), "k_norm_w", q_norm_w.dtype)
+    _expect(cu_seqlens, (N + 1,), "cu_seqlens", torch.int32)
+    _expect(positions, (3, T), "positions", torch.int32)
+    _expect(pos0, (N,), "pos0", torch.int32)
+    _expect(o, (T, H_q, ATTN_HEAD_DIM), "o", torch.bfloat16)
+    _expect(k_rot, (T, H_kv, ATTN_HEAD_DIM), "k_rot", torch.float16)
+    _expect(v_h, (T, H_kv, ATTN_HEAD_DIM), "v_h", torch.float16)
+    if o is None:
+        o = torch.empty((T, H_q, ATTN_HEAD_DIM), dtype=torch.bfloat16, device=q.device)
+    if k_rot is None:
+        k_rot = torch.empty((T, H_kv, ATTN_HEAD_DIM), dtype=torch.float16, device=q.device)
+    if v_h is None:
+        v_h = torch.empty((T, H_kv, ATTN_HEAD_DIM), dtype=torch.float16, device=q.device)
+    need = load().gdn_attention_prefill_workspace(T, H_q, ATTN_HEAD_DIM)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check("gdn_attention_prefill", load().gdn_attention_prefill(
+        _ptr(q), qs, _ptr(k), ks, _ptr(v), vs, _ptr(gate), gs, _ptr(q_norm_w), _ptr(k_norm_w),
+        _dtype_code(q_norm_w.dtype), _ptr(cu_seqlens), _ptr(positions), _ptr(pos0), N, T, H_q,
+        H_kv, ATTN_HEAD_DIM, eps, rope_dims, rope_base,
+        ATTN_HEAD_DIM ** -0.5 if scale is None else scale, _ptr(o), _ptr(k_rot), _ptr(v_h),
+        _ptr(workspace), ws_bytes, _stream(stream, q.device)))
+    return o, k_rot, v_h
+
+
+def gdn_attention_decode(q, k, v, gate, q_norm_w, k_norm_w, k_cache, v_cache, cache_len, *,
+                         cache_idx=None, positions=None, eps=1e-6, rope_dims=64, rope_base=1e7,
+                         scale=None, o=None, workspace=None, stream=None):
+    """One decode step of the global-attention layer for N sequences: appends
+    the new rotated k and v at row cache_len[n] of slot cache_idx[n] of the
+    fp16 caches [P, L_max, H_kv, 256], attends over rows 0..cache_len[n], and
+    advances cache_len (int32 [N], on the device) by one. Returns o [N, H_q, 256]."""
+    N, H_q, _ = q.shape
+    H_kv = k.shape[1]
+    P, L_max = k_cache.shape[0], k_cache.shape[1]
+    qs = _head_rows(q, N, H_q, "q")
+    ks = _head_rows(k, N, H_kv, "k")
+    vs = _head_rows(v, N, H_kv, "v")
+    gs = _head_rows(gate, N, H_q, "gate")
+    _expect(q_norm_w, (ATTN_HEAD_DIM,), "q_norm_w")
+    _expect(k_norm_w, (ATTN_HEAD_DIM,), "k_norm_w", q_norm_w.dtype)
+    _expect(k_cache, (P, L_max, H_kv, ATTN_HEAD_DIM), "k_cache", torch.float16)
+    _expect(v_cache, (P, L_max, H_kv, ATTN_HEAD_DIM), "v_cache", torch.float16)
+    _expect(cache_len, (N,), "cache_len", torch.int32)
+    _expect(cache_idx, (N,), "cache_idx", torch.int32)
+    _expect(positions, (3, N), "positions", torch.int32)
+    _expect(o, (N, H_q, ATTN_HEAD_DIM), "o", torch.bfloat16)
+    if o is None:
+        o = torch.empty((N, H_q, ATTN_HEAD_DIM), dtype=torch.bfloat16, device=q.device)
+    need = load().gdn_attention_decode_workspace(N, H_q, L_max, ATTN_HEAD_DIM)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check("gdn_attention_decode", load().gdn_attention_decode(
+        _ptr(q), qs, _ptr(k), ks, _ptr(v), vs, _ptr(gate), gs, _ptr(q_norm_w), _ptr(k_norm_w),
+        _dtype_code(q_norm_w.dtype), _ptr(k_cache), _ptr(v_cache), _ptr(cache_idx),
+        _ptr(cache_len), _ptr(positions), N, P, L_max, H_q, H_kv, ATTN_HEAD_DIM, eps,
+        rope_dims, rope_base, ATTN_HEAD_DIM ** -0.5 if scale is None else scale, _ptr(o),
+        _ptr(workspace), ws_bytes, _stream(stream, q.device)))
+    return o
+
+
+def gdn_attention_status(workspace, stream=None) -> int:
+    """Waits for `stream`, then returns the status the last attention call left
+    in `workspace`: 0, GDN_ERR_TIMEOUT, or GDN_ERR_INVALID_ARG (a decode
+    sequence with an out-of-range slot or length)."""
+    return int(load().gdn_attention_status(_ptr(workspace), _stream(stream, workspace.device)))
+

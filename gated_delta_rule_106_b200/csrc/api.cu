@@ -337,4 +337,116 @@ gdn_status gdn_gated_rmsnorm(const void* x, gdn_dtype x_dtype, const void* z,
   return from_cuda(gdn::launch_gated_rmsnorm(a));
 }
 
+// ---------------------------------------------------------- global attention
+
+namespace {
+
+constexpr int kAttnHeadDim = 256;
+
+gdn_status check_attn_common(int H_q, int H_kv, int head_dim, int rope_dims, float rope_base,
+                             float eps, gdn_dtype w_dtype) {
+  if (head_dim != kAttnHeadDim) return GDN_ERR_UNSUPPORTED;
+  if (H_q <= 0 || H_kv <= 0 || H_q % H_kv != 0) return GDN_ERR_INVALID_ARG;
+  if (rope_dims < 0 || rope_dims > 64 || rope_dims % 2 != 0) return GDN_ERR_UNSUPPORTED;
+  if (rope_dims > 0 && !(rope_base > 1.0f)) return GDN_ERR_INVALID_ARG;
+  if (!(eps >= 0.0f) || !valid_dtype(w_dtype)) return GDN_ERR_INVALID_ARG;
+  return GDN_OK;
+}
+
+bool attn_stride_ok(int64_t stride, int H) {
+  return stride >= (int64_t)H * kAttnHeadDim && stride % 8 == 0;
+}
+
+}  // namespace
+
+size_t gdn_attention_prefill_workspace(int64_t T_total, int H_q, int head_dim) {
+  if (T_total < 0 || H_q <= 0 || head_dim != kAttnHeadDim) return 0;
+  return gdn::attention_prefill_workspace(T_total, H_q);
+}
+
+gdn_status gdn_attention_prefill(const void* q, int64_t q_row_stride, const void* k,
+                                 int64_t k_row_stride, const void* v, int64_t v_row_stride,
+                                 const void* gate, int64_t gate_row_stride,
+                                 const void* q_norm_w, const void* k_norm_w, gdn_dtype w_dtype,
+                                 const int32_t* cu_seqlens, const int32_t* positions,
+                                 const int32_t* pos0, int N, int64_t T_total, int H_q, int H_kv,
+                                 int head_dim, float eps, int rope_dims, float rope_base,
+                                 float scale, void* o, void* k_rot, void* v_h, void* workspace,
+                                 size_t workspace_bytes, cudaStream_t stream) {
+  gdn_status st = check_attn_common(H_q, H_kv, head_dim, rope_dims, rope_base, eps, w_dtype);
+  if (st != GDN_OK) return st;
+  if ((H_q / H_kv) % 2 != 0) return GDN_ERR_UNSUPPORTED;   // query heads go in pairs
+  if (N < 0 || T_total < 0 || T_total > (int64_t)1 << 30) return GDN_ERR_INVALID_ARG;
+  if (N == 0 && T_total > 0) return GDN_ERR_INVALID_ARG;
+  if (!attn_stride_ok(q_row_stride, H_q) || !attn_stride_ok(gate_row_stride, H_q) ||
+      !attn_stride_ok(k_row_stride, H_kv) || !attn_stride_ok(v_row_stride, H_kv))
+    return GDN_ERR_MISALIGNED;
+  if (T_total == 0) return GDN_OK;
+  if (!q || !k || !v || !gate || !q_norm_w || !k_norm_w || !cu_seqlens || !o || !k_rot ||
+      !v_h || !workspace)
+    return GDN_ERR_INVALID_ARG;
+  if (workspace_bytes < gdn::attention_prefill_workspace(T_total, H_q)) return GDN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(gate) || !aligned16(o) ||
+      !aligned16(k_rot) || !aligned16(v_h) || !aligned16(workspace))
+    return GDN_ERR_MISALIGNED;
+  const int wb = gdn::elem_bytes(w_dtype);
+  if (!aligned_to(q_norm_w, wb) || !aligned_to(k_norm_w, wb)) return GDN_ERR_MISALIGNED;
+  gdn::AttnPrefillArgs a{q, k, v, gate, q_row_stride, k_row_stride, v_row_stride,
+                         gate_row_stride, q_norm_w, k_norm_w, w_dtype, cu_seqlens, positions,
+                         pos0, N, T_total, H_q, H_kv, eps, rope_dims, rope_base, scale, o,
+                         k_rot, v_h, workspace, stream};
+  return from_cuda(gdn::launch_attention_prefill(a));
+}
+
+size_t gdn_attention_decode_workspace(int N, int H_q, int L_max, int head_dim) {
+  if (N < 0 || H_q <= 0 || L_max <= 0 || head_dim != kAttnHeadDim) return 0;
+  return gdn::attention_decode_workspace(N, H_q, L_max);
+}
+
+gdn_status gdn_attention_decode(const void* q, int64_t q_row_stride, const void* k,
+                                int64_t k_row_stride, const void* v, int64_t v_row_stride,
+                                const void* gate, int64_t gate_row_stride,
+                                const void* q_norm_w, const void* k_norm_w, gdn_dtype w_dtype,
+                                void* k_cache, void* v_cache, const int32_t* cache_idx,
+                                int32_t* cache_len, const int32_t* positions, int N, int P,
+                                int L_max, int H_q, int H_kv, int head_dim, float eps,
+                                int rope_dims, float rope_base, float scale, void* o,
+                                void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  gdn_status st = check_attn_common(H_q, H_kv, head_dim, rope_dims, rope_base, eps, w_dtype);
+  if (st != GDN_OK) return st;
+  const int G = H_q / H_kv;
+  if (G != 1 && G != 2 && G != 4 && G != 6 && G != 8) return GDN_ERR_UNSUPPORTED;
+  if (N < 0 || N > 65535 || P < 0 || L_max <= 0 || H_q > 65535) return GDN_ERR_INVALID_ARG;
+  if (!attn_stride_ok(q_row_stride, H_q) || !attn_stride_ok(gate_row_stride, H_q) ||
+      !attn_stride_ok(k_row_stride, H_kv) || !attn_stride_ok(v_row_stride, H_kv))
+    return GDN_ERR_MISALIGNED;
+  if (N == 0) return GDN_OK;
+  if (P == 0) return GDN_ERR_INVALID_ARG;
+  if (!q || !k || !v || !gate || !q_norm_w || !k_norm_w || !k_cache || !v_cache ||
+      !cache_len || !o || !workspace)
+    return GDN_ERR_INVALID_ARG;
+  if (workspace_bytes < gdn::attention_decode_workspace(N, H_q, L_max))
+    return GDN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(gate) || !aligned16(o) ||
+      !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(workspace))
+    return GDN_ERR_MISALIGNED;
+  const int wb = gdn::elem_bytes(w_dtype);
+  if (!aligned_to(q_norm_w, wb) || !aligned_to(k_norm_w, wb)) return GDN_ERR_MISALIGNED;
+  gdn::AttnDecodeArgs a{q, k, v, gate, q_row_stride, k_row_stride, v_row_stride,
+                        gate_row_stride, q_norm_w, k_norm_w, w_dtype, k_cache, v_cache,
+                        cache_idx, cache_len, positions, N, P, L_max, H_q, H_kv, eps,
+                        rope_dims, rope_base, scale, o, workspace, stream};
+  return from_cuda(gdn::launch_attention_decode(a));
+}
+
+gdn_status gdn_attention_status(const void* workspace, cudaStream_t stream) {
+  if (!workspace) return GDN_ERR_INVALID_ARG;
+  if (!aligned16(workspace)) return GDN_ERR_MISALIGNED;
+  int word = 0;
+  if (gdn::attention_status_word(workspace, stream, &word) != cudaSuccess) return GDN_ERR_CUDA;
+  if (word == 1) return GDN_ERR_TIMEOUT;
+  if (word == 2) return GDN_ERR_INVALID_ARG;
+  return GDN_OK;
+}
+
 }  // extern "C"

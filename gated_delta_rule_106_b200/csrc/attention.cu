@@ -1,0 +1,884 @@
+// Global-attention layer of the hybrid decoder: the quarter of its layers
+// that keep a KV cache (Agnes-3.0-Flash Preview model card, section 架构,
+// rows 全局注意力 and 位置编码; leaderboard commentary, section 二.1):
+// 24 query / 4 key-value heads (GQA 6 : 1), head dim 256, RMS-norm on q and k,
+// three-axis rotary (text / height / width interleaved, base 1e7) on the first
+// 64 dims, causal softmax attention, sigmoid gate on each head's output.
+//
+// Prefill is two launches:
+//  * attn_qk_prologue_kernel: per (token, head) row, RMS-norm with the weight
+//    vector and rotary (angles in fp64, shared by all heads of a token); writes
+//    rotated q into the workspace and rotated k where the caller wants its KV
+//    cache, both in fp16: after the norm every element is at most
+//    16 * sqrt(2) * max|w| in magnitude, well inside fp16's range, and fp16
+//    keeps three more significand bits than bf16 for the score product. The
+//    values go to fp16 as well (the value cache's dtype): a bf16 value in
+//    fp16's normal range converts exactly, so P V can take P in fp16 too.
+//  * attn_prefill_kernel: causal flash attention on tcgen05. A CTA owns 64
+//    query tokens of two query heads that share a key-value head (128 rows),
+//    walks 64-key blocks up to the diagonal, S = Q K^T (128 x 64, K = 256) and
+//    O += P V (128 x 256, K = 64), fp16 operands, accumulate in TMEM, the online softmax runs
+//    in 4 warps (one row per thread) and rescales O in TMEM only when a row's
+//    running max grows by more than 2^8; the epilogue divides by the row sum
+//    and applies sigmoid(gate).
+#include <cudaTypedefs.h>
+#include <math.h>
+
+#include "gdn_common.cuh"
+#include "launch.h"
+#include "sm100.cuh"
+
+namespace gdn {
+namespace {
+
+using namespace sm100;
+
+constexpr int kAD = 256;        // head dim of the attention layer
+constexpr int kTileTok = 64;    // query tokens per tile (two heads -> 128 rows)
+constexpr int kBlk = 64;        // keys per block
+constexpr uint64_t kAttnLimitNs = 2000000000ull;
+
+// --------------------------------------------------------------- prologue --
+
+constexpr int kProTok = 4;      // tokens per prologue CTA
+
+struct ProParams {
+  const __nv_bfloat16* q; const __nv_bfloat16* k; int64_t q_stride, k_stride;
+  const void* wq; const void* wk;
+  const int32_t* cu; int N; int64_t T;
+  const int32_t* positions;     // [3][T] or null
+  const int32_t* pos0;          // [N] or null
+  int Hq, Hkv; float eps; int R; double log2_base;
+  const __nv_bfloat16* v; int64_t v_stride;
+  __half* q_out; __half* k_out; __half* v_out;   // [T][H][256] dense
+};
+
+__device__ __forceinline__ float ldw(const float* w, int i) { return w[i]; }
+__device__ __forceinline__ float ldw(const __nv_bfloat16* w, int i) {
+  return __bfloat162float(w[i]);
+}
+
+// Sequence of token t: the n with cu[n] <= t < cu[n + 1].
+__device__ __forceinline__ int seq_of(const int32_t* cu, int N, int64_t t) {
+  int lo = 0, hi = N;        // cu[lo] <= t, answer in [lo, hi)
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (cu[mid] <= t) lo = mid; else hi = mid;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ void store8h(__half* p, const float (&f)[8]) {
+  uint4 u;
+  __half2* h = reinterpret_cast<__half2*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) h[i] = __floats2half2_rn(f[2 * i], f[2 * i + 1]);
+  *reinterpret_cast<uint4*>(p) = u;
+}
+
+// bf16 -> fp16 for a value row: exact in fp16's normal range; beyond +-65504
+// the value saturates there.
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 u) {
+  const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&u);
+  uint4 r;
+  __half2* h = reinterpret_cast<__half2*>(&r);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 f = __bfloat1622float2(b[i]);
+    f.x = fminf(fmaxf(f.x, -65504.f), 65504.f);
+    f.y = fminf(fmaxf(f.y, -65504.f), 65504.f);
+    h[i] = __floats2half2_rn(f.x, f.y);
+  }
+  return r;
+}
+
+// One (token, head) row of 256 by one warp: RMS-norm with weight w, then
+// rotary on dims [0, R) with the token's (cos, sin) per pair; lane l returns
+// dims 8l .. 8l + 7. `row` is this warp's 256-float staging area.
+template <class Tw>
+__device__ __forceinline__ void norm_rope_row(const __nv_bfloat16* src, const Tw* w,
+                                              const float2* cs, float* row, int R, float eps,
+                                              int lane, float (&x)[8]) {
+  const int half = R >> 1;
+  load8(src + lane * 8, x);
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) ss += x[i] * x[i];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float inv = rsqrtf(ss * (1.0f / kAD) + eps);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    x[i] = x[i] * inv * ldw(w, lane * 8 + i);
+    row[lane * 8 + i] = x[i];
+  }
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int d = lane * 8 + i;
+    if (d < half) {
+      const float2 a = cs[d];
+      x[i] = row[d] * a.x - row[d + half] * a.y;
+    } else if (d < R) {
+      const float2 a = cs[d - half];
+      x[i] = row[d] * a.x + row[d - half] * a.y;
+    }
+  }
+  __syncwarp();
+}
+
+// (cos, sin) of rotary pair i at position pos, angle in fp64.
+__device__ __forceinline__ float2 rope_cs(int64_t pos, int i, int R, double log2_base) {
+  const double theta = (double)pos * exp2(-(2.0 * i / R) * log2_base);
+  double s, c;
+  sincos(theta, &s, &c);
+  return make_float2((float)c, (float)s);
+}
+
+template <class Tw>
+__global__ void __launch_bounds__(256) attn_qk_prologue_kernel(const ProParams p) {
+  __shared__ float2 cs[kProTok][32];       // (cos, sin) per token and rotary pair
+  __shared__ float row[8][kAD];            // one staged row per warp
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t t0 = (int64_t)blockIdx.x * kProTok;
+  const int half = p.R >> 1;
+  if (tid < kProTok * 32) {
+    const int tt = tid >> 5, i = tid & 31;
+    const int64_t t = t0 + tt;
+    if (t < p.T && i < half) {
+      const int axis = i % 3;
+      int64_t pos;
+      if (p.positions) {
+        pos = p.positions[(int64_t)axis * p.T + t];
+      } else {
+        const int n = seq_of(p.cu, p.N, t);
+        pos = t - p.cu[n] + (p.pos0 ? p.pos0[n] : 0);
+      }
+      cs[tt][i] = rope_cs(pos, i, p.R, p.log2_base);
+    }
+  }
+  __syncthreads();
+  const int H = p.Hq + p.Hkv;
+  const Tw* wq = static_cast<const Tw*>(p.wq);
+  const Tw* wk = static_cast<const Tw*>(p.wk);
+  for (int r = warp; r < kProTok * H; r += 8) {
+    const int tt = r / H, hh = r % H;
+    const int64_t t = t0 + tt;
+    if (t >= p.T) break;
+    const bool isq = hh < p.Hq;
+    const __nv_bfloat16* src = isq ? p.q + t * p.q_stride + (int64_t)hh * kAD
+                                   : p.k + t * p.k_stride + (int64_t)(hh - p.Hq) * kAD;
+    float x[8];
+    norm_rope_row(src, isq ? wq : wk, cs[tt], row[warp], p.R, p.eps, lane, x);
+    if (isq) {
+      store8h(p.q_out + (t * p.Hq + hh) * kAD + lane * 8, x);
+    } else {
+      const int g = hh - p.Hq;
+      const int64_t o = (t * p.Hkv + g) * kAD + lane * 8;
+      store8h(p.k_out + o, x);
+      *reinterpret_cast<uint4*>(p.v_out + o) = bf16x8_to_f16x8(
+          *reinterpret_cast<const uint4*>(p.v + t * p.v_stride + (int64_t)g * kAD + lane * 8));
+    }
+  }
+}
+
+// ---------------------------------------------------------- flash attention --
+
+// Shared memory (offsets from a 1024-byte aligned base). Operand tiles are
+// 128-byte-swizzled rows of 64 bf16, as the TMA writes them.
+constexpr uint32_t A_Q = 0;          // 4 dim chunks x [128 rows][128 B] (16 KB each)
+constexpr uint32_t A_K = 65536;      // 2 slots x 4 dim chunks x [64 keys][128 B]
+constexpr uint32_t A_V = 131072;     // 2 slots x 4 dim chunks x [64 keys][128 B]
+constexpr uint32_t A_P = 196608;     // 2 buffers x [128 rows][64 keys] bf16
+constexpr uint32_t A_BAR = 229376;
+constexpr uint32_t A_SMEM = A_BAR + 256 + 1024;   // + alignment slack
+
+// TMEM columns: O accumulator [0, 256), S buffers at 256 and 320.
+constexpr uint32_t T_O = 0, T_S = 256;
+
+struct AttnBars {
+  uint64_t q_full, k_full[2], v_full[2], s_full[2], o_done[2], p_full[2];
+  uint32_t tmem;
+  int n, tile;          // item: sequence and query tile (n < 0: nothing to do)
+};
+
+struct AttnParams {
+  const int32_t* cu; int N; int64_t T; int Hq, Hkv;
+  int grid_tiles;       // tiles the grid was sized for (>= the real count)
+  float sl2;            // softmax scale * log2(e)
+  const __nv_bfloat16* gate; int64_t gate_stride;
+  __nv_bfloat16* o;     // [T][Hq][256]
+  int* status;          // set to 1 when a wait ran out
+};
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ void fail(const AttnParams& p) { atomicExch(p.status, 1); }
+
+// Locate tile u (counted over all sequences, ceil(len / 64) tiles each) with
+// one warp: returns (n, tile) or n = -1 when u is past the last tile.
+__device__ __forceinline__ int cu_at(const int32_t* cu, int n, int64_t T) {
+  const int64_t c = cu[n];
+  return (int)(c < 0 ? 0 : (c > T ? T : c));
+}
+
+__device__ void find_tile(const int32_t* cu, int N, int64_t T, int u, int lane, int* n_out,
+                          int* t_out) {
+  int base = 0;
+  for (int n0 = 0; n0 < N; n0 += 32) {
+    const int n = n0 + lane;
+    const int len = n < N ? max(cu_at(cu, n + 1, T) - cu_at(cu, n, T), 0) : 0;
+    const int tiles = (len + kTileTok - 1) / kTileTok;
+    int incl = tiles;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const int excl = incl - tiles;
+    if (n < N && u >= base + excl && u < base + incl) {
+      *n_out = n;
+      *t_out = u - base - excl;
+    }
+    base += __shfl_sync(0xffffffffu, incl, 31);
+    __syncwarp();
+  }
+}
+
+__global__ void __launch_bounds__(256, 1)
+attn_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
+                    const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* sm = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  const uint32_t sa = smem_u32(sm);
+  AttnBars& B = *reinterpret_cast<AttnBars*>(sm + A_BAR);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int pairs = p.Hq >> 1;
+  const int pair = blockIdx.x % pairs;
+  const int u = p.grid_tiles - 1 - (int)(blockIdx.x / pairs);   // heaviest tiles first
+
+  if (tid == 0) {
+    B.n = -1;
+    mbar_init(&B.q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&B.k_full[i], 1);
+      mbar_init(&B.v_full[i], 1);
+      mbar_init(&B.s_full[i], 1);
+      mbar_init(&B.o_done[i], 1);
+      mbar_init(&B.p_full[i], 128);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int n = -1, t = 0;
+    find_tile(p.cu, p.N, p.T, u, lane, &n, &t);
+    // the lane that found it holds the answer; share through shared memory
+    if (n >= 0) { B.n = n; B.tile = t; }
+  }
+  if (warp == 2) {
+    tmem_alloc(&B.tmem, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const int n = B.n;
+  const uint32_t tmem = B.tmem;
+  if (n >= 0) {
+    const int tile = B.tile;
+    const int s0 = cu_at(p.cu, n, p.T), s1 = max(cu_at(p.cu, n + 1, p.T), s0);
+    const int q0 = s0 + tile * kTileTok;
+    const int nb = tile + 1;                    // key blocks up to the diagonal
+    const int h0 = 2 * pair;
+    const int g = h0 / (p.Hq / p.Hkv);
+
+    if (warp == 0 && lane == 0) {
+      // ---------------------------------------------------------- producer
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      mbar_arrive_expect_tx(&B.q_full, 65536);
+      for (int c = 0; c < 4; ++c)
+        for (int hh = 0; hh < 2; ++hh)
+          tma_load_2d(sm + A_Q + c * 16384 + hh * 8192, &tm_q, (h0 + hh) * kAD + c * 64, q0,
+                      &B.q_full);
+      bool ok = true;
+      int k_issued = 0, v_issued = 0;
+      for (int j = 0; j < nb && ok; ++j) {
+        const int sl = j & 1;
+        const uint32_t par = (uint32_t)(((j - 2) >> 1) & 1);
+        if (j >= 2) ok = mbar_wait_bounded(&B.s_full[sl], par, kAttnLimitNs);   // S_{j-2} read K
+        if (!ok) break;
+        mbar_arrive_expect_tx(&B.k_full[sl], 32768);
+        for (int c = 0; c < 4; ++c)
+          tma_load_2d(sm + A_K + sl * 32768 + c * 8192, &tm_k, g * kAD + c * 64, s0 + j * kBlk,
+                      &B.k_full[sl]);
+        k_issued = j + 1;
+        if (j >= 2) ok = mbar_wait_bounded(&B.o_done[sl], par, kAttnLimitNs);   // O_{j-2} read V
+        if (!ok) break;
+        mbar_arrive_expect_tx(&B.v_full[sl], 32768);
+        for (int c = 0; c < 4; ++c)
+          tma_load_2d(sm + A_V + sl * 32768 + c * 8192, &tm_v, g * kAD + c * 64, s0 + j * kBlk,
+                      &B.v_full[sl]);
+        v_issued = j + 1;
+      }
+      if (!ok) fail(p);
+      // leave only once every copy issued here has landed
+      mbar_wait_bounded(&B.q_full, 0, kAttnLimitNs);
+      for (int j = (k_issued > 2 ? k_issued - 2 : 0); j < k_issued; ++j)
+        mbar_wait_bounded(&B.k_full[j & 1], (uint32_t)((j >> 1) & 1), kAttnLimitNs);
+      for (int j = (v_issued > 2 ? v_issued - 2 : 0); j < v_issued; ++j)
+        mbar_wait_bounded(&B.v_full[j & 1], (uint32_t)((j >> 1) & 1), kAttnLimitNs);
+    } else if (warp == 1 && lane == 0) {
+      // ------------------------------------------------------- MMA issuer
+      const uint32_t id_s = idesc_f16(128, kBlk, false, false);
+      const uint32_t id_o = idesc_f16(128, kAD, false, true);
+      auto issue_s = [&](int j) {
+        const int sl = j & 1;
+        const uint32_t kb = sa + A_K + sl * 32768;
+#pragma unroll
+        for (int kk = 0; kk < 16; ++kk) {
+          const uint32_t off_q = (kk >> 2) * 16384 + (kk & 3) * 32;
+          const uint32_t off_k = (kk >> 2) * 8192 + (kk & 3) * 32;
+          mma_f16(tmem + T_S + sl * kBlk, sw128_desc(sa + A_Q + off_q, 16, 1024),
+                  sw128_desc(kb + off_k, 16, 1024), id_s, kk > 0);
+        }
+        mma_commit(&B.s_full[sl]);
+      };
+      bool ok = mbar_wait_bounded(&B.q_full, 0, kAttnLimitNs);
+      for (int j = 0; j < 2 && j < nb && ok; ++j) {
+        ok = mbar_wait_bounded(&B.k_full[j], 0, kAttnLimitNs);
+        if (ok) {
+          tc_fence_after();
+          issue_s(j);
+        }
+      }
+      for (int j = 0; j < nb && ok; ++j) {
+        const int sl = j & 1;
+        const uint32_t par = (uint32_t)((j >> 1) & 1);
+        ok = mbar_wait_bounded(&B.p_full[sl], par, kAttnLimitNs) &&
+             mbar_wait_bounded(&B.v_full[sl], par, kAttnLimitNs);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t pb = sa + A_P + sl * 16384, vb = sa + A_V + sl * 32768;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_f16(tmem + T_O, sw128_desc(pb + kk * 32, 16, 1024),
+                  sw128_desc(vb + kk * 2048, 8192, 1024), id_o, (j > 0 || kk > 0));
+        mma_commit(&B.o_done[sl]);
+        if (j + 2 < nb) {
+          ok = mbar_wait_bounded(&B.k_full[sl], (uint32_t)(((j + 2) >> 1) & 1), kAttnLimitNs);
+          if (!ok) break;
+          tc_fence_after();
+          issue_s(j + 2);
+        }
+      }
+      if (!ok) fail(p);
+    } else if (warp >= 4) {
+      // ------------------------------------------- softmax, then epilogue
+      const int r = tid - 128;                 // row = TMEM lane
+      const int quad = warp & 3;
+      const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+      const int tq_off = r & 63;               // token offset within the tile
+      float m = -INFINITY, l = 0.f;
+      bool ok = true;
+      for (int j = 0; j < nb; ++j) {
+        const int sl = j & 1;
+        ok = mbar_wait_bounded(&B.s_full[sl], (uint32_t)((j >> 1) & 1), kAttnLimitNs);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t sr[64];
+        tmem_ld32_nowait(trow + T_S + sl * kBlk, *reinterpret_cast<uint32_t(*)[32]>(sr));
+        tmem_ld32_nowait(trow + T_S + sl * kBlk + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
+        tmem_wait_ld();
+        float s[64];
+        const bool diag = (j == nb - 1);
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          s[c] = (diag && c > tq_off) ? -INFINITY : __uint_as_float(sr[c]);
+          mx = fmaxf(mx, s[c]);
+        }
+        const float mb = mx * p.sl2;
+        if (j == 0) {
+          m = mb;
+        } else {
+          const bool need = mb > m + 8.0f;
+          if (__any_sync(0xffffffffu, need)) {
+            const float m_new = fmaxf(m, mb);
+            const float f = ex2(m - m_new);
+            m = m_new;
+            l *= f;
+            // O holds P_0..P_{j-1} V: wait for the last of them, rescale in place
+            ok = mbar_wait_bounded(&B.o_done[(j - 1) & 1], (uint32_t)(((j - 1) >> 1) & 1),
+                                   kAttnLimitNs);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            tc_fence_after();
+#pragma unroll 1
+            for (int cc = 0; cc < kAD / 32; ++cc) {
+              uint32_t ov[32];
+              tmem_ld32_nowait(trow + T_O + cc * 32, ov);
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * f);
+              tmem_st32(trow + T_O + cc * 32, ov);
+            }
+            tmem_wait_st();
+          }
+        }
+        // P_j goes to buffer j & 1, which O_{j-2} read
+        if (j >= 2) {
+          ok = mbar_wait_bounded(&B.o_done[sl], (uint32_t)(((j - 2) >> 1) & 1), kAttnLimitNs);
+          if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        }
+        uint8_t* prow = sm + A_P + sl * 16384 + r * 128;
+        float sum = 0.f;
+#pragma unroll
+        for (int c16 = 0; c16 < 8; ++c16) {
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float a = ex2(fmaf(s[c16 * 8 + 2 * e], p.sl2, -m));
+            const float b = ex2(fmaf(s[c16 * 8 + 2 * e + 1], p.sl2, -m));
+            sum += a + b;
+            __half2 h2 = __floats2half2_rn(a, b);
+            w[e] = *reinterpret_cast<uint32_t*>(&h2);
+          }
+          *reinterpret_cast<uint4*>(prow + ((c16 ^ (r & 7)) << 4)) =
+              make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        l += sum;
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&B.p_full[sl]);
+      }
+      if (ok)
+        ok = mbar_wait_bounded(&B.o_done[(nb - 1) & 1], (uint32_t)(((nb - 1) >> 1) & 1),
+                               kAttnLimitNs);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) {
+        if (lane == 0) fail(p);
+      } else {
+        tc_fence_after();
+        const int tq = q0 + tq_off;
+        const int h = h0 + (r >> 6);
+        const bool valid = tq < s1;
+        const float inv_l = 1.0f / l;
+        const __nv_bfloat16* gp = p.gate + (int64_t)tq * p.gate_stride + (int64_t)h * kAD;
+        __nv_bfloat16* op = p.o + ((int64_t)tq * p.Hq + h) * kAD;
+#pragma unroll 1
+        for (int cc = 0; cc < kAD / 32; ++cc) {
+          uint32_t ov[32];
+          tmem_ld32_nowait(trow + T_O + cc * 32, ov);
+          tmem_wait_ld();
+          if (valid) {
+#pragma unroll
+            for (int q8 = 0; q8 < 4; ++q8) {
+              float gt[8], y[8];
+              load8(gp + cc * 32 + q8 * 8, gt);
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                y[i] = __uint_as_float(ov[q8 * 8 + i]) * inv_l / (1.0f + __expf(-gt[i]));
+              store8(op + cc * 32 + q8 * 8, y);
+            }
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------ decode --
+//
+// One new token per sequence against a pooled KV cache [P][L_max][Hkv][256]:
+//  * attn_decode_prologue_kernel (one CTA per sequence): norm + rotary of the
+//    new q and k at position cache_len[n] (or the given three-axis
+//    positions); rotated q to the workspace in fp32, rotated k and v appended
+//    to the sequence's cache slot at row cache_len[n];
+//  * attn_decode_split_kernel (one CTA per sequence, key-value head and split
+//    of kSplit cached tokens): the G query heads of the group share every K / V
+//    row the CTA streams; writes the split's un-normalised output with its
+//    running max and sum;
+//  * attn_decode_combine_kernel (one CTA per sequence and query head): merges
+//    the splits, divides by the sum, applies sigmoid(gate), and advances
+//    cache_len[n] by one.
+
+constexpr int kSplit = 512;     // cached tokens per split CTA
+
+struct DecParams {
+  const __nv_bfloat16* q; const __nv_bfloat16* k; const __nv_bfloat16* v;
+  const __nv_bfloat16* gate;
+  int64_t q_stride, k_stride, v_stride, gate_stride;   // per sequence row (elements)
+  const void* wq; const void* wk;
+  __half* kc; __half* vc;                 // [P][L_max][Hkv][256]
+  const int32_t* idx;                     // [N] slots, or null (slot n)
+  int32_t* len;                           // [N] cached tokens before this step
+  const int32_t* positions;               // [3][N] or null
+  int N, P, L_max, Hq, Hkv; float eps; int R; double log2_base; float sl2;
+  float* q_rot;                           // [N][Hq][256]
+  float* part_ml;                         // [N][Hq][S][2]: max (log2 units), sum
+  float* part_o;                          // [N][Hq][S][256]
+  int S;
+  __nv_bfloat16* o;                       // [N][Hq][256]
+  int* status;                            // 2: a sequence's slot or length was out of range
+};
+
+__device__ __forceinline__ bool dec_valid(const DecParams& p, int n, int* slot, int* L) {
+  *slot = p.idx ? p.idx[n] : n;
+  *L = p.len[n];
+  return *slot >= 0 && *slot < p.P && *L >= 0 && *L < p.L_max;
+}
+
+template <class Tw>
+__global__ void __launch_bounds__(256) attn_decode_prologue_kernel(const DecParams p) {
+  __shared__ float2 cs[32];
+  __shared__ float row[8][kAD];
+  const int n = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  int slot, L;
+  const bool ok = dec_valid(p, n, &slot, &L);
+  if (!ok) {
+    if (tid == 0) atomicExch(p.status, 2);
+    return;
+  }
+  if (tid < (p.R >> 1)) {
+    const int64_t pos = p.positions ? p.positions[(int64_t)(tid % 3) * p.N + n] : L;
+    cs[tid] = rope_cs(pos, tid, p.R, p.log2_base);
+  }
+  __syncthreads();
+  const Tw* wq = static_cast<const Tw*>(p.wq);
+  const Tw* wk = static_cast<const Tw*>(p.wk);
+  for (int r = warp; r < p.Hq + p.Hkv; r += 8) {
+    float x[8];
+    if (r < p.Hq) {
+      norm_rope_row(p.q + n * p.q_stride + (int64_t)r * kAD, wq, cs, row[warp], p.R, p.eps,
+                    lane, x);
+      float* dst = p.q_rot + ((int64_t)n * p.Hq + r) * kAD + lane * 8;
+      store8(dst, x);
+    } else {
+      const int g = r - p.Hq;
+      norm_rope_row(p.k + n * p.k_stride + (int64_t)g * kAD, wk, cs, row[warp], p.R, p.eps,
+                    lane, x);
+      const int64_t crow = (((int64_t)slot * p.L_max + L) * p.Hkv + g) * kAD + lane * 8;
+      store8h(p.kc + crow, x);
+      *reinterpret_cast<uint4*>(p.vc + crow) = bf16x8_to_f16x8(
+          *reinterpret_cast<const uint4*>(p.v + n * p.v_stride + (int64_t)g * kAD + lane * 8));
+    }
+  }
+}
+
+template <int G>
+__global__ void __launch_bounds__(256) attn_decode_split_kernel(const DecParams p) {
+  extern __shared__ float dsm[];
+  float* q_s = dsm;                         // [G][256]
+  float* p_s = q_s + G * kAD;               // [G][kSplit]
+  float* red = p_s + G * kSplit;            // [8][G][256]
+  const int split = blockIdx.x, g = blockIdx.y, n = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t hq0 = (int64_t)n * p.Hq + g * G;     // first query head of the group
+  int slot, L;
+  const bool ok = dec_valid(p, n, &slot, &L);
+  const int t_beg = split * kSplit;
+  const int n_tok = ok ? min(kSplit, L + 1 - t_beg) : 0;
+  if (n_tok <= 0) {
+    if (tid < G) {
+      float* ml = p.part_ml + ((hq0 + tid) * p.S + split) * 2;
+      ml[0] = ok ? -INFINITY : 0.f;
+      ml[1] = ok ? 0.f : __int_as_float(0x7fc00000);
+    }
+    return;
+  }
+  for (int i = tid; i < G * kAD; i += 256) q_s[i] = p.q_rot[hq0 * kAD + i];
+  __syncthreads();
+  const __half* kb = p.kc + (((int64_t)slot * p.L_max + t_beg) * p.Hkv + g) * kAD;
+  const __half* vb = p.vc + (((int64_t)slot * p.L_max + t_beg) * p.Hkv + g) * kAD;
+  const int64_t tok_stride = (int64_t)p.Hkv * kAD;
+  // scores: 8 lanes per token, lane j of a group reads 16-byte chunks j, j+8, j+16, j+24
+  {
+    const int sub = lane >> 3, j = lane & 7;
+#pragma unroll 2
+    for (int base = warp * 4; base < n_tok; base += 32) {
+      const int i = base + sub;
+      float acc[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) acc[h] = 0.f;
+      if (i < n_tok) {
+        uint4 raw[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          raw[c] = __ldcs(reinterpret_cast<const uint4*>(kb + i * tok_stride + (c * 8 + j) * 8));
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const __half2* h2 = reinterpret_cast<const __half2*>(&raw[c]);
+          float x[8];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __half22float2(h2[e]);
+            x[2 * e] = f.x;
+            x[2 * e + 1] = f.y;
+          }
+          const int d0 = (c * 8 + j) * 8;
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            const float4 qa = *reinterpret_cast<const float4*>(q_s + h * kAD + d0);
+            const float4 qb = *reinterpret_cast<const float4*>(q_s + h * kAD + d0 + 4);
+            acc[h] += x[0] * qa.x + x[1] * qa.y + x[2] * qa.z + x[3] * qa.w + x[4] * qb.x +
+                      x[5] * qb.y + x[6] * qb.z + x[7] * qb.w;
+          }
+        }
+      }
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        acc[h] += __shfl_xor_sync(0xffffffffu, acc[h], 1);
+        acc[h] += __shfl_xor_sync(0xffffffffu, acc[h], 2);
+        acc[h] += __shfl_xor_sync(0xffffffffu, acc[h], 4);
+      }
+      if (j == 0 && i < n_tok) {
+#pragma unroll
+        for (int h = 0; h < G; ++h) p_s[h * kSplit + i] = acc[h] * p.sl2;
+      }
+    }
+  }
+  __syncthreads();
+  // softmax statistics of this split, one warp per query head
+  if (warp < G) {
+    float* ps = p_s + warp * kSplit;
+    float m = -INFINITY;
+    for (int i = lane; i < n_tok; i += 32) m = fmaxf(m, ps[i]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float l = 0.f;
+    for (int i = lane; i < n_tok; i += 32) {
+      const float e = ex2(ps[i] - m);
+      ps[i] = e;
+      l += e;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+    if (lane == 0) {
+      float* ml = p.part_ml + ((hq0 + warp) * p.S + split) * 2;
+      ml[0] = m;
+      ml[1] = l;
+    }
+  }
+  __syncthreads();
+  // P V: a warp per token, lane l owns dims 8l .. 8l + 7
+  float acc[G][8];
+#pragma unroll
+  for (int h = 0; h < G; ++h)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[h][e] = 0.f;
+#pragma unroll 4
+  for (int i = warp; i < n_tok; i += 8) {
+    float x[8];
+    const uint4 raw = __ldcs(reinterpret_cast<const uint4*>(vb + i * tok_stride + lane * 8));
+    const __half2* h2 = reinterpret_cast<const __half2*>(&raw);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __half22float2(h2[e]);
+      x[2 * e] = f.x;
+      x[2 * e + 1] = f.y;
+    }
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float pw = p_s[h * kSplit + i];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[h][e] = fmaf(pw, x[e], acc[h][e]);
+    }
+  }
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    float* r = red + (warp * G + h) * kAD + lane * 8;
+    *reinterpret_cast<float4*>(r) = make_float4(acc[h][0], acc[h][1], acc[h][2], acc[h][3]);
+    *reinterpret_cast<float4*>(r + 4) = make_float4(acc[h][4], acc[h][5], acc[h][6], acc[h][7]);
+  }
+  __syncthreads();
+  for (int k = tid; k < G * kAD; k += 256) {
+    const int h = k / kAD, d = k % kAD;
+    float sum = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) sum += red[(w * G + h) * kAD + d];
+    p.part_o[((hq0 + h) * p.S + split) * kAD + d] = sum;
+  }
+}
+
+__global__ void __launch_bounds__(256) attn_decode_combine_kernel(const DecParams p) {
+  const int h = blockIdx.x, n = blockIdx.y, d = threadIdx.x;
+  const int64_t hq = (int64_t)n * p.Hq + h;
+  const float* ml = p.part_ml + hq * p.S * 2;
+  float M = -INFINITY;
+  for (int s = 0; s < p.S; ++s)
+    if (ml[2 * s + 1] > 0.f) M = fmaxf(M, ml[2 * s]);
+  float Lsum = 0.f, acc = 0.f;
+  for (int s = 0; s < p.S; ++s) {
+    const float l = ml[2 * s + 1];
+    if (l > 0.f) {
+      const float w = ex2(ml[2 * s] - M);
+      Lsum += w * l;
+      acc += w * p.part_o[(hq * p.S + s) * kAD + d];
+    }
+  }
+  const float gt = __bfloat162float(p.gate[n * p.gate_stride + (int64_t)h * kAD + d]);
+  const float y = (Lsum > 0.f ? acc / Lsum : __int_as_float(0x7fc00000)) / (1.0f + __expf(-gt));
+  p.o[hq * kAD + d] = __float2bfloat16_rn(y);
+  if (h == 0 && d == 0) {
+    int slot, L;
+    if (dec_valid(p, n, &slot, &L)) p.len[n] = L + 1;
+  }
+}
+
+// ------------------------------------------------------------------ host --
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void* ptr = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// [rows][cols] 16-bit elements with a row stride, 64 x 64 boxes, 128-byte swizzle.
+bool make_attn_map(CUtensorMap* m, const void* base, int64_t cols, int64_t rows,
+                   int64_t stride_elems, CUtensorMapDataType type) {
+  auto fn = tensor_map_encoder();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(stride_elems * 2)};
+  cuuint32_t box[2] = {64, 64};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, type, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+}  // namespace
+
+size_t attention_prefill_workspace(int64_t T, int Hq) {
+  return 256 + (size_t)T * Hq * kAD * 2;
+}
+
+cudaError_t launch_attention_prefill(const AttnPrefillArgs& a) {
+  if (a.T == 0) return cudaSuccess;
+  uint8_t* ws = static_cast<uint8_t*>(a.workspace);
+  int* status = reinterpret_cast<int*>(ws);
+  __half* q_rot = reinterpret_cast<__half*>(ws + 256);
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), a.stream);
+  if (e != cudaSuccess) return e;
+
+  ProParams pp{static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k),
+               a.q_row_stride, a.k_row_stride, a.wq, a.wk, a.cu_seqlens, a.N, a.T,
+               a.positions, a.pos0, a.Hq, a.Hkv, a.eps, a.rope_dims, log2((double)a.rope_base),
+               static_cast<const __nv_bfloat16*>(a.v), a.v_row_stride, q_rot,
+               static_cast<__half*>(a.k_rot), static_cast<__half*>(a.v_h)};
+  const unsigned pgrid = (unsigned)((a.T + kProTok - 1) / kProTok);
+  if (a.w_dtype == GDN_F32)
+    attn_qk_prologue_kernel<float><<<pgrid, 256, 0, a.stream>>>(pp);
+  else
+    attn_qk_prologue_kernel<__nv_bfloat16><<<pgrid, 256, 0, a.stream>>>(pp);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+
+  CUtensorMap mq, mk, mv;
+  if (!make_attn_map(&mq, q_rot, (int64_t)a.Hq * kAD, a.T, (int64_t)a.Hq * kAD,
+                     CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
+      !make_attn_map(&mk, a.k_rot, (int64_t)a.Hkv * kAD, a.T, (int64_t)a.Hkv * kAD,
+                     CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
+      !make_attn_map(&mv, a.v_h, (int64_t)a.Hkv * kAD, a.T, (int64_t)a.Hkv * kAD,
+                     CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+    return cudaErrorInvalidValue;
+  const int grid_tiles = (int)((a.T + kTileTok - 1) / kTileTok) + a.N;
+  AttnParams ap{a.cu_seqlens, a.N, a.T, a.Hq, a.Hkv, grid_tiles,
+                a.scale * 1.4426950408889634f, static_cast<const __nv_bfloat16*>(a.gate),
+                a.gate_row_stride, static_cast<__nv_bfloat16*>(a.o), status};
+  static bool attr_set = false;
+  if (!attr_set) {
+    e = cudaFuncSetAttribute(attn_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)A_SMEM);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const unsigned grid = (unsigned)grid_tiles * (unsigned)(a.Hq / 2);
+  attn_prefill_kernel<<<grid, 256, A_SMEM, a.stream>>>(mq, mk, mv, ap);
+  return cudaGetLastError();
+}
+
+cudaError_t attention_status_word(const void* workspace, cudaStream_t stream, int* word) {
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return e;
+  return cudaMemcpy(word, workspace, sizeof(int), cudaMemcpyDeviceToHost);
+}
+
+size_t attention_decode_workspace(int N, int Hq, int L_max) {
+  const size_t S = (size_t)((L_max + kSplit - 1) / kSplit);
+  return 256 + (size_t)N * Hq * kAD * 4 + (size_t)N * Hq * S * 2 * 4 +
+         (size_t)N * Hq * S * kAD * 4;
+}
+
+template <int G>
+cudaError_t launch_split(const DecParams& dp, dim3 grid, cudaStream_t stream) {
+  const size_t smem = (size_t)(G * kAD + G * kSplit + 8 * G * kAD) * sizeof(float);
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(attn_decode_split_kernel<G>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  attn_decode_split_kernel<G><<<grid, 256, smem, stream>>>(dp);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attention_decode(const AttnDecodeArgs& a) {
+  if (a.N == 0) return cudaSuccess;
+  uint8_t* ws = static_cast<uint8_t*>(a.workspace);
+  int* status = reinterpret_cast<int*>(ws);
+  const int S = (a.L_max + kSplit - 1) / kSplit;
+  float* q_rot = reinterpret_cast<float*>(ws + 256);
+  float* part_ml = q_rot + (size_t)a.N * a.Hq * kAD;
+  float* part_o = part_ml + (size_t)a.N * a.Hq * S * 2;
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), a.stream);
+  if (e != cudaSuccess) return e;
+  DecParams dp{static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k),
+               static_cast<const __nv_bfloat16*>(a.v), static_cast<const __nv_bfloat16*>(a.gate),
+               a.q_row_stride, a.k_row_stride, a.v_row_stride, a.gate_row_stride, a.wq, a.wk,
+               static_cast<__half*>(a.k_cache), static_cast<__half*>(a.v_cache),
+               a.cache_idx, a.cache_len, a.positions, a.N, a.P, a.L_max, a.Hq, a.Hkv, a.eps,
+               a.rope_dims, log2((double)a.rope_base), a.scale * 1.4426950408889634f, q_rot,
+               part_ml, part_o, S, static_cast<__nv_bfloat16*>(a.o), status};
+  if (a.w_dtype == GDN_F32)
+    attn_decode_prologue_kernel<float><<<a.N, 256, 0, a.stream>>>(dp);
+  else
+    attn_decode_prologue_kernel<__nv_bfloat16><<<a.N, 256, 0, a.stream>>>(dp);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const dim3 grid((unsigned)S, (unsigned)a.Hkv, (unsigned)a.N);
+  switch (a.Hq / a.Hkv) {
+    case 1: e = launch_split<1>(dp, grid, a.stream); break;
+    case 2: e = launch_split<2>(dp, grid, a.stream); break;
+    case 4: e = launch_split<4>(dp, grid, a.stream); break;
+    case 6: e = launch_split<6>(dp, grid, a.stream); break;
+    case 8: e = launch_split<8>(dp, grid, a.stream); break;
+    default: return cudaErrorInvalidValue;
+  }
+  if (e != cudaSuccess) return e;
+  attn_decode_combine_kernel<<<dim3((unsigned)a.Hq, (unsigned)a.N), kAD, 0, a.stream>>>(dp);
+  return cudaGetLastError();
+}
+
+}  // namespace gdn

@@ -65,6 +65,37 @@ struct LayerPrefillArgs {
   cudaStream_t stream;
 };
 
+// Global-attention prefill: q/k RMS-norm + rotary, then causal GQA flash
+// attention with the sigmoid output gate. q, k, v, gate and o are bf16 with
+// head dim 256; the rotated keys k_rot and the values v_h (as the KV cache
+// holds them) are fp16; the norm weights are w_dtype.
+struct AttnPrefillArgs {
+  const void* q; const void* k; const void* v; const void* gate;
+  int64_t q_row_stride, k_row_stride, v_row_stride, gate_row_stride;
+  const void* wq; const void* wk; gdn_dtype w_dtype;
+  const int32_t* cu_seqlens; const int32_t* positions; const int32_t* pos0;
+  int N; int64_t T; int Hq; int Hkv;
+  float eps; int rope_dims; float rope_base; float scale;
+  void* o; void* k_rot; void* v_h;
+  void* workspace;
+  cudaStream_t stream;
+};
+
+// Global-attention decode: one new token per sequence against a pooled KV
+// cache [P][L_max][Hkv][256] (fp16 keys and values); cache_len[n] is read, the new k / v go to
+// that row, and it is advanced by one.
+struct AttnDecodeArgs {
+  const void* q; const void* k; const void* v; const void* gate;
+  int64_t q_row_stride, k_row_stride, v_row_stride, gate_row_stride;
+  const void* wq; const void* wk; gdn_dtype w_dtype;
+  void* k_cache; void* v_cache; const int32_t* cache_idx; int32_t* cache_len;
+  const int32_t* positions;
+  int N; int P; int L_max; int Hq; int Hkv;
+  float eps; int rope_dims; float rope_base; float scale;
+  void* o; void* workspace;
+  cudaStream_t stream;
+};
+
 struct NormArgs {
   const void* x; gdn_dtype x_dtype; const void* z; gdn_dtype z_dtype;
   const void* w; gdn_dtype w_dtype; int64_t rows; int dim; float eps;
@@ -92,6 +123,13 @@ size_t prefill_pc_workspace(int N, int64_t T_total, int H_v);
 // The same kernel on the library-owned static scratch (no workspace argument).
 cudaError_t launch_prefill_pc_noalloc(const RecurArgs& a);
 size_t prefill_noalloc_scratch_bytes();
+cudaError_t launch_attention_prefill(const AttnPrefillArgs& a);
+size_t attention_prefill_workspace(int64_t T, int Hq);
+cudaError_t launch_attention_decode(const AttnDecodeArgs& a);
+size_t attention_decode_workspace(int N, int Hq, int L_max);
+// Synchronises `stream`, then reads the status word the last attention call
+// left in `workspace` (1: a wait inside the kernel ran out).
+cudaError_t attention_status_word(const void* workspace, cudaStream_t stream, int* word);
 // Limit of the chunk kernel's waits on another CTA's flag (0 restores 2 s).
 void set_wait_limit_ns(uint64_t ns);
 uint64_t wait_limit_ns();

@@ -15,6 +15,11 @@ leaderboard commentary (section 二.1): 16 key heads, 48 value heads, head dim
 * initial recurrent states ~ N(0, 0.02) (variance 0.02);
 * packed varlen lengths: integers uniform in [512, 16384].
 
+The global-attention layer of the same decoder (model card, section 架构,
+rows 全局注意力 and 位置编码): 24 query / 4 key-value heads, head dim 256.
+Its projections q, k, v and the output gate are drawn N(0, 1) and stored
+bf16; the q/k RMS-norm weights are 1 + N(0, 0.1^2).
+
 Every generator is a numpy PCG64 stream keyed by (seed, tag), so any part can
 be regenerated alone. bf16 rounding uses torch's CPU cast (round to nearest
 even); the oracle is always handed the rounded values.
@@ -161,3 +166,18 @@ def decode_initial(N=256, seed=0):
     pre-conv cache [N,3,10240] ~ N(0,1) (the 3 prior tokens, oldest first)."""
     return dict(state=initial_states(seed, N, tag="dstate"),
                 conv_state=to_bf16(normal(seed, "dconv", (N, 3, CONV_CHANNELS))))
+
+
+ATTN_H_Q, ATTN_H_KV, ATTN_D = 24, 4, 256
+
+
+def attention_inputs(T, seed=0, H_q=ATTN_H_Q, H_kv=ATTN_H_KV, d=ATTN_D, tag="attn"):
+    """q, gate [T, H_q, d]; k, v [T, H_kv, d] (bf16, N(0,1)); q_norm_w, k_norm_w
+    [d] (bf16, 1 + N(0, 0.01))."""
+    out = {}
+    for name, H in (("q", H_q), ("k", H_kv), ("v", H_kv), ("gate", H_q)):
+        out[name] = to_bf16(normal(seed, (tag, name), (T, H, d)))
+    for name in ("q_norm_w", "k_norm_w"):
+        out[name] = to_bf16(1.0 + normal(seed, (tag, name), (d,), std=0.1))
+    return out
+

@@ -350,6 +350,105 @@ gdn_status gdn_gated_rmsnorm(const void* x, gdn_dtype x_dtype, const void* z,
                              float eps, void* y, gdn_dtype y_dtype,
                              cudaStream_t stream);
 
+/* ------------------------------------------------------------------------
+ * Global-attention layer: the hybrid decoder's other layer type, one of
+ * every four layers (18 of 72) and the only one holding a KV cache ([P3 架构],
+ * rows 全局注意力 and 位置编码; [P2 二.1], attn_output_gate true). Per token:
+ *   qn = q / sqrt(mean(q^2) + eps) * q_norm_w   (per head over head_dim)
+ *   kn = k / sqrt(mean(k^2) + eps) * k_norm_w
+ *   rotary on dims [0, rope_dims): pair i couples dims i and i + rope_dims/2
+ *     and turns (counter-clockwise: (a, b) -> (a c - b s, b c + a s)) by
+ *     theta_i = p_{i mod 3} * rope_base^(-2i / rope_dims), where (p_0, p_1,
+ *     p_2) are the token's text, height and width positions (the pages'
+ *     interleaved 11 : 11 : 10 split of the 32 pairs at rope_dims = 64);
+ *   o_h = sum_j softmax_j(scale * qn_h . kn_j) v_j over the earlier tokens j
+ *     of the same sequence and itself, query head h reading key-value head
+ *     h / (H_q / H_kv);
+ *   out_h = o_h * sigmoid(gate_h)   (elementwise).
+ * The model's sizes are H_q = 24, H_kv = 4, head_dim = 256, rope_dims = 64,
+ * rope_base = 1e7; head_dim must be 256 and rope_dims even and <= 64
+ * (GDN_ERR_UNSUPPORTED otherwise). q, k, v, gate and o are bf16. The KV
+ * cache is fp16: the normed, rotated keys are bounded by
+ * 16 * sqrt(2) * max|k_norm_w|, inside fp16's range, and fp16 keeps three
+ * more significand bits than bf16 for the score product; a bf16 value in
+ * fp16's normal range converts to fp16 exactly (beyond +-65504 it saturates),
+ * and fp16 values let the softmax weights P enter P V in fp16 as well. The
+ * norm weights are w_dtype (bf16 or fp32). Row strides are per
+ * token (prefill) or per sequence (decode), in elements, multiples of 8 and
+ * at least H * 256; each head's 256 values are contiguous.
+ * ---------------------------------------------------------------------- */
+
+/*
+ * gdn_attention_prefill -- causal attention over a packed batch of prompts.
+ *   q, gate [T_total, H_q, 256]; k, v [T_total, H_kv, 256] (row strides as
+ *   given); cu_seqlens as for the delta-rule layer.
+ *   positions  [3, T_total] int32 (text, height, width) or NULL: then every
+ *              axis carries the token's index within its sequence plus
+ *              pos0[n] (pos0 [N] int32, or NULL for 0) -- a prompt that
+ *              continues a cached prefix passes the prefix length there.
+ *   o          [T_total, H_q, 256] contiguous: the gated output.
+ *   k_rot      [T_total, H_kv, 256] contiguous fp16: the normed, rotated
+ *              keys, as the key cache holds them.
+ *   v_h        [T_total, H_kv, 256] contiguous fp16: v as the value cache
+ *              holds it.
+ *   workspace  gdn_attention_prefill_workspace(T_total, H_q, 256) bytes,
+ *              16-byte aligned (the rotated queries and a status word).
+ * (H_q / H_kv) must be even: a CTA works on two query heads of one group.
+ * Each attention CTA's waits on its own copies and tensor-core products are
+ * bounded (2 s); gdn_attention_status reports one that ran out. Additional
+ * entry point (the pages describe the layer, not an interface).
+ */
+size_t gdn_attention_prefill_workspace(int64_t T_total, int H_q, int head_dim);
+gdn_status gdn_attention_prefill(const void* q, int64_t q_row_stride, const void* k,
+                                 int64_t k_row_stride, const void* v, int64_t v_row_stride,
+                                 const void* gate, int64_t gate_row_stride,
+                                 const void* q_norm_w, const void* k_norm_w, gdn_dtype w_dtype,
+                                 const int32_t* cu_seqlens, const int32_t* positions,
+                                 const int32_t* pos0, int N, int64_t T_total, int H_q, int H_kv,
+                                 int head_dim, float eps, int rope_dims, float rope_base,
+                                 float scale, void* o, void* k_rot, void* v_h, void* workspace,
+                                 size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * gdn_attention_decode -- one new token for each of N sequences against a
+ * pooled KV cache.
+ *   q, gate [N, H_q, 256]; k, v [N, H_kv, 256] (row strides per sequence).
+ *   k_cache, v_cache  [P, L_max, H_kv, 256] fp16 pools; sequence n lives in
+ *              slot cache_idx[n] (cache_idx NULL: slot n) and has
+ *              cache_len[n] tokens cached (rotated keys, as
+ *              gdn_attention_prefill's k_rot and v_h). The new token's
+ *              rotated k and its v (in fp16) are written at row cache_len[n], the token attends to
+ *              rows 0 .. cache_len[n], and cache_len[n] is then advanced by
+ *              one on the device (the caller's copy of it stays in step).
+ *   positions  [3, N] int32 or NULL (then cache_len[n] on every axis).
+ *   o          [N, H_q, 256] contiguous.
+ *   workspace  gdn_attention_decode_workspace(N, H_q, L_max, 256) bytes.
+ * H_q / H_kv must be 1, 2, 4, 6 or 8. A sequence whose slot is outside
+ * [0, P) or whose cache_len is outside [0, L_max) is skipped: its cache and
+ * cache_len stay untouched, its output is NaN, and gdn_attention_status
+ * returns GDN_ERR_INVALID_ARG. Distinct sequences must use distinct slots.
+ * Additional entry point.
+ */
+size_t gdn_attention_decode_workspace(int N, int H_q, int L_max, int head_dim);
+gdn_status gdn_attention_decode(const void* q, int64_t q_row_stride, const void* k,
+                                int64_t k_row_stride, const void* v, int64_t v_row_stride,
+                                const void* gate, int64_t gate_row_stride,
+                                const void* q_norm_w, const void* k_norm_w, gdn_dtype w_dtype,
+                                void* k_cache, void* v_cache, const int32_t* cache_idx,
+                                int32_t* cache_len, const int32_t* positions, int N, int P,
+                                int L_max, int H_q, int H_kv, int head_dim, float eps,
+                                int rope_dims, float rope_base, float scale, void* o,
+                                void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * gdn_attention_status -- waits for `stream` (it synchronises), then reads the
+ * status word that the last attention call working in `workspace` left:
+ * GDN_OK; GDN_ERR_TIMEOUT when a bounded wait inside the prefill kernel ran
+ * out (the affected output tiles are left unwritten); GDN_ERR_INVALID_ARG when
+ * a decode sequence had an out-of-range slot or length. Additional entry point.
+ */
+gdn_status gdn_attention_status(const void* workspace, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

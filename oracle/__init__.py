@@ -83,8 +83,8 @@ def _load():
             _dp, _dp, _dp, _dp, _ip, ctypes.POINTER(ctypes.c_int64),
             ctypes.POINTER(ctypes.c_int64), ctypes.c_int,
             ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, _dp, _dp,
-            ctypes.c_double, ctypes.c_int, ctypes.c_double, ctypes.c_double, _dp, _dp, _dp,
-            ctypes.c_int]
+            ctypes.c_double, ctypes.c_int, ctypes.c_double, ctypes.c_double,
+            ctypes.POINTER(ctypes.c_uint8), _dp, _dp, _dp, ctypes.c_int]
         lib.oracle_gated_rmsnorm.restype = None
         lib.oracle_gated_rmsnorm.argtypes = [
             _dp, _dp, _dp, ctypes.c_int64, ctypes.c_int, ctypes.c_double, _dp,
@@ -188,7 +188,7 @@ def gated_rmsnorm(x, z, w, eps=1e-6, threads=0):
 
 
 def attention(q, k, v, gate, wq, wk, cu_seqlens=None, pos0=None, positions=None,
-              eps=1e-6, rope_dims=64, rope_base=1e7, scale=None, threads=0):
+              eps=1e-6, rope_dims=64, rope_base=1e7, scale=None, rows=None, threads=0):
     """Global-attention layer (fp64): per token and head, q and k RMS-normed
     over the head dim with weights wq / wk, rotary (rotate-half pairs
     (i, i + R/2), theta = p * base^(-2i/R)) on the first ``rope_dims`` dims,
@@ -201,7 +201,8 @@ def attention(q, k, v, gate, wq, wk, cu_seqlens=None, pos0=None, positions=None,
 
     q, gate [T, Hq, D]; k, v [T, Hkv, D]; wq, wk [D]; pos0 [N] or None.
     Returns (out [T, Hq, D], q_rot [T, Hq, D], k_rot [T, Hkv, D]); scale
-    defaults to D**-0.5."""
+    defaults to D**-0.5. ``rows`` (token indices) limits the output rows that
+    are computed; the others are returned as zeros."""
     q, k, v, gate, wq, wk = (_f64(a) for a in (q, k, v, gate, wq, wk))
     T, Hq, D = q.shape
     Hkv = k.shape[1]
@@ -223,11 +224,17 @@ def attention(q, k, v, gate, wq, wk, cu_seqlens=None, pos0=None, positions=None,
     qr = np.zeros_like(q)
     kr = np.zeros_like(k)
     i64 = ctypes.POINTER(ctypes.c_int64)
+    want = None
+    if rows is not None:
+        want = np.zeros(T, dtype=np.uint8)
+        want[np.asarray(rows, dtype=np.int64)] = 1
     _load().oracle_attention(
         _ptr(q), _ptr(k), _ptr(v), _ptr(gate), cu.ctypes.data_as(_ip),
         None if p0 is None else p0.ctypes.data_as(i64),
         None if p3 is None else p3.ctypes.data_as(i64), N, T, Hq,
         Hkv, D, _ptr(wq), _ptr(wk), float(eps), int(rope_dims), float(rope_base),
-        float(D ** -0.5 if scale is None else scale), _ptr(out), _ptr(qr), _ptr(kr),
+        float(D ** -0.5 if scale is None else scale),
+        None if want is None else want.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)),
+        _ptr(out), _ptr(qr), _ptr(kr),
         int(threads))
     return out, qr, kr

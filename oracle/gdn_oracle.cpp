@@ -246,7 +246,8 @@ void oracle_attention(const double* q, const double* k, const double* v,
                       const double* gate, const int32_t* cu_seqlens, const int64_t* pos0,
                       const int64_t* pos3, int N, int64_t T, int Hq, int Hkv, int D,
                       const double* wq, const double* wk, double eps, int R, double base,
-                      double scale, double* out, double* q_rot, double* k_rot, int threads) {
+                      double scale, const uint8_t* want, double* out, double* q_rot,
+                      double* k_rot, int threads) {
   // Per-head RMS-norm with weight w, then rotary on dims [0, R): pair i couples
   // dims i and i + R/2 and turns by theta_i = p * base^(-2i/R), where p is the
   // token's position on axis i mod 3 (text, height, width interleaved, which
@@ -287,6 +288,7 @@ void oracle_attention(const double* q, const double* k, const double* v,
     const int64_t s0 = cu_seqlens[n], s1 = cu_seqlens[n + 1];
     std::vector<double> sc((size_t)(s1 - s0)), o(D);
     for (int64_t t = s0; t < s1; ++t) {
+      if (want && !want[t]) continue;   // output row not asked for
       const double* qt = qr.data() + (t * Hq + h) * D;
       double m = -INFINITY;
       for (int64_t j = s0; j <= t; ++j) {

@@ -286,3 +286,102 @@ def test_decode_layer_binding_checks(lib):
         call(z=z.float())
     with pytest.raises(ValueError, match="norm_w: dtype"):
         call(nw=nw.bfloat16())
+
+
+def attn_prefill(lib, **kw):
+    a = dict(q=A, qs=24 * 256, k=A, ks=4 * 256, v=A, vs=4 * 256, gate=A, gs=24 * 256, wq=A,
+             wk=A, wdt=BF16, cu=A, pos=None, pos0=None, N=1, T=128, Hq=24, Hkv=4, D=256,
+             eps=1e-6, R=64, base=1e7, scale=0.0625, o=A, k_rot=A, v_h=A, ws=A,
+             ws_bytes=1 << 40, s=None)
+    a.update(kw)
+    return lib.gdn_attention_prefill(*a.values())
+
+
+def attn_decode(lib, **kw):
+    a = dict(q=A, qs=24 * 256, k=A, ks=4 * 256, v=A, vs=4 * 256, gate=A, gs=24 * 256, wq=A,
+             wk=A, wdt=BF16, kc=A, vc=A, idx=None, len=A, pos=None, N=4, P=4, L=1024, Hq=24,
+             Hkv=4, D=256, eps=1e-6, R=64, base=1e7, scale=0.0625, o=A, ws=A,
+             ws_bytes=1 << 40, s=None)
+    a.update(kw)
+    return lib.gdn_attention_decode(*a.values())
+
+
+def test_attention_prefill_validation(lib):
+    assert attn_prefill(lib, D=128) == UNSUPPORTED
+    assert attn_prefill(lib, Hkv=5) == INVALID               # 24 % 5
+    assert attn_prefill(lib, Hq=12, Hkv=4, qs=12 * 256, gs=12 * 256) == UNSUPPORTED  # 3 per group
+    assert attn_prefill(lib, R=66) == UNSUPPORTED
+    assert attn_prefill(lib, R=63) == UNSUPPORTED
+    assert attn_prefill(lib, base=1.0) == INVALID
+    assert attn_prefill(lib, eps=-1.0) == INVALID
+    assert attn_prefill(lib, wdt=7) == INVALID
+    assert attn_prefill(lib, N=0) == INVALID                 # tokens but no sequence
+    assert attn_prefill(lib, qs=24 * 256 - 8) == MISALIGNED  # stride below H_q * 256
+    assert attn_prefill(lib, vs=4 * 256 + 4) == MISALIGNED   # not a multiple of 8 elements
+    assert attn_prefill(lib, cu=None) == INVALID
+    assert attn_prefill(lib, k_rot=None) == INVALID
+    assert attn_prefill(lib, v_h=None) == INVALID
+    assert attn_prefill(lib, v_h=A + 8) == MISALIGNED
+    assert attn_prefill(lib, ws_bytes=1024) == INVALID
+    assert attn_prefill(lib, q=A + 2) == MISALIGNED
+    assert attn_prefill(lib, ws=A + 8) == MISALIGNED
+    assert attn_prefill(lib, wq=A + 2, wdt=F32) == MISALIGNED
+    assert attn_prefill(lib, T=0) == OK
+    need = lib.gdn_attention_prefill_workspace(8192, 24, 256)
+    assert need >= 8192 * 24 * 256 * 2
+    assert lib.gdn_attention_prefill_workspace(8192, 24, 128) == 0
+
+
+def test_attention_decode_validation(lib):
+    assert attn_decode(lib, D=128) == UNSUPPORTED
+    assert attn_decode(lib, Hq=12, Hkv=4, qs=12 * 256, gs=12 * 256) == UNSUPPORTED  # 3 per group
+    assert attn_decode(lib, N=-1) == INVALID
+    assert attn_decode(lib, N=70000) == INVALID
+    assert attn_decode(lib, P=0) == INVALID
+    assert attn_decode(lib, L=0) == INVALID
+    assert attn_decode(lib, len=None) == INVALID
+    assert attn_decode(lib, kc=None) == INVALID
+    assert attn_decode(lib, kc=A + 8) == MISALIGNED
+    assert attn_decode(lib, ks=4 * 256 + 2) == MISALIGNED
+    assert attn_decode(lib, ws_bytes=256) == INVALID
+    assert attn_decode(lib, N=0) == OK
+    assert lib.gdn_attention_decode_workspace(256, 24, 4224, 256) > 256 * 24 * 256 * 4
+    assert lib.gdn_attention_status(None, None) == INVALID
+    assert lib.gdn_attention_status(A + 4, None) == MISALIGNED
+
+
+def test_attention_binding_checks(lib):
+    import torch
+    T, N = 16, 1
+    q = torch.zeros(T, 24, 256, dtype=torch.bfloat16)
+    k = torch.zeros(T, 4, 256, dtype=torch.bfloat16)
+    w = torch.ones(256, dtype=torch.bfloat16)
+    cu = torch.tensor([0, T], dtype=torch.int32)
+    with pytest.raises(ValueError, match="k: dtype"):
+        gdn.gdn_attention_prefill(q, k.float(), k, q, w, w, cu)
+    with pytest.raises(ValueError, match="gate: shape"):
+        gdn.gdn_attention_prefill(q, k, k, k, w, w, cu)
+    with pytest.raises(ValueError, match="k_norm_w: dtype"):
+        gdn.gdn_attention_prefill(q, k, k, q, w, w.float(), cu)
+    with pytest.raises(ValueError, match="cu_seqlens: dtype"):
+        gdn.gdn_attention_prefill(q, k, k, q, w, w, cu.long())
+    with pytest.raises(ValueError, match="positions: shape"):
+        gdn.gdn_attention_prefill(q, k, k, q, w, w, cu,
+                                  positions=torch.zeros(T, 3, dtype=torch.int32))
+    with pytest.raises(ValueError, match="CUDA tensors only"):
+        gdn.gdn_attention_prefill(q, k, k, q, w, w, cu)
+    kc = torch.zeros(2, 64, 4, 256, dtype=torch.float16)
+    vb = torch.zeros(2, 64, 4, 256, dtype=torch.bfloat16)
+    ln = torch.zeros(N, dtype=torch.int32)
+    with pytest.raises(ValueError, match="k_cache: dtype"):
+        gdn.gdn_attention_decode(q[:N], k[:N], k[:N], q[:N], w, w, vb, kc, ln)
+    with pytest.raises(ValueError, match="v_cache: dtype"):
+        gdn.gdn_attention_decode(q[:N], k[:N], k[:N], q[:N], w, w, kc, vb, ln)
+    with pytest.raises(ValueError, match="cache_len: dtype"):
+        gdn.gdn_attention_decode(q[:N], k[:N], k[:N], q[:N], w, w, kc, kc, ln.long())
+    with pytest.raises(ValueError, match="v_h: dtype"):
+        gdn.gdn_attention_prefill(q, k, k, q, w, w, cu,
+                                  v_h=torch.zeros(T, 4, 256, dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="k_rot: dtype"):
+        gdn.gdn_attention_prefill(q, k, k, q, w, w, cu,
+                                  k_rot=torch.zeros(T, 4, 256, dtype=torch.bfloat16))

@@ -198,3 +198,13 @@ def test_against_a_separate_numpy_formulation():
     np.testing.assert_allclose(qr, wqr, rtol=1e-12, atol=1e-12)
     np.testing.assert_allclose(kr, wkr, rtol=1e-12, atol=1e-12)
     np.testing.assert_allclose(got, want, rtol=1e-10, atol=1e-12)
+
+
+def test_selected_rows_equal_the_full_computation():
+    T = 20
+    q, k, v, gate = rnd(30, T, 2, 16), rnd(31, T, 1, 16), rnd(32, T, 1, 16), rnd(33, T, 2, 16)
+    full, _, _ = oracle.attention(q, k, v, gate, np.ones(16), np.ones(16), rope_dims=8)
+    part, _, _ = oracle.attention(q, k, v, gate, np.ones(16), np.ones(16), rope_dims=8,
+                                  rows=[0, 7, 19])
+    np.testing.assert_array_equal(part[[0, 7, 19]], full[[0, 7, 19]])
+    assert not part[[1, 8, 18]].any()
