@@ -508,15 +508,13 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
 //    new q and k at position cache_len[n] (or the given three-axis
 //    positions); rotated q to the workspace in fp32, rotated k and v appended
 //    to the sequence's cache slot at row cache_len[n];
-//  * attn_decode_split_kernel (one CTA per sequence, key-value head and split
-//    of kSplit cached tokens): the G query heads of the group share every K / V
-//    row the CTA streams; writes the split's un-normalised output with its
+//  * attn_decode_split_kernel (one warp per sequence, key-value head and unit
+//    of kUnit cached tokens): the G query heads of the group share every K / V
+//    row the warp streams; writes the unit's un-normalised output with its
 //    running max and sum;
 //  * attn_decode_combine_kernel (one CTA per sequence and query head): merges
 //    the splits, divides by the sum, applies sigmoid(gate), and advances
 //    cache_len[n] by one.
-
-constexpr int kSplit = 512;     // cached tokens per split CTA
 
 struct DecParams {
   const __nv_bfloat16* q; const __nv_bfloat16* k; const __nv_bfloat16* v;
@@ -531,7 +529,7 @@ struct DecParams {
   float* q_rot;                           // [N][Hq][256]
   float* part_ml;                         // [N][Hq][S][2]: max (log2 units), sum
   float* part_o;                          // [N][Hq][S][256]
-  int S;
+  int S;                                  // units per (sequence, key-value head)
   __nv_bfloat16* o;                       // [N][Hq][256]
   int* status;                            // 2: a sequence's slot or length was out of range
 };
@@ -579,138 +577,188 @@ __global__ void __launch_bounds__(256) attn_decode_prologue_kernel(const DecPara
   }
 }
 
+// ---- split kernel: one warp streams kUnit cached tokens of one (sequence,
+// key-value head) in groups of 16 through a two-stage cp.async ring in its own
+// shared memory, and runs both products on the tensor cores (mma.sync
+// m16n8k16, fp16 in, fp32 accumulate): S = Q K^T with the G query heads of the
+// group as rows (rows G..15 zero), then O += P V with P taken straight from the
+// S registers. Online softmax per row with the same lazy rescale as prefill.
+// Each warp writes its own partial (max, sum, un-normalised O); no CTA-wide
+// synchronisation.
+constexpr int kGrp = 16;                     // tokens per group
+constexpr int kUnit = 512;                   // tokens per warp
+constexpr int kRowB = 528;                   // smem row stride: 512 B + 16 (no bank conflicts)
+constexpr int kStageB = 2 * kGrp * kRowB;    // K and V rows of one group
+constexpr int kDecWarps = 2;                 // warps (units) per CTA; they share Q
+constexpr int kQB = 8 * kRowB;               // Q rows 0..7 in fp16 (rows >= G zero)
+constexpr int kDecSmem = kQB + kDecWarps * 2 * kStageB;
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];"
+               : "=r"(r0), "=r"(r1)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+// d += A B, A rows 8..15 zero (a1 = a3 = 0)
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_h2(float a, float b) {
+  __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
 template <int G>
-__global__ void __launch_bounds__(256) attn_decode_split_kernel(const DecParams p) {
-  extern __shared__ float dsm[];
-  float* q_s = dsm;                         // [G][256]
-  float* p_s = q_s + G * kAD;               // [G][kSplit]
-  float* red = p_s + G * kSplit;            // [8][G][256]
-  const int split = blockIdx.x, g = blockIdx.y, n = blockIdx.z;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t hq0 = (int64_t)n * p.Hq + g * G;     // first query head of the group
+__global__ void __launch_bounds__(32 * kDecWarps, 3) attn_decode_split_kernel(const DecParams p) {
+  extern __shared__ __align__(16) uint8_t dsm[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int unit = blockIdx.x * kDecWarps + warp, g = blockIdx.y, n = blockIdx.z;
+  const int64_t hq0 = (int64_t)n * p.Hq + g * G;
   int slot, L;
   const bool ok = dec_valid(p, n, &slot, &L);
-  const int t_beg = split * kSplit;
-  const int n_tok = ok ? min(kSplit, L + 1 - t_beg) : 0;
+  // Q of the group's G heads -> fp16 rows of shared memory (rows G..7 zero)
+  const uint32_t qbase = smem_u32(dsm);
+  for (int i = threadIdx.x; i < 8 * kAD / 2; i += 32 * kDecWarps) {
+    const int r = i / (kAD / 2), c = 2 * (i % (kAD / 2));
+    uint32_t v = 0u;
+    if (ok && r < G) {
+      const float* qr = p.q_rot + (hq0 + r) * kAD + c;
+      v = pack_h2(qr[0], qr[1]);
+    }
+    *reinterpret_cast<uint32_t*>(dsm + r * kRowB + c * 2) = v;
+  }
+  __syncthreads();
+  if (unit >= p.S) return;
+  const int t_beg = unit * kUnit;
+  const int n_tok = ok ? min(kUnit, L + 1 - t_beg) : 0;
   if (n_tok <= 0) {
-    if (tid < G) {
-      float* ml = p.part_ml + ((hq0 + tid) * p.S + split) * 2;
+    if (lane < G) {
+      float* ml = p.part_ml + ((hq0 + lane) * p.S + unit) * 2;
       ml[0] = ok ? -INFINITY : 0.f;
       ml[1] = ok ? 0.f : __int_as_float(0x7fc00000);
     }
     return;
   }
-  for (int i = tid; i < G * kAD; i += 256) q_s[i] = p.q_rot[hq0 * kAD + i];
-  __syncthreads();
-  const __half* kb = p.kc + (((int64_t)slot * p.L_max + t_beg) * p.Hkv + g) * kAD;
-  const __half* vb = p.vc + (((int64_t)slot * p.L_max + t_beg) * p.Hkv + g) * kAD;
+  const uint32_t sbase = qbase + kQB + warp * 2 * kStageB;
+  const int row = lane >> 2, qd = lane & 3;     // fragment row (query head) and quad
+  const bool live = row < G;
   const int64_t tok_stride = (int64_t)p.Hkv * kAD;
-  // scores: 8 lanes per token, lane j of a group reads 16-byte chunks j, j+8, j+16, j+24
-  {
-    const int sub = lane >> 3, j = lane & 7;
-#pragma unroll 2
-    for (int base = warp * 4; base < n_tok; base += 32) {
-      const int i = base + sub;
-      float acc[G];
+  const int64_t base = (((int64_t)slot * p.L_max + t_beg) * p.Hkv + g) * kAD;
+  const __half* kb = p.kc + base;
+  const __half* vb = p.vc + base;
+  const int n_grp = (n_tok + kGrp - 1) / kGrp;
+  const __half* kl = kb + lane * 8;
+  const __half* vl = vb + lane * 8;
+  auto issue = [&](int gi) {
+    const uint32_t st = sbase + (gi & 1) * kStageB + lane * 16;
 #pragma unroll
-      for (int h = 0; h < G; ++h) acc[h] = 0.f;
-      if (i < n_tok) {
-        uint4 raw[4];
+    for (int r = 0; r < kGrp; ++r) {          // 16 rows x 32 chunks of 16 B, K then V
+      const int t = gi * kGrp + r;
+      const bool valid = t < n_tok;
+      const int64_t off = (int64_t)(valid ? t : 0) * tok_stride;
+      cp_async16(st + r * kRowB, kl + off, valid);
+      cp_async16(st + (kGrp + r) * kRowB, vl + off, valid);
+    }
+    cp_async_commit();
+  };
+  float o[32][4];
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-          raw[c] = __ldcs(reinterpret_cast<const uint4*>(kb + i * tok_stride + (c * 8 + j) * 8));
+  for (int j = 0; j < 32; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+  float m = -INFINITY, l = 0.f;
+  issue(0);
+  if (n_grp > 1) issue(1);
+  // ldmatrix row addresses: matrix j = lane / 8, row i = lane % 8
+  const int mj = lane >> 3, mi = lane & 7;
+  const uint32_t k_off = (uint32_t)(((mj >> 1) * 8 + mi) * kRowB + (mj & 1) * 16);
+  const uint32_t q_off = (uint32_t)(mi * kRowB + (mj & 1) * 16);   // x2: lanes 0..15
+  const uint32_t v_off = (uint32_t)(((mj & 1) * 8 + mi) * kRowB + (mj >> 1) * 16);
+  for (int gi = 0; gi < n_grp; ++gi) {
+    if (gi + 1 < n_grp) cp_async_wait<1>(); else cp_async_wait<0>();
+    __syncwarp();
+    const uint32_t kst = sbase + (gi & 1) * kStageB, vst = kst + kGrp * kRowB;
+    float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const __half2* h2 = reinterpret_cast<const __half2*>(&raw[c]);
-          float x[8];
+    for (int kk = 0; kk < 16; ++kk) {
+      uint32_t b[4], a0, a2;
+      ldsm_x2(qbase + q_off + kk * 32, a0, a2);
+      ldsm_x4(kst + k_off + kk * 32, b);
+      mma16816(s0, a0, a2, b[0], b[1]);
+      mma16816(s1, a0, a2, b[2], b[3]);
+    }
+    // this lane's scores: row `row`, tokens 2qd, 2qd+1 (s0) and 8+2qd, 9+2qd (s1)
+    const int t0 = gi * kGrp + 2 * qd;
+    float x[4] = {t0 < n_tok ? s0[0] * p.sl2 : -INFINITY,
+                  t0 + 1 < n_tok ? s0[1] * p.sl2 : -INFINITY,
+                  t0 + 8 < n_tok ? s1[0] * p.sl2 : -INFINITY,
+                  t0 + 9 < n_tok ? s1[1] * p.sl2 : -INFINITY};
+    float mb = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+    mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 1));
+    mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 2));
+    if (mb > m + 8.0f) {               // same for the 4 lanes of a row
+      const float f = ex2(m - mb);
+      m = mb;
+      l *= f;
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = __half22float2(h2[e]);
-            x[2 * e] = f.x;
-            x[2 * e + 1] = f.y;
-          }
-          const int d0 = (c * 8 + j) * 8;
-#pragma unroll
-          for (int h = 0; h < G; ++h) {
-            const float4 qa = *reinterpret_cast<const float4*>(q_s + h * kAD + d0);
-            const float4 qb = *reinterpret_cast<const float4*>(q_s + h * kAD + d0 + 4);
-            acc[h] += x[0] * qa.x + x[1] * qa.y + x[2] * qa.z + x[3] * qa.w + x[4] * qb.x +
-                      x[5] * qb.y + x[6] * qb.z + x[7] * qb.w;
-          }
-        }
-      }
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        acc[h] += __shfl_xor_sync(0xffffffffu, acc[h], 1);
-        acc[h] += __shfl_xor_sync(0xffffffffu, acc[h], 2);
-        acc[h] += __shfl_xor_sync(0xffffffffu, acc[h], 4);
-      }
-      if (j == 0 && i < n_tok) {
-#pragma unroll
-        for (int h = 0; h < G; ++h) p_s[h * kSplit + i] = acc[h] * p.sl2;
+      for (int j = 0; j < 32; ++j) {
+        o[j][0] *= f;
+        o[j][1] *= f;
       }
     }
+    float pv[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      pv[e] = ex2(x[e] - m);
+      l += pv[e];
+    }
+    const uint32_t pa0 = pack_h2(pv[0], pv[1]), pa2 = pack_h2(pv[2], pv[3]);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      uint32_t b[4];
+      ldsm_x4_t(vst + v_off + j * 32, b);
+      mma16816(o[2 * j], pa0, pa2, b[0], b[1]);
+      mma16816(o[2 * j + 1], pa0, pa2, b[2], b[3]);
+    }
+    __syncwarp();
+    if (gi + 2 < n_grp) issue(gi + 2);
   }
-  __syncthreads();
-  // softmax statistics of this split, one warp per query head
-  if (warp < G) {
-    float* ps = p_s + warp * kSplit;
-    float m = -INFINITY;
-    for (int i = lane; i < n_tok; i += 32) m = fmaxf(m, ps[i]);
+  l += __shfl_xor_sync(0xffffffffu, l, 1);
+  l += __shfl_xor_sync(0xffffffffu, l, 2);
+  if (live) {
+    float* po = p.part_o + ((hq0 + row) * p.S + unit) * kAD + 2 * qd;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    float l = 0.f;
-    for (int i = lane; i < n_tok; i += 32) {
-      const float e = ex2(ps[i] - m);
-      ps[i] = e;
-      l += e;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-    if (lane == 0) {
-      float* ml = p.part_ml + ((hq0 + warp) * p.S + split) * 2;
+    for (int j = 0; j < 32; ++j)
+      *reinterpret_cast<float2*>(po + j * 8) = make_float2(o[j][0], o[j][1]);
+    if (qd == 0) {
+      float* ml = p.part_ml + ((hq0 + row) * p.S + unit) * 2;
       ml[0] = m;
       ml[1] = l;
     }
-  }
-  __syncthreads();
-  // P V: a warp per token, lane l owns dims 8l .. 8l + 7
-  float acc[G][8];
-#pragma unroll
-  for (int h = 0; h < G; ++h)
-#pragma unroll
-    for (int e = 0; e < 8; ++e) acc[h][e] = 0.f;
-#pragma unroll 4
-  for (int i = warp; i < n_tok; i += 8) {
-    float x[8];
-    const uint4 raw = __ldcs(reinterpret_cast<const uint4*>(vb + i * tok_stride + lane * 8));
-    const __half2* h2 = reinterpret_cast<const __half2*>(&raw);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 f = __half22float2(h2[e]);
-      x[2 * e] = f.x;
-      x[2 * e + 1] = f.y;
-    }
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      const float pw = p_s[h * kSplit + i];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) acc[h][e] = fmaf(pw, x[e], acc[h][e]);
-    }
-  }
-#pragma unroll
-  for (int h = 0; h < G; ++h) {
-    float* r = red + (warp * G + h) * kAD + lane * 8;
-    *reinterpret_cast<float4*>(r) = make_float4(acc[h][0], acc[h][1], acc[h][2], acc[h][3]);
-    *reinterpret_cast<float4*>(r + 4) = make_float4(acc[h][4], acc[h][5], acc[h][6], acc[h][7]);
-  }
-  __syncthreads();
-  for (int k = tid; k < G * kAD; k += 256) {
-    const int h = k / kAD, d = k % kAD;
-    float sum = 0.f;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) sum += red[(w * G + h) * kAD + d];
-    p.part_o[((hq0 + h) * p.S + split) * kAD + d] = sum;
   }
 }
 
@@ -825,14 +873,14 @@ cudaError_t attention_status_word(const void* workspace, cudaStream_t stream, in
 }
 
 size_t attention_decode_workspace(int N, int Hq, int L_max) {
-  const size_t S = (size_t)((L_max + kSplit - 1) / kSplit);
+  const size_t S = (size_t)((L_max + kUnit - 1) / kUnit);
   return 256 + (size_t)N * Hq * kAD * 4 + (size_t)N * Hq * S * 2 * 4 +
          (size_t)N * Hq * S * kAD * 4;
 }
 
 template <int G>
 cudaError_t launch_split(const DecParams& dp, dim3 grid, cudaStream_t stream) {
-  const size_t smem = (size_t)(G * kAD + G * kSplit + 8 * G * kAD) * sizeof(float);
+  const size_t smem = (size_t)kDecSmem;
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(attn_decode_split_kernel<G>,
@@ -840,7 +888,7 @@ cudaError_t launch_split(const DecParams& dp, dim3 grid, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  attn_decode_split_kernel<G><<<grid, 256, smem, stream>>>(dp);
+  attn_decode_split_kernel<G><<<grid, 32 * kDecWarps, smem, stream>>>(dp);
   return cudaGetLastError();
 }
 
@@ -848,7 +896,7 @@ cudaError_t launch_attention_decode(const AttnDecodeArgs& a) {
   if (a.N == 0) return cudaSuccess;
   uint8_t* ws = static_cast<uint8_t*>(a.workspace);
   int* status = reinterpret_cast<int*>(ws);
-  const int S = (a.L_max + kSplit - 1) / kSplit;
+  const int S = (a.L_max + kUnit - 1) / kUnit;
   float* q_rot = reinterpret_cast<float*>(ws + 256);
   float* part_ml = q_rot + (size_t)a.N * a.Hq * kAD;
   float* part_o = part_ml + (size_t)a.N * a.Hq * S * 2;
@@ -867,7 +915,7 @@ cudaError_t launch_attention_decode(const AttnDecodeArgs& a) {
     attn_decode_prologue_kernel<__nv_bfloat16><<<a.N, 256, 0, a.stream>>>(dp);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const dim3 grid((unsigned)S, (unsigned)a.Hkv, (unsigned)a.N);
+  const dim3 grid((unsigned)((S + kDecWarps - 1) / kDecWarps), (unsigned)a.Hkv, (unsigned)a.N);
   switch (a.Hq / a.Hkv) {
     case 1: e = launch_split<1>(dp, grid, a.stream); break;
     case 2: e = launch_split<2>(dp, grid, a.stream); break;
