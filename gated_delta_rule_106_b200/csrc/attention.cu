@@ -16,11 +16,12 @@
 //    fp16's normal range converts exactly, so P V can take P in fp16 too.
 //  * attn_prefill_kernel: causal flash attention on tcgen05. A CTA owns 64
 //    query tokens of two query heads that share a key-value head (128 rows),
-//    walks 64-key blocks up to the diagonal, S = Q K^T (128 x 64, K = 256) and
-//    O += P V (128 x 256, K = 64), fp16 operands, accumulate in TMEM, the online softmax runs
-//    in 4 warps (one row per thread) and rescales O in TMEM only when a row's
-//    running max grows by more than 2^8; the epilogue divides by the row sum
-//    and applies sigmoid(gate).
+//    walks 64-key blocks up to the diagonal. S = Q K^T (128 x 64, K = 256) and
+//    O += P V (128 x 256, K = 64) take fp16 operands and accumulate in TMEM.
+//    The online softmax runs in 8 warps (two per TMEM lane quadrant, each on
+//    half of a row's columns; row maxima and sums meet in shared memory) and
+//    rescales O in TMEM only when a row's running max grows by more than 2^8;
+//    the epilogue divides by the row sum and applies sigmoid(gate).
 #include <cudaTypedefs.h>
 #include <math.h>
 
@@ -189,9 +190,12 @@ __global__ void __launch_bounds__(256) attn_qk_prologue_kernel(const ProParams p
 constexpr uint32_t A_Q = 0;          // 4 dim chunks x [128 rows][128 B] (16 KB each)
 constexpr uint32_t A_K = 65536;      // 2 slots x 4 dim chunks x [64 keys][128 B]
 constexpr uint32_t A_V = 131072;     // 2 slots x 4 dim chunks x [64 keys][128 B]
-constexpr uint32_t A_P = 196608;     // 2 buffers x [128 rows][64 keys] bf16
-constexpr uint32_t A_BAR = 229376;
+constexpr uint32_t A_P = 196608;     // [128 rows][64 keys] fp16 (P_j is written after
+                                     // O_{j-1} has read P_{j-1})
+constexpr uint32_t A_RED = 212992;   // [2 block parities][2 column halves][128 rows] fp32
+constexpr uint32_t A_BAR = 215040;
 constexpr uint32_t A_SMEM = A_BAR + 256 + 1024;   // + alignment slack
+constexpr int kAttnThreads = 384;    // producer, MMA, TMEM, idle, 8 softmax warps
 
 // TMEM columns: O accumulator [0, 256), S buffers at 256 and 320.
 constexpr uint32_t T_O = 0, T_S = 256;
@@ -249,7 +253,7 @@ __device__ void find_tile(const int32_t* cu, int N, int64_t T, int u, int lane, 
   }
 }
 
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(kAttnThreads, 1)
 attn_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
@@ -271,7 +275,7 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_init(&B.v_full[i], 1);
       mbar_init(&B.s_full[i], 1);
       mbar_init(&B.o_done[i], 1);
-      mbar_init(&B.p_full[i], 128);
+      mbar_init(&B.p_full[i], 256);
     }
     fence_mbar_init();
   }
@@ -367,7 +371,7 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
              mbar_wait_bounded(&B.v_full[sl], par, kAttnLimitNs);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t pb = sa + A_P + sl * 16384, vb = sa + A_V + sl * 32768;
+        const uint32_t pb = sa + A_P, vb = sa + A_V + sl * 32768;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_f16(tmem + T_O, sw128_desc(pb + kk * 32, 16, 1024),
@@ -383,70 +387,84 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (!ok) fail(p);
     } else if (warp >= 4) {
       // ------------------------------------------- softmax, then epilogue
-      const int r = tid - 128;                 // row = TMEM lane
-      const int quad = warp & 3;
+      // Two warps per TMEM lane quadrant: `half` 0 takes score columns 0..31
+      // and output columns 0..127, `half` 1 the rest; they exchange row maxima
+      // (and, at the end, row sums) through shared memory.
+      const int quad = warp & 3, half = (warp - 4) >> 2;
+      const int r = quad * 32 + lane;           // row = TMEM lane
       const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+      float* red = reinterpret_cast<float*>(sm + A_RED);
       const int tq_off = r & 63;               // token offset within the tile
       float m = -INFINITY, l = 0.f;
+      // A wait that runs out clears `ok`; the loop still runs to the end with
+      // no further waits, so that both warps of a pair pass the same named
+      // barriers (what it computes then is discarded: the status word is set).
       bool ok = true;
       for (int j = 0; j < nb; ++j) {
         const int sl = j & 1;
-        ok = mbar_wait_bounded(&B.s_full[sl], (uint32_t)((j >> 1) & 1), kAttnLimitNs);
-        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        if (ok) ok = mbar_wait_bounded(&B.s_full[sl], (uint32_t)((j >> 1) & 1), kAttnLimitNs);
+        ok = __all_sync(0xffffffffu, ok);
         tc_fence_after();
-        uint32_t sr[64];
-        tmem_ld32_nowait(trow + T_S + sl * kBlk, *reinterpret_cast<uint32_t(*)[32]>(sr));
-        tmem_ld32_nowait(trow + T_S + sl * kBlk + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
+        uint32_t sr[32];
+        tmem_ld32_nowait(trow + T_S + sl * kBlk + half * 32, sr);
         tmem_wait_ld();
-        float s[64];
+        float s[32];
         const bool diag = (j == nb - 1);
         float mx = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          s[c] = (diag && c > tq_off) ? -INFINITY : __uint_as_float(sr[c]);
+        for (int c = 0; c < 32; ++c) {
+          s[c] = (diag && half * 32 + c > tq_off) ? -INFINITY : __uint_as_float(sr[c]);
           mx = fmaxf(mx, s[c]);
         }
+        float* rb = red + (j & 1) * 256;
+        rb[half * 128 + r] = mx;
+        bar_sync_n(1 + quad, 64);
+        mx = fmaxf(mx, rb[(1 - half) * 128 + r]);
         const float mb = mx * p.sl2;
+        bool o_prev_done = false;
         if (j == 0) {
           m = mb;
         } else {
           const bool need = mb > m + 8.0f;
-          if (__any_sync(0xffffffffu, need)) {
+          if (__any_sync(0xffffffffu, need) && ok) {   // the partner warp decides the same
             const float m_new = fmaxf(m, mb);
             const float f = ex2(m - m_new);
             m = m_new;
             l *= f;
-            // O holds P_0..P_{j-1} V: wait for the last of them, rescale in place
-            ok = mbar_wait_bounded(&B.o_done[(j - 1) & 1], (uint32_t)(((j - 1) >> 1) & 1),
-                                   kAttnLimitNs);
-            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            // O holds P_0..P_{j-1} V: wait for the last of them, rescale this half
+            ok = __all_sync(0xffffffffu,
+                            mbar_wait_bounded(&B.o_done[(j - 1) & 1],
+                                              (uint32_t)(((j - 1) >> 1) & 1), kAttnLimitNs));
+            o_prev_done = true;
             tc_fence_after();
 #pragma unroll 1
-            for (int cc = 0; cc < kAD / 32; ++cc) {
+            for (int cc = 0; cc < 4 && ok; ++cc) {
               uint32_t ov[32];
-              tmem_ld32_nowait(trow + T_O + cc * 32, ov);
+              const uint32_t ta = trow + T_O + half * 128 + cc * 32;
+              tmem_ld32_nowait(ta, ov);
               tmem_wait_ld();
 #pragma unroll
               for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * f);
-              tmem_st32(trow + T_O + cc * 32, ov);
+              tmem_st32(ta, ov);
             }
             tmem_wait_st();
           }
         }
-        // P_j goes to buffer j & 1, which O_{j-2} read
-        if (j >= 2) {
-          ok = mbar_wait_bounded(&B.o_done[sl], (uint32_t)(((j - 2) >> 1) & 1), kAttnLimitNs);
-          if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-        }
-        uint8_t* prow = sm + A_P + sl * 16384 + r * 128;
+        // one P buffer: O_{j-1} must have read P_{j-1}
+        if (j >= 1 && !o_prev_done && ok)
+          ok = __all_sync(0xffffffffu,
+                          mbar_wait_bounded(&B.o_done[(j - 1) & 1],
+                                            (uint32_t)(((j - 1) >> 1) & 1), kAttnLimitNs));
+        uint8_t* prow = sm + A_P + r * 128;
         float sum = 0.f;
 #pragma unroll
-        for (int c16 = 0; c16 < 8; ++c16) {
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const int c16 = half * 4 + q4;
           uint32_t w[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float a = ex2(fmaf(s[c16 * 8 + 2 * e], p.sl2, -m));
-            const float b = ex2(fmaf(s[c16 * 8 + 2 * e + 1], p.sl2, -m));
+            const float a = ex2(fmaf(s[q4 * 8 + 2 * e], p.sl2, -m));
+            const float b = ex2(fmaf(s[q4 * 8 + 2 * e + 1], p.sl2, -m));
             sum += a + b;
             __half2 h2 = __floats2half2_rn(a, b);
             w[e] = *reinterpret_cast<uint32_t*>(&h2);
@@ -458,6 +476,12 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(&B.p_full[sl]);
+      }
+      {
+        float* rb = red + (nb & 1) * 256;
+        rb[half * 128 + r] = l;
+        bar_sync_n(1 + quad, 64);
+        l += rb[(1 - half) * 128 + r];
       }
       if (ok)
         ok = mbar_wait_bounded(&B.o_done[(nb - 1) & 1], (uint32_t)(((nb - 1) >> 1) & 1),
@@ -471,12 +495,13 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
         const int h = h0 + (r >> 6);
         const bool valid = tq < s1;
         const float inv_l = 1.0f / l;
-        const __nv_bfloat16* gp = p.gate + (int64_t)tq * p.gate_stride + (int64_t)h * kAD;
-        __nv_bfloat16* op = p.o + ((int64_t)tq * p.Hq + h) * kAD;
+        const __nv_bfloat16* gp =
+            p.gate + (int64_t)tq * p.gate_stride + (int64_t)h * kAD + half * 128;
+        __nv_bfloat16* op = p.o + ((int64_t)tq * p.Hq + h) * kAD + half * 128;
 #pragma unroll 1
-        for (int cc = 0; cc < kAD / 32; ++cc) {
+        for (int cc = 0; cc < 4; ++cc) {
           uint32_t ov[32];
-          tmem_ld32_nowait(trow + T_O + cc * 32, ov);
+          tmem_ld32_nowait(trow + T_O + half * 128 + cc * 32, ov);
           tmem_wait_ld();
           if (valid) {
 #pragma unroll
@@ -862,7 +887,7 @@ cudaError_t launch_attention_prefill(const AttnPrefillArgs& a) {
     attr_set = true;
   }
   const unsigned grid = (unsigned)grid_tiles * (unsigned)(a.Hq / 2);
-  attn_prefill_kernel<<<grid, 256, A_SMEM, a.stream>>>(mq, mk, mv, ap);
+  attn_prefill_kernel<<<grid, kAttnThreads, A_SMEM, a.stream>>>(mq, mk, mv, ap);
   return cudaGetLastError();
 }
 
