@@ -452,35 +452,34 @@ class AttentionDecodeWorkload:
     one new token per sequence (q, k, v, gate bf16 N(0, 1)), which appends to
     the caches and advances cache_len."""
 
-    def __init__(self, gdn, dev, seed, steps, kv=(0, A_HKV)):
-        self.gdn = gdn
+    def __init__(self, gdn, dev, seed, steps, kv=(0, A_HKV), n=N_DECODE):
+        self.gdn, self.n = gdn, n
         G = A_HQ // A_HKV
         self.H_kv = kv[1] - kv[0]
         self.H_q = self.H_kv * G
         gen = torch.Generator(device=dev)
         gen.manual_seed(1000 + seed)
-        shape = (N_DECODE, A_LMAX, self.H_kv, A_D)
+        shape = (n, A_LMAX, self.H_kv, A_D)
         self.kc = torch.randn(shape, generator=gen, device=dev, dtype=torch.float16)
         self.vc = torch.randn(shape, generator=gen, device=dev, dtype=torch.float16)
         self.idx = torch.from_numpy(
-            np.random.default_rng(seed).permutation(N_DECODE).astype(np.int32)).to(dev)
-        self.len = torch.full((N_DECODE,), A_CTX, dtype=torch.int32, device=dev)
+            np.random.default_rng(seed).permutation(n).astype(np.int32)).to(dev)
+        self.len = torch.full((n,), A_CTX, dtype=torch.int32, device=dev)
         self.inputs = []
         for s in range(min(steps, 16)):
-            a = gi.attention_inputs(N_DECODE, seed=seed, tag=("attn_decode", s))
+            a = gi.attention_inputs(n, seed=seed, tag=("attn_decode", s))
             self.inputs.append({k: (v[:, kv[0] * G:kv[1] * G] if k in ("q", "gate") else
                                     v[:, kv[0]:kv[1]] if k in ("k", "v") else v)
                                 .contiguous().to(dev) for k, v in a.items()})
-        self.o = torch.empty((N_DECODE, self.H_q, A_D), dtype=torch.bfloat16, device=dev)
-        self.ws = torch.empty(gdn.load().gdn_attention_decode_workspace(N_DECODE, self.H_q,
-                                                                        A_LMAX, A_D),
+        self.o = torch.empty((n, self.H_q, A_D), dtype=torch.bfloat16, device=dev)
+        self.ws = torch.empty(gdn.load().gdn_attention_decode_workspace(n, self.H_q, A_LMAX, A_D),
                               dtype=torch.uint8, device=dev)
 
     def reset(self):
         self.len.fill_(A_CTX)
 
     def bytes_for(self, first_len, steps):
-        return sum(attn_decode_bytes(N_DECODE, first_len + s, self.H_q, self.H_kv)
+        return sum(attn_decode_bytes(self.n, first_len + s, self.H_q, self.H_kv)
                    for s in range(steps))
 
     def step(self, s, ev=None):
@@ -1010,7 +1009,8 @@ def profile_case(args):
             raise SystemExit("attn case runs the T=8192 workload (--t 8192)")
         run = lambda: wl.step(0)
     elif name == "adec":
-        wl = AttentionDecodeWorkload(gdn, dev, 0, 1)
+        # N sequences (--n) of 4096 cached tokens: 64 hold 1.1 GB of cache
+        wl = AttentionDecodeWorkload(gdn, dev, 0, 1, n=N)
         run = lambda: (wl.reset(), wl.step(0))
     else:
         raise SystemExit(f"unknown profile case {name}")

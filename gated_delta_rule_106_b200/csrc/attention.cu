@@ -450,29 +450,30 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
             tmem_wait_st();
           }
         }
+        // P in registers first, so the exponentials overlap O_{j-1}
+        uint32_t w[16];
+        float sum = 0.f;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float a = ex2(fmaf(s[2 * e], p.sl2, -m));
+          const float b = ex2(fmaf(s[2 * e + 1], p.sl2, -m));
+          sum += a + b;
+          __half2 h2 = __floats2half2_rn(a, b);
+          w[e] = *reinterpret_cast<uint32_t*>(&h2);
+        }
+        l += sum;
         // one P buffer: O_{j-1} must have read P_{j-1}
         if (j >= 1 && !o_prev_done && ok)
           ok = __all_sync(0xffffffffu,
                           mbar_wait_bounded(&B.o_done[(j - 1) & 1],
                                             (uint32_t)(((j - 1) >> 1) & 1), kAttnLimitNs));
         uint8_t* prow = sm + A_P + r * 128;
-        float sum = 0.f;
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
           const int c16 = half * 4 + q4;
-          uint32_t w[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float a = ex2(fmaf(s[q4 * 8 + 2 * e], p.sl2, -m));
-            const float b = ex2(fmaf(s[q4 * 8 + 2 * e + 1], p.sl2, -m));
-            sum += a + b;
-            __half2 h2 = __floats2half2_rn(a, b);
-            w[e] = *reinterpret_cast<uint32_t*>(&h2);
-          }
           *reinterpret_cast<uint4*>(prow + ((c16 ^ (r & 7)) << 4)) =
-              make_uint4(w[0], w[1], w[2], w[3]);
+              make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
         }
-        l += sum;
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(&B.p_full[sl]);
