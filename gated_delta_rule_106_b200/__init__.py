@@ -25,6 +25,7 @@ __all__ = ["GDN_BF16", "GDN_F32", "GdnError", "library_path", "load",
            "gdn_chunked_prefill_workspace", "gdn_chunked_prefill_noalloc",
            "gdn_stepwise_prefill", "gdn_decode_layer_step", "gdn_prefill_layer",
            "gdn_chunked_prefill_status", "gdn_set_wait_limit_ns", "GDN_ERR_TIMEOUT",
+           "gdn_prefill_layer_workspace",
            "gdn_decode_step",
            "gdn_gated_rmsnorm", "gdn_status_string", "gdn_version",
            "gdn_attention_prefill", "gdn_attention_decode", "gdn_attention_status",
@@ -66,6 +67,7 @@ _SIGNATURES = {
                                    _int, _f32, _vp, _int, _vp, ctypes.c_size_t,
                                    _vp]),
     "gdn_chunked_prefill_workspace": (ctypes.c_size_t, [_int, _i64, _int, _int]),
+    "gdn_prefill_layer_workspace": (ctypes.c_size_t, [_int, _i64, _int, _int]),
     "gdn_chunked_prefill_status": (_int, [_vp, _vp]),
     "gdn_prefill_layer": (_int, [_vp, _i64, _vp, _int, _vp, _vp, _vp, _vp, _vp, _int, _vp,
                                  _vp, _vp, _int, _i64, _int, _int, _f32, _f32, _vp, _vp,
@@ -276,7 +278,7 @@ def gdn_prefill_layer(x, conv_w, g, beta, cu_seqlens, z, norm_w, *, conv_bias=No
     _expect(y, (T, H_v, HEAD_DIM), "y")
     if y is None:
         y = torch.empty((T, H_v, HEAD_DIM), dtype=y_dtype or torch.bfloat16, device=x.device)
-    need = gdn_chunked_prefill_workspace(N, T, H_k, H_v)
+    need = gdn_prefill_layer_workspace(N, T, H_k, H_v)
     if workspace is None and need:
         workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
@@ -287,6 +289,11 @@ def gdn_prefill_layer(x, conv_w, g, beta, cu_seqlens, z, norm_w, *, conv_bias=No
         _ptr(z), _ptr(norm_w), norm_eps, _ptr(y), _dtype_code(y.dtype), _ptr(workspace),
         ws_bytes, _stream(stream, x.device)))
     return y
+
+
+def gdn_prefill_layer_workspace(N, T_total, H_k=H_K, H_v=H_V) -> int:
+    """Bytes of workspace gdn_prefill_layer needs (chunk ring + q/k conv scratch)."""
+    return int(load().gdn_prefill_layer_workspace(N, T_total, H_k, H_v))
 
 
 def gdn_chunked_prefill_status(workspace=None, stream=None) -> int:

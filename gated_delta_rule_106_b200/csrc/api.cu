@@ -183,7 +183,7 @@ gdn_status gdn_prefill_layer(const void* x, int64_t x_row_stride, const void* co
   if (partial_overlap(conv_state_in, cs_bytes, conv_state_out, cs_bytes))
     return GDN_ERR_INVALID_ARG;
   if (T_total > 0) {
-    if (workspace_bytes < gdn_chunked_prefill_workspace(N, T_total, H_k, H_v) || !workspace)
+    if (workspace_bytes < gdn_prefill_layer_workspace(N, T_total, H_k, H_v) || !workspace)
       return GDN_ERR_INVALID_ARG;
     if (!aligned16(workspace)) return GDN_ERR_MISALIGNED;
   }
@@ -192,6 +192,12 @@ gdn_status gdn_prefill_layer(const void* x, int64_t x_row_stride, const void* co
                           cu_seqlens, N, T_total, H_k, H_v, scale, l2_eps, z, norm_w,
                           norm_eps, y, y_dtype, workspace, workspace_bytes, stream};
   return from_cuda(gdn::launch_prefill_layer(a));
+}
+
+size_t gdn_prefill_layer_workspace(int N, int64_t T_total, int H_k, int H_v) {
+  if (N < 0 || T_total < 0 || H_k <= 0 || H_v <= 0 || H_v % H_k != 0) return 0;
+  if (T_total == 0) return 0;
+  return gdn::prefill_layer_workspace(N, T_total, H_k, H_v);
 }
 
 gdn_status gdn_chunked_prefill_status(const void* workspace, cudaStream_t stream) {

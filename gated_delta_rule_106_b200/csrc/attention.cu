@@ -97,11 +97,9 @@ __device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 u) {
 // rotary on dims [0, R) with the token's (cos, sin) per pair; lane l returns
 // dims 8l .. 8l + 7. `row` is this warp's 256-float staging area.
 template <class Tw>
-__device__ __forceinline__ void norm_rope_row(const __nv_bfloat16* src, const Tw* w,
-                                              const float2* cs, float* row, int R, float eps,
-                                              int lane, float (&x)[8]) {
+__device__ __forceinline__ void norm_rope_vals(const Tw* w, const float2* cs, float* row, int R,
+                                               float eps, int lane, float (&x)[8]) {
   const int half = R >> 1;
-  load8(src + lane * 8, x);
   float ss = 0.f;
 #pragma unroll
   for (int i = 0; i < 8; ++i) ss += x[i] * x[i];
@@ -126,6 +124,13 @@ __device__ __forceinline__ void norm_rope_row(const __nv_bfloat16* src, const Tw
     }
   }
   __syncwarp();
+}
+template <class Tw>
+__device__ __forceinline__ void norm_rope_row(const __nv_bfloat16* src, const Tw* w,
+                                              const float2* cs, float* row, int R, float eps,
+                                              int lane, float (&x)[8]) {
+  load8(src + lane * 8, x);
+  norm_rope_vals(w, cs, row, R, eps, lane, x);
 }
 
 // (cos, sin) of rotary pair i at position pos, angle in fp64.
@@ -162,23 +167,48 @@ __global__ void __launch_bounds__(256) attn_qk_prologue_kernel(const ProParams p
   const int H = p.Hq + p.Hkv;
   const Tw* wq = static_cast<const Tw*>(p.wq);
   const Tw* wk = static_cast<const Tw*>(p.wk);
-  for (int r = warp; r < kProTok * H; r += 8) {
-    const int tt = r / H, hh = r % H;
-    const int64_t t = t0 + tt;
-    if (t >= p.T) break;
-    const bool isq = hh < p.Hq;
-    const __nv_bfloat16* src = isq ? p.q + t * p.q_stride + (int64_t)hh * kAD
-                                   : p.k + t * p.k_stride + (int64_t)(hh - p.Hq) * kAD;
-    float x[8];
-    norm_rope_row(src, isq ? wq : wk, cs[tt], row[warp], p.R, p.eps, lane, x);
-    if (isq) {
-      store8h(p.q_out + (t * p.Hq + hh) * kAD + lane * 8, x);
-    } else {
-      const int g = hh - p.Hq;
-      const int64_t o = (t * p.Hkv + g) * kAD + lane * 8;
-      store8h(p.k_out + o, x);
-      *reinterpret_cast<uint4*>(p.v_out + o) = bf16x8_to_f16x8(
-          *reinterpret_cast<const uint4*>(p.v + t * p.v_stride + (int64_t)g * kAD + lane * 8));
+  // two rows per warp and round, both loaded before either is normed
+  for (int r0 = warp; r0 < kProTok * H; r0 += 16) {
+    uint4 raw[2];
+    bool live[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int r = r0 + 8 * u;
+      const int tt = r / H, hh = r % H;
+      const int64_t t = t0 + tt;
+      live[u] = r < kProTok * H && t < p.T;
+      const __nv_bfloat16* src = hh < p.Hq ? p.q + t * p.q_stride + (int64_t)hh * kAD
+                                           : p.k + t * p.k_stride + (int64_t)(hh - p.Hq) * kAD;
+      raw[u] = live[u] ? __ldg(reinterpret_cast<const uint4*>(src + lane * 8))
+                       : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      if (!live[u]) continue;     // warp-uniform
+      const int r = r0 + 8 * u;
+      const int tt = r / H, hh = r % H;
+      const int64_t t = t0 + tt;
+      const bool isq = hh < p.Hq;
+      float x[8];
+      {
+        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&raw[u]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(b2[e]);
+          x[2 * e] = f.x;
+          x[2 * e + 1] = f.y;
+        }
+      }
+      norm_rope_vals(isq ? wq : wk, cs[tt], row[warp], p.R, p.eps, lane, x);
+      if (isq) {
+        store8h(p.q_out + (t * p.Hq + hh) * kAD + lane * 8, x);
+      } else {
+        const int g = hh - p.Hq;
+        const int64_t o = (t * p.Hkv + g) * kAD + lane * 8;
+        store8h(p.k_out + o, x);
+        *reinterpret_cast<uint4*>(p.v_out + o) = bf16x8_to_f16x8(
+            *reinterpret_cast<const uint4*>(p.v + t * p.v_stride + (int64_t)g * kAD + lane * 8));
+      }
     }
   }
 }

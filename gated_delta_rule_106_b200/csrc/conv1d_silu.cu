@@ -157,7 +157,8 @@ __global__ void __launch_bounds__(kConvThreads)
 conv_silu_kernel(const Tx* __restrict__ x, int64_t xs, const Tw* __restrict__ w,
                  const Tw* __restrict__ bias, int C, int l2c, float eps,
                  const int32_t* __restrict__ cu, int N, int64_t T,
-                 const Tx* __restrict__ cs_in, Tx* cs_out, Ty* __restrict__ y, int64_t ys) {
+                 const Tx* __restrict__ cs_in, int64_t css, Tx* cs_out, Ty* __restrict__ y,
+                 int64_t ys) {
   const int c = (blockIdx.x * kConvThreads + threadIdx.x) * kV;
   const bool active = c < C;
   const bool any_l2 = (int)blockIdx.x * kConvThreads * kV < l2c;
@@ -226,7 +227,7 @@ conv_silu_kernel(const Tx* __restrict__ x, int64_t xs, const Tw* __restrict__ w,
         src[i][k].zero();
         if (active && t < T) {
           if (pr >= st) src[i][k].load(x + pr * xs + c);
-          else if (cs_in) src[i][k].load(cs_in + ((int64_t)n * 3 + (3 + (pr - st))) * C + c);
+          else if (cs_in) src[i][k].load(cs_in + ((int64_t)n * 3 + (3 + (pr - st))) * css + c);
         }
       }
     }
@@ -244,7 +245,7 @@ conv_silu_kernel(const Tx* __restrict__ x, int64_t xs, const Tw* __restrict__ w,
       if constexpr (R == 2) {   // only the short-sequence tiles are given cs_out
         if (cs_out && active && t < T && t == s_hi[i] - 1 && s_lo[i] >= t0 + i0) {
 #pragma unroll
-          for (int r = 0; r < 3; ++r) src[i][r + 1].store(cs_out + ((int64_t)nn[i] * 3 + r) * C + c);
+          for (int r = 0; r < 3; ++r) src[i][r + 1].store(cs_out + ((int64_t)nn[i] * 3 + r) * css + c);
         }
       }
     }
@@ -306,6 +307,7 @@ cudaError_t launch_typed(const ConvArgs& a) {
         static_cast<const Tw*>(a.w), static_cast<const Tw*>(a.bias), a.channels,
         a.l2norm_channels, a.l2_eps, a.cu_seqlens, a.N, a.T_total,
         static_cast<const Tx*>(a.conv_state_in),
+        a.cs_row_stride ? a.cs_row_stride : (int64_t)a.channels,
         fused_rb ? static_cast<Tx*>(a.conv_state_out) : nullptr, static_cast<Ty*>(a.y),
         a.y_row_stride);
     cudaError_t e = cudaGetLastError();

@@ -18,6 +18,9 @@ struct ConvArgs {
   const void* conv_state_in; void* conv_state_out;
   void* y; int64_t y_row_stride; gdn_dtype y_dtype;
   cudaStream_t stream;
+  // elements per row of conv_state_in when it holds more channels than are
+  // convolved here (the layer's q/k-only conv); 0: `channels`
+  int64_t cs_row_stride;
 };
 
 struct RecurArgs {
@@ -109,6 +112,9 @@ cudaError_t launch_conv_state_roll(const void* x, int64_t x_row_stride, gdn_dtyp
                                    int channels, const int32_t* cu, int N, int64_t T,
                                    const void* cs_in, void* cs_out, cudaStream_t stream);
 cudaError_t launch_prefill_layer(const LayerPrefillArgs& a);
+// Workspace of gdn_prefill_layer: the chunk ring plus a bf16 [T, 2 H_k 128]
+// scratch for the q/k conv output.
+size_t prefill_layer_workspace(int N, int64_t T_total, int H_k, int H_v);
 cudaError_t launch_gated_rmsnorm(const NormArgs& a);
 cudaError_t launch_decode_step(const RecurArgs& a);
 cudaError_t launch_decode_layer(const DecodeLayerArgs& a);

@@ -327,25 +327,21 @@ __device__ __forceinline__ void merge_level(const float* Af, float* Tf, float* X
   bar_sync_n(bar, kPipeThreads);
 }
 
-// The layer's prologue inside a prep pipeline: the K, Q (key head kh) and V
-// (value head h) tiles of the chunk at t0 (L tokens of sequence n, which starts
-// at s0) from the pre-conv input: causal conv k=4 (+ bias) over rows t0-3 ..
-// t0+63, SiLU, and the per-token L2 norm of the q and k heads, rounded to bf16
-// into the 128-byte-swizzled [64 tokens][64 channels] blocks that the tensor
-// cores read (the layout the tensor-map loads of the plain path produce). Rows
-// before the sequence start come from the carried conv history (zeros if none);
-// tokens at or past L are written as zeros. Warps 0-5: warp = 2 * part + half,
-// part 0/1/2 = q/k/v, half = tokens 0-31 / 32-63; lane = 4 channels. The
-// arithmetic (and its order) is the conv kernel's, so the tiles hold exactly
-// the values that kernel would store.
+// The layer's prologue inside a prep pipeline: the V tile (value head h) of
+// the chunk at t0 (L tokens of sequence n, which starts at s0) from the
+// pre-conv input: causal conv k=4 (+ bias) over rows t0-3 .. t0+63 and SiLU,
+// rounded to bf16 into the 128-byte-swizzled [64 tokens][64 channels] blocks
+// that the tensor cores read (the layout the tensor-map loads of the plain
+// path produce). The q and k heads, which all value heads of a key head share,
+// come convolved and normed from a separate conv launch into a scratch buffer
+// and load by TMA. Rows before the sequence start come from the carried conv
+// history (zeros if none); tokens at or past L are written as zeros. Warps 0-3
+// take 16 tokens each; lane = 4 channels. The arithmetic (and its order) is the
+// conv kernel's, so the tile holds exactly the values that kernel would store.
 template <class Tw>
-__device__ __forceinline__ void conv_fill(const PcParams& p, uint8_t* kq, uint8_t* vv, int n,
-                                          int kh, int h, int64_t s0, int64_t t0, int L,
-                                          int warp, int lane) {
-  const int part = warp >> 1, half = warp & 1;
-  const int c = (part == 0 ? kh * kHeadDim
-                           : part == 1 ? (p.H_k + kh) * kHeadDim : (2 * p.H_k + h) * kHeadDim) +
-                lane * 4;
+__device__ __forceinline__ void conv_fill_v(const PcParams& p, uint8_t* vv, int n, int h,
+                                            int64_t s0, int64_t t0, int L, int warp, int lane) {
+  const int c = (2 * p.H_k + h) * kHeadDim + lane * 4;
   const Tw* w = static_cast<const Tw*>(p.cw);
   const Tw* bias = static_cast<const Tw*>(p.cb);
   float wt[4][4], b[4];
@@ -370,50 +366,36 @@ __device__ __forceinline__ void conv_fill(const PcParams& p, uint8_t* kq, uint8_
     const float2 bb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
     f[0] = a.x; f[1] = a.y; f[2] = bb.x; f[3] = bb.y;
   };
-  uint8_t* tile = (part == 0 ? kq + 8192 : part == 1 ? kq : vv) +
-                  (lane >> 4) * (part == 2 ? 8192 : 16384);
+  uint8_t* tile = vv + (lane >> 4) * 8192;
   const int chunk = (lane & 15) >> 1, sub = (lane & 1) * 8;
+  const int tb = warp * 16;
+  uint2 raw[19];
+#pragma unroll
+  for (int i = 0; i < 19; ++i) raw[i] = load_row(tb - 3 + i);   // every load issued first
   float h0[4], h1[4], h2[4];
-#pragma unroll 1
-  for (int bt = 0; bt < 2; ++bt) {   // two batches of 16 tokens, every load issued first
-    const int tb = half * 32 + bt * 16;
-    uint2 raw[19];
+  unpack(raw[0], h0);
+  unpack(raw[1], h1);
+  unpack(raw[2], h2);
 #pragma unroll
-    for (int i = 0; i < 19; ++i) raw[i] = (bt == 0 || i >= 3) ? load_row(tb - 3 + i) : make_uint2(0u, 0u);
-    if (bt == 0) {
-      unpack(raw[0], h0);
-      unpack(raw[1], h1);
-      unpack(raw[2], h2);
+  for (int i = 0; i < 16; ++i) {
+    const int tt = tb + i;
+    float h3[4], out[4];
+    unpack(raw[3 + i], h3);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float a = fmaf(wt[e][3], h3[e], fmaf(wt[e][2], h2[e], fmaf(wt[e][1], h1[e], fmaf(wt[e][0], h0[e], b[e]))));
+      out[e] = silu(a);
     }
+    const bool live = tt < L;
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(live ? out[0] : 0.f, live ? out[1] : 0.f);
+    const __nv_bfloat162 hi = __floats2bfloat162_rn(live ? out[2] : 0.f, live ? out[3] : 0.f);
+    *reinterpret_cast<uint2*>(tile + swz(tt, chunk) + sub) =
+        make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int tt = tb + i;
-      float h3[4], out[4], ss = 0.f;
-      unpack(raw[3 + i], h3);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float a = fmaf(wt[e][3], h3[e], fmaf(wt[e][2], h2[e], fmaf(wt[e][1], h1[e], fmaf(wt[e][0], h0[e], b[e]))));
-        out[e] = silu(a);
-        ss = fmaf(out[e], out[e], ss);
-      }
-      if (part < 2) {   // warp-uniform: the warp is one 128-channel q or k head
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-        const float inv = rsqrtf(ss + p.l2_eps);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) out[e] *= inv;
-      }
-      const bool live = tt < L;
-      const __nv_bfloat162 lo = __floats2bfloat162_rn(live ? out[0] : 0.f, live ? out[1] : 0.f);
-      const __nv_bfloat162 hi = __floats2bfloat162_rn(live ? out[2] : 0.f, live ? out[3] : 0.f);
-      *reinterpret_cast<uint2*>(tile + swz(tt, chunk) + sub) =
-          make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        h0[e] = h1[e];
-        h1[e] = h2[e];
-        h2[e] = h3[e];
-      }
+    for (int e = 0; e < 4; ++e) {
+      h0[e] = h1[e];
+      h1[e] = h2[e];
+      h2[e] = h3[e];
     }
   }
 }
@@ -483,7 +465,8 @@ __device__ void prep_role(const PcParams& p, const CUtensorMap* tm_q, const CUte
     } while (x < E && !locate(p, cu, x % p.NS, x / p.NS, &it_, &c_));
     return x;
   };
-  // TMA of item x's K, Q (key head) and V (value head) tiles
+  // TMA of item x's K, Q (key head) and V (value head) tiles; the layer's form
+  // loads K and Q from the q/k conv scratch and convolves V itself
   auto issue_tiles = [&](int x) {
     int it_, c_;
     locate(p, cu, x % p.NS, x / p.NS, &it_, &c_);
@@ -492,12 +475,12 @@ __device__ void prep_role(const PcParams& p, const CUtensorMap* tm_q, const CUte
     seq_chunks(cu, p.T, n_, &a_, &b_);
     const int y = (int)(a_ + (int64_t)c_ * kChunk);
     fence_proxy_async_smem();
-    mbar_arrive_expect_tx(&ss.bar_tma, 6 * 8192);
+    mbar_arrive_expect_tx(&ss.bar_tma, (Fused ? 4 : 6) * 8192);
 #pragma unroll
     for (int b = 0; b < 2; ++b) {
       tma_load_2d(kq + b * 16384, tm_k, kh_ * kHeadDim + b * 64, y, &ss.bar_tma);
       tma_load_2d(kq + b * 16384 + 8192, tm_q, kh_ * kHeadDim + b * 64, y, &ss.bar_tma);
-      tma_load_2d(vv + b * 8192, tm_v, h_ * kHeadDim + b * 64, y, &ss.bar_tma);
+      if (!Fused) tma_load_2d(vv + b * 8192, tm_v, h_ * kHeadDim + b * 64, y, &ss.bar_tma);
     }
   };
   bool pend = false;   // kIssuer: tile loads in flight that no item has waited on
@@ -505,7 +488,7 @@ __device__ void prep_role(const PcParams& p, const CUtensorMap* tm_q, const CUte
   if (ptid == kIssuer) {
     const int x = claim();
     ss.claim = x;
-    if (!Fused && x < E) {
+    if (x < E) {
       issue_tiles(x);
       pend = true;
     }
@@ -534,8 +517,8 @@ __device__ void prep_role(const PcParams& p, const CUtensorMap* tm_q, const CUte
     // (the layer's form waits in warp 6, which has no share of the conv)
     if (ptid == (Fused ? 192 : 0))
       ss.ok = wait_flag_ge(flags_of(p.ws, s) + kRing, r + 1 - kRing, &ctrl[1], p.wait_ns);
-    if constexpr (Fused) {   // the chunk's q, k, v tiles from the pre-conv input
-      if (warp < 6) conv_fill<Tw>(p, kq, vv, n, h / (p.H_v / p.H_k), h, s0, t0, L, warp, lane);
+    if constexpr (Fused) {   // the chunk's v tile from the pre-conv input
+      if (warp < 4) conv_fill_v<Tw>(p, vv, n, h, s0, t0, L, warp, lane);
     }
     if (warp == (Fused ? 7 : 1)) {   // gates: cumulative log-decay and derived vectors
       const Tg* g = static_cast<const Tg*>(p.g);
@@ -573,21 +556,19 @@ __device__ void prep_role(const PcParams& p, const CUtensorMap* tm_q, const CUte
       }
       if (lane == 0) ss.gL = __expf(Gl);
     }
-    if constexpr (Fused) {
-      fence_proxy_async_smem();   // the tensor cores read what the threads wrote
-    } else {
-      ok = mbar_wait_bounded(&ss.bar_tma, tma_par, kLimitNs);
-      if (ok) {   // a phase seen complete by this thread
-        tma_par ^= 1;
-        if (ptid == kIssuer) pend = false;
-      }
+    if constexpr (Fused) fence_proxy_async_smem();   // the tensor cores read the v tile
+    ok = mbar_wait_bounded(&ss.bar_tma, tma_par, kLimitNs);
+    if (ok) {   // a phase seen complete by this thread
+      tma_par ^= 1;
+      if (ptid == kIssuer) pend = false;
     }
     bar_sync_n(bar, kPipeThreads);
     ok = ok && ss.ok;
     if (bar_or_n(bar, kPipeThreads, !ok)) goto fail;
 
-    if (!Fused && L < kChunk) {   // rows past the sequence end hold other data: zero them
-      for (int idx = ptid; idx < 3072; idx += kPipeThreads) {
+    if (L < kChunk) {   // rows past the sequence end hold other data: zero them
+      // (the layer's v tile has them zero already)
+      for (int idx = ptid; idx < (Fused ? 2048 : 3072); idx += kPipeThreads) {
         const int rr = (idx & 511) >> 3;
         if (rr >= L) {
           uint8_t* ptr = idx < 2048 ? kq + idx * 16 : vv + (idx - 2048) * 16;
@@ -753,7 +734,7 @@ __device__ void prep_role(const PcParams& p, const CUtensorMap* tm_q, const CUte
     mma_par ^= 1;
     tc_fence_after();
     // the tiles are free: start the next item's loads
-    if (!Fused && ptid == kIssuer && ok && next < E) {
+    if (ptid == kIssuer && ok && next < E) {
       issue_tiles(next);
       pend = true;
     }
@@ -1416,10 +1397,23 @@ namespace {
 template <class Tg, class To, class Tw>
 cudaError_t launch_layer_typed(const LayerPrefillArgs& a, int nsm, int NS) {
   const int64_t C = 2 * (int64_t)a.H_k * kHeadDim + (int64_t)a.H_v * kHeadDim;
-  CUtensorMap mx, mo;
-  // the q/k/v tensor maps of the plain path are not read in the layer's form;
-  // a valid map over x stands in their place
-  if (!make_map(&mx, a.x, C, a.T_total, a.x_row_stride)) return cudaErrorInvalidValue;
+  const int64_t Cqk = 2 * (int64_t)a.H_k * kHeadDim;
+  // q and k once per key head: conv + SiLU + L2 of the leading 2 H_k heads into
+  // the scratch behind the ring (all value heads of a key head read them)
+  __nv_bfloat16* qk = reinterpret_cast<__nv_bfloat16*>(
+      static_cast<uint8_t*>(a.workspace) + CTRL_BYTES + (size_t)NS * kRing * SLOT_BYTES);
+  ConvArgs ca{a.x, a.x_row_stride, GDN_BF16, a.conv_w, a.w_dtype, a.conv_bias, (int)Cqk,
+              (int)Cqk, a.l2_eps, a.cu_seqlens, a.N, a.T_total, a.conv_state_in, nullptr, qk,
+              Cqk, GDN_BF16, a.stream, C};
+  cudaError_t e = launch_conv1d_silu(ca);
+  if (e != cudaSuccess) return e;
+  CUtensorMap mx, mq, mk, mo;
+  // the v map of the plain path is not read in the layer's form; a valid map
+  // over x stands in its place
+  if (!make_map(&mx, a.x, C, a.T_total, a.x_row_stride) ||
+      !make_map(&mq, qk, (int64_t)a.H_k * kHeadDim, a.T_total, Cqk) ||
+      !make_map(&mk, qk + (int64_t)a.H_k * kHeadDim, (int64_t)a.H_k * kHeadDim, a.T_total, Cqk))
+    return cudaErrorInvalidValue;
   if (sizeof(To) == 2) {
     if (!make_out_map(&mo, a.y, (int64_t)a.H_v * kHeadDim, a.T_total)) return cudaErrorInvalidValue;
   } else {
@@ -1429,7 +1423,7 @@ cudaError_t launch_layer_typed(const LayerPrefillArgs& a, int nsm, int NS) {
              a.scale, a.y, static_cast<uint8_t*>(a.workspace), NS, wait_limit_ns(),
              a.x, a.x_row_stride, a.conv_w, a.conv_bias, a.conv_state_in, (int)C, a.l2_eps,
              a.z, a.norm_w, a.norm_eps};
-  return launch_kernel<Tg, To, true, Tw>(mx, mx, mx, mo, p, nsm, a.workspace, a.stream);
+  return launch_kernel<Tg, To, true, Tw>(mq, mk, mx, mo, p, nsm, a.workspace, a.stream);
 }
 template <class Tg, class To>
 cudaError_t layer_pick_w(const LayerPrefillArgs& a, int nsm, int NS) {
@@ -1444,6 +1438,14 @@ cudaError_t layer_pick_o(const LayerPrefillArgs& a, int nsm, int NS) {
 
 }  // namespace
 
+size_t prefill_layer_workspace(int N, int64_t T_total, int H_k, int H_v) {
+  const int nsm = sm_count();
+  if (nsm < 2) return 0;
+  const int NS = state_ctas((int64_t)N * H_v, H_v, nsm);
+  return CTRL_BYTES + (size_t)NS * kRing * SLOT_BYTES +
+         (size_t)T_total * 2 * H_k * kHeadDim * 2;
+}
+
 cudaError_t launch_prefill_layer(const LayerPrefillArgs& a) {
   if (a.N == 0) return cudaSuccess;
   cudaError_t e = cudaSuccess;
@@ -1451,7 +1453,8 @@ cudaError_t launch_prefill_layer(const LayerPrefillArgs& a) {
     const int nsm = sm_count();
     if (nsm < 2) return cudaErrorInvalidDevice;
     const int NS = state_ctas((int64_t)a.N * a.H_v, a.H_v, nsm);
-    if (a.workspace_bytes < CTRL_BYTES + (size_t)NS * kRing * SLOT_BYTES || !a.workspace)
+    if (a.workspace_bytes < prefill_layer_workspace(a.N, a.T_total, a.H_k, a.H_v) ||
+        !a.workspace)
       return cudaErrorInvalidValue;
     e = a.gate_dtype == GDN_F32 ? layer_pick_o<float>(a, nsm, NS)
                                 : layer_pick_o<__nv_bfloat16>(a, nsm, NS);

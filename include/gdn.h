@@ -150,15 +150,16 @@ gdn_status gdn_chunked_prefill(const void* q, const void* k, const void* v,
 size_t gdn_chunked_prefill_workspace(int N, int64_t T_total, int H_k, int H_v);
 
 /*
- * gdn_prefill_layer -- the whole prefill of the delta-rule layer in one launch
- * of the tensor-core chunk kernel: the causal conv (kernel 4) + SiLU + per-head
- * L2 norm of q and k ([P2 二.1], [P3 架构]) is computed in the kernel's load
- * stage from the pre-conv input, the chunked (chunk = 64) gated delta rule
- * ([P2 二.1]) as in gdn_chunked_prefill, and the gated RMS-norm ([P3 架构]) is
- * applied to each output tile before it leaves. The result equals
+ * gdn_prefill_layer -- the whole prefill of the delta-rule layer as two
+ * launches: the causal conv (kernel 4) + SiLU + per-head L2 norm of the q and k
+ * heads ([P2 二.1], [P3 架构]) once per key head into a workspace scratch, then
+ * the tensor-core chunk kernel, which convolves each value head's v channels in
+ * its load stage from the pre-conv input, runs the chunked (chunk = 64) gated
+ * delta rule ([P2 二.1]) as in gdn_chunked_prefill, and applies the gated
+ * RMS-norm ([P3 架构]) to each output tile before it leaves. The result equals
  * gdn_conv1d_silu -> gdn_chunked_prefill (o in y_dtype) -> gdn_gated_rmsnorm:
  * the conv values enter the chunk products rounded to bf16 exactly as the conv
- * kernel stores them, and the norm reads the outputs in y_dtype. Neither the
+ * kernel stores them, and the norm reads the outputs in y_dtype. Neither the v
  * conv output nor the un-normed output is written to memory. Additional entry
  * point (fused form of the three calls).
  *
@@ -168,13 +169,16 @@ size_t gdn_chunked_prefill_workspace(int N, int64_t T_total, int H_k, int H_v);
  *   conv_state_in   [N, 3, C] bf16 history before each sequence, or NULL (zeros).
  *   conv_state_out  [N, 3, C] bf16 or NULL: each sequence's last three pre-conv
  *                rows (may alias conv_state_in; written after the kernel has read it).
- *   g, beta, state_in, state_out, cu_seqlens, N, T_total, H_k, H_v, scale,
- *                workspace: as gdn_chunked_prefill (gdn_chunked_prefill_workspace).
+ *   g, beta, state_in, state_out, cu_seqlens, N, T_total, H_k, H_v, scale:
+ *                as gdn_chunked_prefill.
+ *   workspace    gdn_prefill_layer_workspace(N, T_total, H_k, H_v) bytes, 16-byte
+ *                aligned: the chunk ring and a bf16 [T_total, 2*H_k*128] q/k scratch.
  *   l2_eps       q/k L2 epsilon: y / sqrt(sum y^2 + l2_eps).
  *   z            [T_total, H_v, 128] bf16 gate; norm_w [128] w_dtype; norm_eps.
  *   y            [T_total, H_v, 128] contiguous, y_dtype: the normed output.
  * A bounded wait that gives up is reported by gdn_chunked_prefill_status.
  */
+size_t gdn_prefill_layer_workspace(int N, int64_t T_total, int H_k, int H_v);
 gdn_status gdn_prefill_layer(const void* x, int64_t x_row_stride, const void* conv_w,
                              gdn_dtype w_dtype, const void* conv_bias,
                              const void* conv_state_in, void* conv_state_out,
