@@ -204,3 +204,44 @@ def test_decode_out_of_range_slot_is_skipped():
     v0 = p["v"][0].double().repeat_interleave(6, dim=0)
     want = v0 / (1 + np.exp(-p["gate"][0].double()))
     assert torch.allclose(o[0].double(), want, rtol=2 ** -7, atol=1e-3)
+
+
+@pytest.mark.parametrize("H_q,H_kv", [(8, 4), (16, 2)])
+def test_other_head_layouts_fp32_weights_far_positions(H_q, H_kv):
+    """GQA groups of 2 and 8 (other instances of the decode kernel), fp32 norm
+    weights, and a prompt continuing 250 000 cached positions (rotary angles in
+    the long-context range); prefill then one decode step from its cache rows."""
+    lens = [90, 33]
+    steps = 1
+    tot = [l + steps for l in lens]
+    cu_full = np.concatenate([[0], np.cumsum(tot)])
+    p = gi.attention_inputs(int(cu_full[-1]), seed=11, H_q=H_q, H_kv=H_kv)
+    wq = p["q_norm_w"].float()
+    wk = p["k_norm_w"].float()
+    pos0 = np.array([250_000, 7], dtype=np.int64)
+    ref, _, kref = oracle.attention(f64(p["q"]), f64(p["k"]), f64(p["v"]), f64(p["gate"]),
+                                    f64(wq), f64(wk), cu_seqlens=cu_full, pos0=pos0)
+    rows = np.concatenate([np.arange(cu_full[n], cu_full[n] + l) for n, l in enumerate(lens)])
+    sub = {k: p[k][rows].to(DEV) for k in ("q", "k", "v", "gate")}
+    cu_p = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32, device=DEV)
+    o, k_rot, v_h = gdn.gdn_attention_prefill(
+        sub["q"], sub["k"], sub["v"], sub["gate"], wq.to(DEV), wk.to(DEV), cu_p,
+        pos0=torch.from_numpy(pos0.astype(np.int32)).to(DEV))
+    torch.cuda.synchronize()
+    check(f64(o), ref[rows])
+    check_cache_rows(k_rot, v_h, kref[rows], p["v"][rows])
+    # one decode step at positions 250 000 + 90 and 7 + 33: positions passed explicitly
+    kc = torch.zeros(2, 256, H_kv, 256, dtype=torch.float16, device=DEV)
+    vc = torch.zeros_like(kc)
+    for n, l in enumerate(lens):
+        s0 = int(cu_p[n])
+        kc[n, :l], vc[n, :l] = k_rot[s0:s0 + l], v_h[s0:s0 + l]
+    new = [int(cu_full[n]) + l for n, l in enumerate(lens)]
+    pos = torch.tensor([[int(pos0[n]) + l for n, l in enumerate(lens)]] * 3, dtype=torch.int32)
+    lens_d = torch.tensor(lens, dtype=torch.int32, device=DEV)
+    od = gdn.gdn_attention_decode(*(p[k][new].to(DEV) for k in ("q", "k", "v", "gate")),
+                                  wq.to(DEV), wk.to(DEV), kc, vc, lens_d,
+                                  positions=pos.to(DEV))
+    torch.cuda.synchronize()
+    check(f64(od), ref[new])
+    assert lens_d.cpu().tolist() == [l + 1 for l in lens]
