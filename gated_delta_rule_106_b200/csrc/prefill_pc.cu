@@ -1149,6 +1149,9 @@ __device__ void state_role(const PcParams& p, const CUtensorMap* tm_o, uint8_t* 
     float ov[16];
     tc_fence_after();
     load_out(((r - 1) & 1) ? ST_D1B : ST_D1A, ov);
+    // an earlier tile store may still read this buffer's stage
+    if (tid == 32) bulk_wait_read_all();
+    __syncthreads();
     uint8_t* lbuf = sm + S_BUF + ((r - 1) & 1) * SL_OPS;
     stage_out(lbuf, ov);
     fence_proxy_async_smem();
