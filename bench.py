@@ -191,6 +191,16 @@ def head_shard(rank, world, H_k=H_K, H_v=H_V):
     return kh0, kh0 + per, kh0 * grp, (kh0 + per) * grp
 
 
+def attn_kv_shard(rank, world, heads):
+    """Key-value heads [g0, g1) of the attention layer on one rank: with the
+    head split (`heads`) and 4 key-value heads dividing over the ranks, each rank
+    takes whole GQA groups (its 6 query heads per key-value head come along);
+    otherwise every rank runs the whole layer."""
+    if heads and A_HKV % world == 0:
+        return rank * A_HKV // world, (rank + 1) * A_HKV // world
+    return 0, A_HKV
+
+
 def shard_channels(kh0, kh1, vh0, vh1, H_k=H_K):
     """Indices of the conv channels (q | k | v of the full layer) that a head
     shard owns, in the order q | k | v."""
@@ -700,9 +710,7 @@ def gpu_arm(args):
         del lc
 
         # global-attention layer; head shards split its 4 key-value heads
-        akv = (0, A_HKV)
-        if heads and A_HKV % world == 0:
-            akv = (rank * A_HKV // world, (rank + 1) * A_HKV // world)
+        akv = attn_kv_shard(rank, world, heads)
         apre = AttentionPrefillWorkload(gdn, dev, seed, akv)
         a_step, a_kern = timed_loop(apre.step, args.steps, args.warmup, barrier)
         a_ms, a_kms = mean_max(a_step), mean_max(a_kern)

@@ -94,7 +94,7 @@ def _shards(rank, world, port, out):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
-        mine = bench.head_shard(rank, world)
+        mine = (bench.head_shard(rank, world), bench.attn_kv_shard(rank, world, True))
         got = [None] * world
         dist.all_gather_object(got, mine)
         out[rank] = got
@@ -114,8 +114,9 @@ def test_head_shards_tile_the_layer_on_gloo_ranks(world):
                        start_method="spawn")
     views = [out[r] for r in range(world)]
     assert all(v == views[0] for v in views)          # every rank sees the same plan
-    kh, vh = [], []
-    for r, (k0, k1, v0, v1) in enumerate(views[0]):
+    kh, vh, gk = [], [], []
+    for r, ((k0, k1, v0, v1), (g0, g1)) in enumerate(views[0]):
+        gk += list(range(g0, g1))
         kh += list(range(k0, k1))
         vh += list(range(v0, v1))
         for j in range(v1 - v0):
@@ -125,5 +126,24 @@ def test_head_shards_tile_the_layer_on_gloo_ranks(world):
         assert ch[0] == 128 * k0 and ch[(k1 - k0) * 128] == 2048 + 128 * k0
         assert ch[2 * (k1 - k0) * 128] == 4096 + 128 * v0
     assert kh == list(range(16)) and vh == list(range(48))
+    assert gk == list(range(4))        # the attention layer's key-value heads tile 0..3
     with pytest.raises(ValueError):
         bench.head_shard(0, 3)
+    assert bench.attn_kv_shard(1, 8, True) == (0, 4)   # 4 heads over 8 ranks: replicas
+    assert bench.attn_kv_shard(1, 2, False) == (0, 4)
+
+
+def test_attention_work_formulas():
+    """The attention legs' algorithmic work, against sums written out:
+    S = Q K^T and O = P V cost 2 * 2 * 256 flops per (query, key) pair and query
+    head over the causal triangle; a decode step reads every cached key and value
+    row once (fp16, 4 key-value heads of 256) plus its own inputs and output."""
+    T = 10
+    pairs = sum(t + 1 for t in range(T))
+    assert bench.attn_prefill_flop(T) == 4 * 256 * 24 * pairs
+    N, L = 3, 7
+    kv = 2 * (L + 1) * 4 * 256 * 2           # keys and values of L cached + 1 new rows
+    new = 2 * 4 * 256 * 2                    # the new key and value written
+    inputs = (24 + 24 + 4 + 4) * 256 * 2     # q, gate, k, v in bf16
+    out = 24 * 256 * 2
+    assert bench.attn_decode_bytes(N, L) == N * (kv + new + inputs + out)
