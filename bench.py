@@ -844,6 +844,9 @@ def gpu_arm(args):
                      "algorithmic_bytes_per_launch": ad_bytes, "kernel_ms": ad_kms},
         "gpu_launches": 3 * DECODE_STEPS}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        acb = attention_cpu_baseline()
+        line["attention_prefill"]["cpu_baseline"] = acb["prefill"]
+        line["attention_decode"]["cpu_baseline"] = acb["decode"]
         cb, ref_out, nheads = cpu_baseline(args.cpu_budget_s)
         line["cpu_baseline"] = cb
         got = pre.out[:, :nheads].double().cpu().numpy()
@@ -907,6 +910,44 @@ def cpu_baseline(budget_s=20.0):
              "sample": f"T={T_PREFILL}: full conv, recurrence + gated RMSNorm for "
                        f"{heads}/{H_V} value heads ({sec:.1f} s), scaled to 48 heads"},
             out, heads)
+
+
+def attention_cpu_baseline(rows=64, dec_seqs=4):
+    """The attention oracle (fp64, host threads over (sequence, query head)) on
+    bounded samples of the two attention legs, scaled to a whole call:
+    prefill -- the last `rows` query rows of the T=8192 prompt (each attends to
+    ~8k keys), scaled by the number of (query, key) pairs of the causal call;
+    decode -- `dec_seqs` sequences whose last row attends to A_CTX + 1 keys, scaled
+    to the leg's 256 sequences."""
+    import oracle
+    f = gi.as_f64
+    out = {}
+    a = gi.attention_inputs(T_PREFILL, seed=0)
+    want = list(range(T_PREFILL - rows, T_PREFILL))
+    t0 = time.perf_counter()
+    oracle.attention(*(f(a[k]) for k in ("q", "k", "v", "gate", "q_norm_w", "k_norm_w")),
+                     rows=want)
+    sec = time.perf_counter() - t0
+    pairs_sampled = sum(t + 1 for t in want)
+    call_s = sec * (T_PREFILL * (T_PREFILL + 1) / 2) / pairs_sampled
+    out["prefill"] = {"value": T_PREFILL / call_s, "unit": "tokens/s",
+                      "cores": min(oracle.hardware_threads(), A_HQ), "kind": "oracle",
+                      "sample": f"T={T_PREFILL}: the last {rows} query rows, all 24 heads "
+                                f"({sec:.1f} s), scaled by (query, key) pairs to the call"}
+    L = A_CTX + 1
+    cu = np.arange(dec_seqs + 1, dtype=np.int64) * L
+    d = gi.attention_inputs(int(cu[-1]), seed=1)
+    t0 = time.perf_counter()
+    oracle.attention(*(f(d[k]) for k in ("q", "k", "v", "gate", "q_norm_w", "k_norm_w")),
+                     cu_seqlens=cu.astype(np.int32), rows=list(cu[1:] - 1))
+    sec = time.perf_counter() - t0
+    step_s = sec * N_DECODE / dec_seqs
+    out["decode"] = {"value": N_DECODE / step_s, "unit": "tokens/s",
+                     "cores": min(oracle.hardware_threads(), dec_seqs * A_HQ), "kind": "oracle",
+                     "sample": f"{dec_seqs} sequences x {L} keys, the last row each ({sec:.1f} s, "
+                               f"q/k norm and rotary of every row included), scaled to "
+                               f"{N_DECODE} sequences"}
+    return out
 
 
 def reference_arm(args):
